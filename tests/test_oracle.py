@@ -1,0 +1,331 @@
+"""Pins for the CPU oracle, against things other than the oracle itself.
+
+Each test checks one oracle function against brute force on tiny inputs, a
+closed form, an invariant, a special case with a known answer, or exact
+rational enumeration, chosen so that a dropped term, a wrong sign or index or
+a transposed operand in the oracle fails at least one of them.
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from oracle import qspec_oracle as orc
+from quantized_speculative_decoding_packed_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+TIE_TOL = 2.0 ** -20
+
+
+def _half_even(fr: Fraction) -> int:
+    """Round an exact rational to the nearest integer, ties to even."""
+    fl = math.floor(fr)
+    d = fr - fl
+    if d > Fraction(1, 2):
+        return fl + 1
+    if d < Fraction(1, 2):
+        return fl
+    return fl if fl % 2 == 0 else fl + 1
+
+
+def _near_half(fr: Fraction) -> bool:
+    d = abs((fr - math.floor(fr)) - Fraction(1, 2))
+    return d <= abs(fr) * TIE_TOL + Fraction(1, 1 << 40)
+
+
+# ---------------------------------------------------------------- weights
+def test_hand_worked_quantization_fixture():
+    fields = {}
+    with open(os.path.join(GOLDEN, "quantize_row_hand.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            key, *vals = line.split()
+            fields[key] = vals
+    group = int(fields["group"][0])
+    w = np.array([float(v) for v in fields["w"]], dtype=np.float32)[None, :]
+    q, s_h = orc.quantize_weights(w, group)
+    assert q[0].tolist() == [int(v) for v in fields["q"]]
+    assert int(s_h.view(np.uint16)[0, 0]) == int(fields["s_h_bits"][0], 16)
+    assert orc.pack_int4(q)[0].tolist() == [int(v, 16) for v in fields["bytes"]]
+
+
+def test_quantize_matches_brute_force_nearest_level():
+    gi = synth.tiny_gemm_inputs()
+    q, s_h = orc.quantize_weights(gi.w, gi.group)
+    n, k = gi.w.shape
+    s_full = np.repeat(s_h.astype(np.float64), gi.group, axis=1)
+    w64 = gi.w.astype(np.float64)
+    levels = np.arange(-8, 8, dtype=np.float64)
+    # float64 differences of these fp32/fp16-derived values are exact
+    err = np.abs(levels[None, None, :] * s_full[:, :, None] - w64[:, :, None])
+    best = err.min(axis=2, keepdims=True)
+    cand = err == best
+    # ties: the even level wins
+    even = (np.arange(-8, 8) % 2 == 0)[None, None, :]
+    pick = np.where(cand.sum(axis=2) > 1,
+                    np.argmax(cand & even, axis=2), np.argmax(cand, axis=2)) - 8
+    mismatch = np.argwhere(pick != q)
+    for (i, j) in mismatch:   # allowed only where the fp32 quotient sits on a half-integer
+        assert _near_half(Fraction(float(gi.w[i, j])) / Fraction(float(s_h[i, j // gi.group])))
+    assert len(mismatch) <= 2
+
+
+def test_quantize_error_bound_and_absmax_maps_to_seven():
+    gi = synth.gemm_inputs("llama2_7b", 1, 512, 1024, 128)
+    q, s_h = orc.quantize_weights(gi.w, 128)
+    deq = orc.dequantize(q, s_h, 128)
+    s_full = np.repeat(s_h.astype(np.float64), 128, axis=1)
+    assert np.all(np.abs(deq - gi.w.astype(np.float64)) <= s_full / 2 * (1 + 2.0 ** -20))
+    wg = gi.w.reshape(512, 8, 128)
+    arg = np.abs(wg).argmax(axis=2)
+    qg = q.reshape(512, 8, 128)
+    top = np.take_along_axis(qg, arg[:, :, None], axis=2)[:, :, 0]
+    sign = np.sign(np.take_along_axis(wg, arg[:, :, None], axis=2)[:, :, 0])
+    assert np.all(top == 7 * sign)
+    assert q.min() >= -8 and q.max() <= 7
+
+
+def test_quantize_exact_grid_reconstructs_and_zero_group():
+    rng = np.random.default_rng(5)
+    c = 2.0 ** -6
+    lv = rng.integers(-7, 8, size=(3, 256))
+    lv[:, 0] = 7
+    lv[:, 128] = -7
+    w = (lv * c).astype(np.float32)
+    w[2, 128:] = 0.0                         # one all-zero group
+    q, s_h = orc.quantize_weights(w, 128)
+    expect = lv.copy()
+    expect[2, 128:] = 0
+    assert np.array_equal(q, expect)
+    assert s_h[0, 0] == np.float16(c) and s_h[1, 1] == np.float16(c)
+    assert s_h[2, 1] == 0
+    assert np.array_equal(orc.dequantize(q, s_h, 128), expect * c)
+
+
+def test_quantize_deterministic_and_pack_roundtrip():
+    gi = synth.tiny_gemm_inputs()
+    q1, s1 = orc.quantize_weights(gi.w, 64)
+    q2, s2 = orc.quantize_weights(gi.w.copy(), 64)
+    b1 = orc.pack_int4(q1)
+    assert np.array_equal(b1, orc.pack_int4(q2)) and np.array_equal(s1.view(np.uint16), s2.view(np.uint16))
+    assert np.array_equal(orc.unpack_int4(b1), q1)
+    # independent byte decode: low nibble = even k, high nibble = odd k
+    b = int(b1[3, 7])
+    lo, hi = b & 15, b >> 4
+    assert (lo - 16 if lo >= 8 else lo) == q1[3, 14]
+    assert (hi - 16 if hi >= 8 else hi) == q1[3, 15]
+
+
+# ---------------------------------------------------------------- activations
+def test_quant_act_brute_force_and_special_rows():
+    gi = synth.tiny_gemm_inputs()
+    x = gi.x.copy()
+    x[3, :] = 0.0                            # zero row
+    q, s_a = orc.quant_act(x)
+    assert s_a[3] == 0 and np.all(q[3] == 0)
+    for m in range(3):
+        a = Fraction(float(np.abs(x[m]).max()))
+        assert s_a[m] == np.float32(float(a) / 7.0) or abs(float(s_a[m]) - float(a) / 7) < 1e-12
+        j = int(np.abs(x[m]).argmax())
+        assert q[m, j] == (7 if x[m, j] > 0 else -7)
+        for k in range(x.shape[1]):
+            exact = Fraction(float(x[m, k])) * 7 / a
+            want = max(-8, min(7, _half_even(exact)))
+            if want != q[m, k]:
+                assert _near_half(exact)
+    assert q.min() >= -8 and q.max() <= 7
+
+
+# ---------------------------------------------------------------- W4A4
+def _decode_nibble(byte_row, k):
+    v = (int(byte_row[k // 2]) >> (4 * (k & 1))) & 15
+    return v - 16 if v >= 8 else v
+
+
+def test_w4a4_accumulators_brute_force():
+    gi = synth.tiny_gemm_inputs()
+    qw, s_h = orc.quantize_weights(gi.w, gi.group)
+    packed = orc.pack_int4(qw)
+    qa, s_a = orc.quant_act(gi.x)
+    y, acc = orc.gemm_w4a4(gi.x, qw, s_h, gi.group, return_acc=True)
+    m_, k_ = qa.shape
+    n_ = qw.shape[0]
+    g_ = k_ // gi.group
+    rows = [[_decode_nibble(packed[n], k) for k in range(k_)] for n in range(n_)]
+    qa_l = qa.tolist()
+    for m in range(m_):
+        for n in range(n_):
+            for g in range(g_):
+                s = 0
+                for k in range(g * gi.group, (g + 1) * gi.group):
+                    s += qa_l[m][k] * rows[n][k]
+                assert acc[m, n, g] == s
+    assert np.abs(acc).max() <= 64 * gi.group
+    # closed form: the grouped rescale equals the plain product of the two dequantized operands
+    deq_a = qa.astype(np.float64) * s_a.astype(np.float64)[:, None]
+    plain = deq_a @ orc.dequantize(qw, s_h, gi.group).T
+    assert np.allclose(y, plain, rtol=1e-12, atol=1e-12 * np.abs(plain).max())
+    # exact rational value of a few outputs
+    for (m, n) in [(0, 0), (1, 77), (3, 255)]:
+        ex = Fraction(float(s_a[m])) * sum(Fraction(float(s_h[n, g])) * int(acc[m, n, g]) for g in range(g_))
+        assert abs(float(ex) - y[m, n]) <= 1e-14 * max(1.0, abs(float(ex)))
+
+
+# ---------------------------------------------------------------- W4A16
+def test_w4a16_exact_rational_and_integer_special_case():
+    gi = synth.tiny_gemm_inputs()
+    qw, s_h = orc.quantize_weights(gi.w, gi.group)
+    y = orc.gemm_w4a16(gi.x, qw, s_h, gi.group)
+    x = gi.x
+    for (m, n) in [(0, 0), (2, 31), (3, 200), (1, 255)]:
+        ex = sum(Fraction(float(x[m, k])) * int(qw[n, k]) * Fraction(float(s_h[n, k // gi.group]))
+                 for k in range(x.shape[1]))
+        assert abs(float(ex) - y[m, n]) <= 1e-12 * float(sum(abs(Fraction(float(x[m, k])) * int(qw[n, k]) * Fraction(float(s_h[n, k // gi.group]))) for k in range(x.shape[1])))
+    # scale exactly 1: integer weights with absmax 7 in every group, integer activations
+    rng = np.random.default_rng(11)
+    lv = rng.integers(-7, 8, size=(32, 256))
+    lv[:, ::64] = 7
+    q1, s1 = orc.quantize_weights(lv.astype(np.float32), 64)
+    assert np.all(s1 == 1) and np.array_equal(q1, lv)
+    xi = rng.integers(-20, 21, size=(5, 256)).astype(np.float32)
+    assert np.array_equal(orc.gemm_w4a16(xi, q1, s1, 64), xi.astype(np.int64) @ lv.T)
+
+
+# ---------------------------------------------------------------- accept / resample
+def _exact_inverse_cdf(r, u):
+    fr = [Fraction(float(v)) for v in r]
+    total = sum(fr)
+    t = Fraction(float(u)) * total
+    c = Fraction(0)
+    for j, v in enumerate(fr):
+        c += v
+        if c > t:
+            return j
+    return len(fr) - 1
+
+
+def test_fixed_point_sampler_matches_exact_inverse_cdf():
+    rng = np.random.default_rng(3)
+    for trial in range(40):
+        v = int(rng.integers(2, 300))
+        r = rng.random(v).astype(np.float32) ** 3
+        r[rng.random(v) < 0.3] = 0.0
+        if r.sum() == 0:
+            r[0] = 1.0
+        r = (r / np.float32(r.sum() * 1.0001)).astype(np.float32)   # a probability row
+        u = np.float32(rng.random())
+        assert orc.sample_fixed_point(r, u) == _exact_inverse_cdf(r, u)
+    # u = 0 picks the first token with positive weight; u just below 1 the last one
+    r = np.array([0, 0, 0.25, 0.5, 0, 0.25, 0], np.float32)
+    assert orc.sample_fixed_point(r, np.float32(0.0)) == 2
+    assert orc.sample_fixed_point(r, np.float32(1 - 2 ** -24)) == 5
+    assert orc.sample_fixed_point(np.zeros(4, np.float32), np.float32(0.3)) is None
+
+
+def test_accept_p_equals_q_accepts_everything():
+    ai = synth.tiny_accept_inputs()
+    q = ai.p[:, :4, :].copy()
+    n, tok = orc.spec_accept(ai.p, q, ai.draft, ai.u_acc, ai.u_res)
+    assert np.all(n == 4)
+    for b in range(2):
+        assert tok[b, :4].tolist() == ai.draft[b].tolist()
+        assert tok[b, 4] == _exact_inverse_cdf(ai.p[b, 4], ai.u_res[b])
+
+
+def test_accept_zero_target_probability_rejects():
+    ai = synth.tiny_accept_inputs()
+    p = ai.p.copy()
+    q = ai.p[:, :4, :].copy()                # everything would be accepted ...
+    x = ai.draft[0, 2]
+    p[0, 2, x] = 0.0                         # ... except position 2 of sequence 0
+    n, tok = orc.spec_accept(p, q, ai.draft, ai.u_acc, ai.u_res)
+    assert n[0] == 2 and n[1] == 4
+    r = np.maximum(np.float32(0), p[0, 2] - q[0, 2])
+    assert not r.any()                       # residual is empty here: the draw falls back to p_n
+    assert tok[0, 2] == _exact_inverse_cdf(p[0, 2], ai.u_res[0]) and tok[0, 2] != x
+    assert tok[0, 3] == -1 and tok[0, 4] == -1
+    assert tok[0, :2].tolist() == ai.draft[0, :2].tolist()
+
+
+def test_accept_one_hot_draft():
+    v = 6
+    p = np.array([[[0.1, 0.2, 0.3, 0.15, 0.05, 0.2], [1 / 6] * 6]], np.float32)
+    q = np.zeros((1, 1, v), np.float32)
+    q[0, 0, 2] = 1.0
+    draft = np.array([[2]], np.int32)
+    for u, acc in [(0.29, True), (0.3, False), (0.31, False), (0.0, True)]:
+        n, tok = orc.spec_accept(p, q, draft, np.array([[u]], np.float32), np.array([0.5], np.float32))
+        assert (n[0] == 1) == (u < np.float32(0.3))
+        if not acc:
+            # residual is p with token 2 removed
+            r = p[0, 0].copy()
+            r[2] = 0
+            assert tok[0, 0] == _exact_inverse_cdf(r, np.float32(0.5)) and tok[0, 0] != 2
+
+
+def test_rule_reproduces_target_exactly_in_rationals():
+    """Exact enumeration (no oracle code): accept-or-resample emits y with probability p(y)."""
+    for p, q in [([Fraction(1, 2), Fraction(1, 4), Fraction(1, 8), Fraction(1, 8)],
+                  [Fraction(1, 10), Fraction(6, 10), Fraction(2, 10), Fraction(1, 10)]),
+                 ([Fraction(1, 3), Fraction(1, 3), Fraction(1, 3), 0, 0],
+                  [Fraction(1, 5)] * 5)]:
+        res = [max(Fraction(0), a - b) for a, b in zip(p, q)]
+        z = sum(res)
+        beta = sum(min(a, b) for a, b in zip(p, q))
+        for y in range(len(p)):
+            acc_y = q[y] * (min(Fraction(1), p[y] / q[y]) if q[y] > 0 else 0)
+            assert acc_y + (1 - beta) * res[y] / z == p[y]
+
+
+def test_oracle_emitted_distribution_matches_target_on_uniform_grids():
+    """The oracle's accept + resample, driven over uniform grids, reproduces p within the grid error."""
+    p = np.array([[[0.5, 0.25, 0.125, 0.125], [0.25] * 4]], np.float32)
+    q = np.array([[[0.1, 0.6, 0.2, 0.1]]], np.float32)
+    k1 = 1 << 12
+    grid = ((np.arange(k1) + 0.5) / k1).astype(np.float32)
+    emitted = np.zeros(4)
+    for x in range(4):
+        d = np.full((k1, 1), x, np.int32)
+        acc = orc.accept_mask(np.repeat(p, k1, 0), np.repeat(q, k1, 0), d, grid[:, None])
+        frac_acc = acc.mean()
+        res = np.zeros(4)
+        r = np.maximum(np.float32(0), p[0, 0] - q[0, 0])
+        for u in grid[::16]:
+            res[orc.sample_fixed_point(r, u)] += 1
+        res /= res.sum()
+        emitted += q[0, 0, x] * (frac_acc * np.eye(4)[x] + (1 - frac_acc) * res)
+    assert np.allclose(emitted, p[0, 0], atol=4 * 16 / k1)
+    # and the full routine over a coarse joint grid
+    kk = 32
+    g = ((np.arange(kk) + 0.5) / kk).astype(np.float32)
+    ua = np.repeat(g, kk)[:, None]
+    ur = np.tile(g, kk)
+    counts = np.zeros(4)
+    for x in range(4):
+        d = np.full((kk * kk, 1), x, np.int32)
+        _, tok = orc.spec_accept(np.repeat(p, kk * kk, 0), np.repeat(q, kk * kk, 0), d, ua, ur)
+        counts += q[0, 0, x] * np.bincount(tok[:, 0], minlength=4) / (kk * kk)
+    assert np.allclose(counts, p[0, 0], atol=4 / kk + 1e-6)
+
+
+def test_mean_acceptance_matches_overlap_closed_form():
+    ai = synth.big_accept_inputs(0.5, batch=64, gamma=5, vocab=8192)
+    acc = orc.accept_mask(ai.p, ai.q, ai.draft, ai.u_acc)
+    alpha = np.minimum(ai.p[:, :5, :].astype(np.float64), ai.q.astype(np.float64)).sum(axis=2)
+    se = math.sqrt(float(np.mean(alpha * (1 - alpha))) / acc.size)
+    assert abs(acc.mean() - alpha.mean()) < 4 * se + 1e-9
+
+
+def test_accept_outputs_shape_and_prefix():
+    ai = synth.tiny_accept_inputs()
+    n, tok = orc.spec_accept(ai.p, ai.q, ai.draft, ai.u_acc, ai.u_res)
+    mask = orc.accept_mask(ai.p, ai.q, ai.draft, ai.u_acc)
+    for b in range(2):
+        first = int(np.argmin(mask[b])) if not mask[b].all() else 4
+        assert n[b] == first
+        assert tok[b, :first].tolist() == ai.draft[b, :first].tolist()
+        assert 0 <= tok[b, first] < 32
+        assert np.all(tok[b, first + 1:] == -1)
