@@ -1,0 +1,173 @@
+/*
+ * qspec.h - C ABI of the shared-INT4 QSpec hot path on B200 (sm_100a).
+ *
+ * The method (QSpec: Speculative Decoding with Complementary Quantization
+ * Schemes, abstract) serves ONE set of 4-bit weights through two linear-layer
+ * modes: a W4A4 drafting mode (weights and activations both 4-bit) and a
+ * W4A16 verifying mode (4-bit weights, 16-bit activations).  The explainer
+ * essay on the same paper (paragraph 4) states that the two modes share the
+ * underlying quantized weights and differ in how activations are handled;
+ * every GEMM entry point below therefore takes the same `wq`/`ws` buffers.
+ * Each draft-verify round ends with the speculative accept / residual
+ * resample step (SpecQuant review, paragraph 5: "the usual Leviathan rule").
+ *
+ * Conventions shared by all entry points
+ *  - Pointers are DEVICE pointers owned by the caller unless stated
+ *    otherwise.  The library never allocates or frees device memory; scratch
+ *    space is the caller's `workspace`, sized with qspec_workspace_size().
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream) and returns after enqueueing its kernels.
+ *  - 16-bit floating point buffers are passed as uint16_t bit patterns:
+ *    bf16 for activations, IEEE fp16 for weight scales.
+ *  - Arguments are validated on the host before anything is launched; a
+ *    failed check returns a status and launches nothing.  Launch failures
+ *    return QSPEC_ERR_CUDA.  Faults seen by a kernel (a bounded wait that ran
+ *    out, a draft token outside the vocabulary) are recorded in a status
+ *    word at the start of the workspace; read it with
+ *    qspec_workspace_status().
+ *  - Device buffers read by TMA (x, wq, and the workspace) must be 16-byte
+ *    aligned; all buffers must be at least 16-byte aligned.
+ *  - The device must be compute capability 10.0 (B200, sm_100a), else
+ *    QSPEC_ERR_UNSUPPORTED_DEVICE.
+ *  - Inputs must be finite.
+ */
+#ifndef QSPEC_H_
+#define QSPEC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum qspec_status {
+  QSPEC_OK = 0,
+  QSPEC_ERR_INVALID_ARG = 1,        /* a size, alignment or pointer check failed */
+  QSPEC_ERR_UNSUPPORTED_DEVICE = 2, /* current device is not sm_100 */
+  QSPEC_ERR_CUDA = 3,               /* a CUDA runtime call or launch failed */
+  QSPEC_ERR_WORKSPACE_TOO_SMALL = 4,
+  QSPEC_ERR_TIMEOUT = 5,            /* a kernel's bounded wait ran out (device status) */
+  QSPEC_ERR_BAD_INPUT = 6           /* a kernel saw invalid data, e.g. a draft token >= vocab */
+} qspec_status;
+
+/* Operation ids for qspec_workspace_size(). */
+enum {
+  QSPEC_OP_QUANTIZE_WEIGHTS = 0,
+  QSPEC_OP_QUANT_ACT = 1,
+  QSPEC_OP_GEMM_W4A4 = 2,
+  QSPEC_OP_GEMM_W4A16 = 3,
+  QSPEC_OP_SPEC_ACCEPT = 4
+};
+
+/*
+ * Offline weight quantization, run once per model (QSpec abstract: both
+ * stages reuse the same quantized weights, "without retraining").
+ * Recipe (the pages give none; this is the library's definition): for output
+ * channel n and group g of `group` consecutive input channels,
+ *   s = max|w| / 7 (fp32), s_h = fp16(s) (round to nearest even),
+ *   q = clamp(rint(w / s_h), -8, 7) (fp32 division, ties to even; q = 0 if s_h = 0).
+ *  w   [n][k] fp32, row-major.
+ *  wq  [n][k/2] bytes out: byte j of a row holds k = 2j in its low nibble and
+ *      k = 2j+1 in its high nibble, two's complement.
+ *  ws  [n][k/group] fp16 bit patterns out.
+ * Requires n >= 1, group in {64, 128}, k a multiple of group.
+ */
+qspec_status qspec_quantize_weights(const float* w, int64_t n, int64_t k, int32_t group,
+                                    uint8_t* wq, uint16_t* ws, void* stream);
+
+/*
+ * Per-token activation quantization of the W4A4 drafting mode (explainer
+ * essay, paragraph 2: W4A4 quantizes both weights and activations).
+ * For each row m: a = max_k |x|, s_a = a / 7, inv = 7 / a (fp32 divisions),
+ *   q = clamp(rint(x * inv), -8, 7) (product rounded to fp32); a zero row gives 0.
+ *  x   [m][k] bf16.
+ *  xq  [m][k/2] bytes out, same nibble order as wq.
+ *  xs  [m] fp32 out: s_a.
+ * Requires m >= 1, k >= 8, k a multiple of 8.
+ */
+qspec_status qspec_quant_act(const uint16_t* x, int64_t m, int64_t k, uint8_t* xq, float* xs,
+                             void* stream);
+
+/*
+ * W4A4 drafting GEMM: y = x . deq(wq, ws)^T with the activations quantized
+ * per token first (QSpec abstract: "low-precision joint quantization for
+ * fast drafting").  Per group g, acc[m][n][g] = sum_{k in g} qa[m][k] qw[n][k]
+ * is computed exactly on the int8 tensor cores (int32), and
+ *   y[m][n] = s_a[m] * sum_g s_h[n][g] * acc[m][n][g]   (fp32 arithmetic).
+ *  x        [m][k] bf16.
+ *  wq, ws   as produced by qspec_quantize_weights for [n][k] weights.
+ *  y        [m][n] fp32 out.
+ *  workspace  device scratch of at least
+ *           qspec_workspace_size(QSPEC_OP_GEMM_W4A4, m, n, k, group, 0, 0, 0)
+ *           bytes; it must be zero-filled before its first use, and every
+ *           call that completes leaves it ready for the next one.
+ *  dbg_acc  optional (may be NULL): [m][n][k/group] int32 out, the per-group
+ *           integer accumulators.
+ * Requires m, n >= 1, group in {64, 128}, k a multiple of 128.
+ */
+qspec_status qspec_gemm_w4a4(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
+                             const uint16_t* ws, int64_t n, int32_t group, float* y,
+                             void* workspace, size_t workspace_bytes, int32_t* dbg_acc,
+                             void* stream);
+
+/*
+ * W4A16 verifying GEMM: y = x . deq(wq, ws)^T with bf16 activations and the
+ * same packed weights as the drafting mode (QSpec abstract: "high-precision
+ * weight-only quantization for accurate verification").  deq = q * s_h is
+ * applied exactly: the integer codes enter the bf16 tensor cores unchanged
+ * and each group's fp32 partial sum is scaled by s_h[n][g].
+ *  Arguments as for qspec_gemm_w4a4 (workspace sized for QSPEC_OP_GEMM_W4A16).
+ */
+qspec_status qspec_gemm_w4a16(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
+                              const uint16_t* ws, int64_t n, int32_t group, float* y,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Speculative accept / residual resample for a batch of sequences (SpecQuant
+ * review, paragraph 5; the rule of "Fast Inference from Transformers via
+ * Speculative Decoding" and "Accelerating Large Language Model Decoding with
+ * Speculative Sampling").  For sequence b and draft position i < gamma with
+ * draft token x:  accept iff u_acc[b][i] * q[b][i][x] < p[b][i][x] (exact).
+ * n = first rejected position, or gamma.  The new token is drawn from
+ * r = max(0, p[b][n] - q[b][n]) if n < gamma, else from p[b][gamma], by the
+ * fixed-point inverse CDF F_j = floor(r_j 2^62), C_j = sum_{i<=j} F_i,
+ * token = min{ j : C_j > floor(u_res[b] * C_{V-1}) }; if C_{V-1} = 0 the draw
+ * uses p[b][n] instead, and the token is -1 if that row is empty as well.
+ *  p          [batch][gamma+1][vocab] fp32 target probabilities (rows sum to <= ~1).
+ *  q          [batch][gamma][vocab] fp32 draft probabilities.
+ *  draft      [batch][gamma] int32 draft tokens.
+ *  u_acc      [batch][gamma] fp32 uniforms in [0, 1).
+ *  u_res      [batch] fp32 uniforms in [0, 1).
+ *  n_accepted [batch] int32 out.
+ *  tokens     [batch][gamma+1] int32 out: accepted draft tokens, then the new
+ *             token, then -1 padding.
+ *  workspace  optional (NULL or >= qspec_workspace_size(QSPEC_OP_SPEC_ACCEPT,...)
+ *             bytes): receives the device status word.  A draft token outside
+ *             [0, vocab) is treated as rejected and reported as BAD_INPUT there.
+ * Requires 1 <= batch <= 65535, 1 <= gamma <= 16, 4 <= vocab <= 409600, vocab % 4 == 0.
+ */
+qspec_status qspec_spec_accept(const float* p, const float* q, const int32_t* draft,
+                               const float* u_acc, const float* u_res, int32_t batch,
+                               int32_t gamma, int32_t vocab, int32_t* n_accepted,
+                               int32_t* tokens, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* Bytes of workspace an operation needs on the current device (0 = none).
+ * Unused size arguments are ignored.  Returns 0 for invalid arguments too. */
+size_t qspec_workspace_size(int32_t op, int64_t m, int64_t n, int64_t k, int32_t group,
+                            int32_t batch, int32_t gamma, int32_t vocab);
+
+/* Synchronizes `stream`, reads the device status word at the start of
+ * `workspace`, clears it, and returns QSPEC_OK, QSPEC_ERR_TIMEOUT or
+ * QSPEC_ERR_BAD_INPUT (or QSPEC_ERR_CUDA if the read itself failed). */
+qspec_status qspec_workspace_status(void* workspace, void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* qspec_status_string(qspec_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QSPEC_H_ */

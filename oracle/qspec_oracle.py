@@ -166,7 +166,7 @@ def gemm_w4a16(x: np.ndarray, qw: np.ndarray, s_h: np.ndarray, group: int) -> np
 # summation order gives the same token:
 #   F_j = floor(r_j * 2^62),  C_j = sum_{i<=j} F_i,  S = C_{V-1},
 #   T = floor(u_res * S)  (exact product),  token = min{ j : C_j > T }.
-# If S == 0 the draw falls back to p_n.
+# If S == 0 the draw falls back to p_n (and gives -1 if that row is empty too).
 # --------------------------------------------------------------------------
 def accept_mask(p: np.ndarray, q: np.ndarray, draft: np.ndarray, u_acc: np.ndarray) -> np.ndarray:
     """Boolean [B][gamma]: the ratio test at every draft position."""
@@ -226,6 +226,8 @@ def spec_accept(p: np.ndarray, q: np.ndarray, draft: np.ndarray, u_acc: np.ndarr
         tok = sample_fixed_point(r, u_res[b])
         if tok is None:
             tok = sample_fixed_point(p[b, n], u_res[b])
+        if tok is None:          # both rows empty (degenerate input): no token
+            tok = -1
         n_acc[b] = n
         tokens[b, :n] = draft[b, :n]
         tokens[b, n] = tok

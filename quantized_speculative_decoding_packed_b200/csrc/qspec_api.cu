@@ -1,0 +1,374 @@
+// C ABI of the shared-INT4 QSpec hot path (declared in include/qspec.h).
+//
+// Host side only: argument validation, workspace layout, TMA descriptors and
+// kernel launches.  Every step of the computation runs in the kernels of
+// quantize.cuh, gemm.cuh and accept.cuh; there is no host fallback.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "accept.cuh"
+#include "gemm.cuh"
+#include "qspec.h"
+#include "quantize.cuh"
+
+namespace qspec {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool probed = false;
+  bool supported = false;
+  int sm_count = 0;
+};
+
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_mutex;
+
+qspec_status current_device(int* dev_out, DeviceInfo* info_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return QSPEC_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return QSPEC_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& d = g_devices[dev];
+  if (!d.probed) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return QSPEC_ERR_CUDA;
+    }
+    d.supported = (major == 10 && minor == 0);
+    d.sm_count = sms;
+    d.probed = true;
+  }
+  if (dev_out) *dev_out = dev;
+  if (info_out) *info_out = d;
+  return d.supported ? QSPEC_OK : QSPEC_ERR_UNSUPPORTED_DEVICE;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ---------------------------------------------------------------- TMA descriptors
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess) {
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    } else {
+      cudaGetLastError();
+    }
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [rows][cols] of `elem` bytes, box [box_rows][box_cols].
+bool make_tmap(CUtensorMap* map, CUtensorMapDataType dtype, size_t elem, const void* base,
+               uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols,
+               CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * elem};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- GEMM planning
+struct GemmPlan {
+  int mt = 16;               // token tile (MMA N)
+  int m_tiles = 1, n_tiles = 1, ku = 1;
+  long long units = 0;
+  int grid = 1;
+  size_t off_counters = 0, off_partials = 0, off_xq = 0, off_sa = 0, total = 0;
+};
+
+int pick_mt(int64_t m) {
+  if (m > 96) return 128;
+  const int r = static_cast<int>((m + 15) / 16) * 16;
+  return r;   // 16, 32, 48, 64, 80, 96
+}
+
+bool gemm_shape_ok(int64_t m, int64_t n, int64_t k, int32_t group) {
+  if (m < 1 || n < 1 || k < 128 || (k % 128) != 0) return false;
+  if (group != 64 && group != 128) return false;
+  if (m > (1ll << 30) || n > (1ll << 30) || k > (1ll << 30)) return false;
+  return true;
+}
+
+GemmPlan plan_gemm(bool int8_mode, int64_t m, int64_t n, int64_t k, int sm_count) {
+  GemmPlan p;
+  p.mt = pick_mt(m);
+  p.m_tiles = static_cast<int>((m + p.mt - 1) / p.mt);
+  p.n_tiles = static_cast<int>((n + kTileN - 1) / kTileN);
+  p.ku = static_cast<int>(k / kUnitK);
+  p.units = static_cast<long long>(p.m_tiles) * p.n_tiles * p.ku;
+  p.grid = static_cast<int>(p.units < sm_count ? p.units : sm_count);
+  size_t off = 256;                                  // status word(s)
+  p.off_counters = off;
+  off += round_up(static_cast<size_t>(p.m_tiles) * p.n_tiles * 4, 256);
+  p.off_partials = off;
+  off += round_up(static_cast<size_t>(2) * p.grid * p.mt * kTileN * 4, 256);
+  if (int8_mode) {
+    p.off_xq = off;
+    off += round_up(static_cast<size_t>(m) * k, 256);
+    p.off_sa = off;
+    off += round_up(static_cast<size_t>(m) * 4, 256);
+  }
+  p.total = off;
+  return p;
+}
+
+template <bool kInt8, int MT>
+qspec_status launch_qgemm_t(const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a,
+                            int grid, int dev, cudaStream_t stream) {
+  using C = GemmCfg<kInt8, MT>;
+  static bool attr_set[kMaxDevices] = {};
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(qgemm_kernel<kInt8, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes) != cudaSuccess) {
+      cudaGetLastError();
+      return QSPEC_ERR_CUDA;
+    }
+    attr_set[dev] = true;
+  }
+  qgemm_kernel<kInt8, MT><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tw, tx, a);
+  return cudaGetLastError() == cudaSuccess ? QSPEC_OK : QSPEC_ERR_CUDA;
+}
+
+template <bool kInt8>
+qspec_status launch_qgemm(int mt, const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a,
+                          int grid, int dev, cudaStream_t stream) {
+  switch (mt) {
+    case 16: return launch_qgemm_t<kInt8, 16>(tw, tx, a, grid, dev, stream);
+    case 32: return launch_qgemm_t<kInt8, 32>(tw, tx, a, grid, dev, stream);
+    case 48: return launch_qgemm_t<kInt8, 48>(tw, tx, a, grid, dev, stream);
+    case 64: return launch_qgemm_t<kInt8, 64>(tw, tx, a, grid, dev, stream);
+    case 80: return launch_qgemm_t<kInt8, 80>(tw, tx, a, grid, dev, stream);
+    case 96: return launch_qgemm_t<kInt8, 96>(tw, tx, a, grid, dev, stream);
+    case 128: return launch_qgemm_t<kInt8, 128>(tw, tx, a, grid, dev, stream);
+    default: return QSPEC_ERR_INVALID_ARG;
+  }
+}
+
+template <bool kInt8>
+qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
+                      const uint16_t* ws, int64_t n, int32_t group, float* y, void* workspace,
+                      size_t workspace_bytes, int32_t* dbg_acc, void* stream_v) {
+  if (!x || !wq || !ws || !y || !workspace) return QSPEC_ERR_INVALID_ARG;
+  if (!gemm_shape_ok(m, n, k, group)) return QSPEC_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(wq, 16) || !aligned(ws, 2) || !aligned(y, 4) ||
+      !aligned(workspace, 16) || (dbg_acc && !aligned(dbg_acc, 4)))
+    return QSPEC_ERR_INVALID_ARG;
+  int dev = 0;
+  DeviceInfo info;
+  qspec_status st = current_device(&dev, &info);
+  if (st != QSPEC_OK) return st;
+  const GemmPlan p = plan_gemm(kInt8, m, n, k, info.sm_count);
+  if (workspace_bytes < p.total) return QSPEC_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  uint8_t* wsp = static_cast<uint8_t*>(workspace);
+
+  CUtensorMap tw, tx;
+  if (!make_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wq, n, k / 2, kTileN, kUnitK / 2,
+                 CU_TENSOR_MAP_SWIZZLE_NONE))
+    return QSPEC_ERR_CUDA;
+  GemmArgs a;
+  a.M = static_cast<int>(m);
+  a.N = static_cast<int>(n);
+  a.K = static_cast<int>(k);
+  a.groups_per_row = static_cast<int>(k / group);
+  a.groups_per_unit = kUnitK / group;
+  a.m_tiles = p.m_tiles;
+  a.n_tiles = p.n_tiles;
+  a.ku = p.ku;
+  a.units = p.units;
+  a.ws = ws;
+  a.y = y;
+  a.dbg_acc = dbg_acc;
+  a.status = reinterpret_cast<uint32_t*>(wsp);
+  a.counters = reinterpret_cast<uint32_t*>(wsp + p.off_counters);
+  a.partials = reinterpret_cast<float*>(wsp + p.off_partials);
+  a.s_a = nullptr;
+  if constexpr (kInt8) {
+    int8_t* xq = reinterpret_cast<int8_t*>(wsp + p.off_xq);
+    float* sa = reinterpret_cast<float*>(wsp + p.off_sa);
+    quant_act_kernel<false><<<static_cast<unsigned>(m), 256, 0, stream>>>(x, k, xq, sa);
+    if (cudaGetLastError() != cudaSuccess) return QSPEC_ERR_CUDA;
+    a.s_a = sa;
+    if (!make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, xq, m, k, p.mt, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+      return QSPEC_ERR_CUDA;
+  } else {
+    if (!make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, m, k, p.mt, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+      return QSPEC_ERR_CUDA;
+  }
+  return launch_qgemm<kInt8>(p.mt, tw, tx, a, p.grid, dev, stream);
+}
+
+}  // namespace
+}  // namespace qspec
+
+using namespace qspec;
+
+extern "C" {
+
+qspec_status qspec_quantize_weights(const float* w, int64_t n, int64_t k, int32_t group,
+                                    uint8_t* wq, uint16_t* ws, void* stream) {
+  if (!w || !wq || !ws) return QSPEC_ERR_INVALID_ARG;
+  if (n < 1 || (group != 64 && group != 128) || k < group || (k % group) != 0)
+    return QSPEC_ERR_INVALID_ARG;
+  if (!aligned(w, 16) || !aligned(wq, 2) || !aligned(ws, 2)) return QSPEC_ERR_INVALID_ARG;
+  const long long warps = n * (k / group);
+  const long long blocks = (warps + 7) / 8;
+  if (blocks > 0x7FFFFFFFll) return QSPEC_ERR_INVALID_ARG;
+  qspec_status st = current_device(nullptr, nullptr);
+  if (st != QSPEC_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (group == 128)
+    quantize_weights_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, n, k, wq, ws);
+  else
+    quantize_weights_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, n, k, wq, ws);
+  return cudaGetLastError() == cudaSuccess ? QSPEC_OK : QSPEC_ERR_CUDA;
+}
+
+qspec_status qspec_quant_act(const uint16_t* x, int64_t m, int64_t k, uint8_t* xq, float* xs,
+                             void* stream) {
+  if (!x || !xq || !xs) return QSPEC_ERR_INVALID_ARG;
+  if (m < 1 || m > 0x7FFFFFFFll || k < 8 || (k % 8) != 0) return QSPEC_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(xq, 4) || !aligned(xs, 4)) return QSPEC_ERR_INVALID_ARG;
+  qspec_status st = current_device(nullptr, nullptr);
+  if (st != QSPEC_OK) return st;
+  quant_act_kernel<true><<<static_cast<unsigned>(m), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      x, k, xq, xs);
+  return cudaGetLastError() == cudaSuccess ? QSPEC_OK : QSPEC_ERR_CUDA;
+}
+
+qspec_status qspec_gemm_w4a4(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
+                             const uint16_t* ws, int64_t n, int32_t group, float* y,
+                             void* workspace, size_t workspace_bytes, int32_t* dbg_acc,
+                             void* stream) {
+  return run_gemm<true>(x, m, k, wq, ws, n, group, y, workspace, workspace_bytes, dbg_acc, stream);
+}
+
+qspec_status qspec_gemm_w4a16(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
+                              const uint16_t* ws, int64_t n, int32_t group, float* y,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  return run_gemm<false>(x, m, k, wq, ws, n, group, y, workspace, workspace_bytes, nullptr,
+                         stream);
+}
+
+qspec_status qspec_spec_accept(const float* p, const float* q, const int32_t* draft,
+                               const float* u_acc, const float* u_res, int32_t batch,
+                               int32_t gamma, int32_t vocab, int32_t* n_accepted,
+                               int32_t* tokens, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  if (!p || !q || !draft || !u_acc || !u_res || !n_accepted || !tokens)
+    return QSPEC_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 65535 || gamma < 1 || gamma > 16 || vocab < 4 || vocab > 409600 ||
+      (vocab % 4) != 0)
+    return QSPEC_ERR_INVALID_ARG;
+  if (!aligned(p, 16) || !aligned(q, 16) || !aligned(draft, 4) || !aligned(u_acc, 4) ||
+      !aligned(u_res, 4) || !aligned(n_accepted, 4) || !aligned(tokens, 4))
+    return QSPEC_ERR_INVALID_ARG;
+  if (workspace && (workspace_bytes < 256 || !aligned(workspace, 16)))
+    return QSPEC_ERR_WORKSPACE_TOO_SMALL;
+  int dev = 0;
+  qspec_status st = current_device(&dev, nullptr);
+  if (st != QSPEC_OK) return st;
+  const int chunk = ((vocab + 4 * kAcceptCluster - 1) / (4 * kAcceptCluster)) * 4;
+  const size_t smem = static_cast<size_t>(chunk) * 4;
+  static bool attr_set[kMaxDevices] = {};
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(spec_accept_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             204800) != cudaSuccess) {
+      cudaGetLastError();
+      return QSPEC_ERR_CUDA;
+    }
+    attr_set[dev] = true;
+  }
+  spec_accept_kernel<<<batch * kAcceptCluster, kAcceptThreads, smem,
+                       static_cast<cudaStream_t>(stream)>>>(
+      p, q, draft, u_acc, u_res, gamma, vocab, chunk, n_accepted, tokens,
+      static_cast<uint32_t*>(workspace));
+  return cudaGetLastError() == cudaSuccess ? QSPEC_OK : QSPEC_ERR_CUDA;
+}
+
+size_t qspec_workspace_size(int32_t op, int64_t m, int64_t n, int64_t k, int32_t group,
+                            int32_t batch, int32_t gamma, int32_t vocab) {
+  (void)batch;
+  (void)gamma;
+  (void)vocab;
+  switch (op) {
+    case QSPEC_OP_QUANTIZE_WEIGHTS:
+    case QSPEC_OP_QUANT_ACT:
+      return 0;
+    case QSPEC_OP_SPEC_ACCEPT:
+      return 256;
+    case QSPEC_OP_GEMM_W4A4:
+    case QSPEC_OP_GEMM_W4A16: {
+      if (!gemm_shape_ok(m, n, k, group)) return 0;
+      DeviceInfo info;
+      if (current_device(nullptr, &info) != QSPEC_OK) return 0;
+      return plan_gemm(op == QSPEC_OP_GEMM_W4A4, m, n, k, info.sm_count).total;
+    }
+    default:
+      return 0;
+  }
+}
+
+qspec_status qspec_workspace_status(void* workspace, void* stream) {
+  if (!workspace) return QSPEC_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, workspace, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return QSPEC_ERR_CUDA;
+  }
+  if (word == 0) return QSPEC_OK;
+  if (cudaMemsetAsync(workspace, 0, 4, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return QSPEC_ERR_CUDA;
+  }
+  return (word & kDevTimeout) ? QSPEC_ERR_TIMEOUT : QSPEC_ERR_BAD_INPUT;
+}
+
+const char* qspec_status_string(qspec_status status) {
+  switch (status) {
+    case QSPEC_OK: return "ok";
+    case QSPEC_ERR_INVALID_ARG: return "invalid argument";
+    case QSPEC_ERR_UNSUPPORTED_DEVICE: return "unsupported device (needs sm_100)";
+    case QSPEC_ERR_CUDA: return "CUDA error";
+    case QSPEC_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case QSPEC_ERR_TIMEOUT: return "kernel wait timed out";
+    case QSPEC_ERR_BAD_INPUT: return "invalid input data seen by a kernel";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

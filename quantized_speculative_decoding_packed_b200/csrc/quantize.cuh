@@ -1,0 +1,131 @@
+// Weight and activation quantizers (QSpec abstract: one INT4 weight set for
+// both stages; explainer essay paragraph 2: W4A4 also quantizes activations).
+//
+// All decisions are taken in IEEE fp32 with round-to-nearest-even:
+//   weights:     s = absmax / 7, s_h = fp16(s), q = clamp(rint(w / s_h), -8, 7)
+//   activations: s_a = absmax / 7, inv = 7 / absmax, q = clamp(rint(x * inv), -8, 7)
+// The explicit __fdiv_rn / __fmul_rn intrinsics pin the rounding regardless of
+// compiler flags and forbid contraction into FMAs.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cstdint>
+
+namespace qspec {
+
+__device__ __forceinline__ int clamp_q(int v) { return v < -8 ? -8 : (v > 7 ? 7 : v); }
+
+// One warp per (row n, group g).  Lane l handles GROUP/32 consecutive values.
+template <int GROUP>
+__global__ void __launch_bounds__(256) quantize_weights_kernel(const float* __restrict__ w,
+                                                               int64_t n_rows, int64_t k,
+                                                               uint8_t* __restrict__ wq,
+                                                               uint16_t* __restrict__ ws) {
+  constexpr int PER_LANE = GROUP / 32;
+  const int64_t groups_per_row = k / GROUP;
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (gw >= n_rows * groups_per_row) return;
+  const int64_t row = gw / groups_per_row;
+  const int64_t g = gw - row * groups_per_row;
+  const float* src = w + row * k + g * GROUP + lane * PER_LANE;
+
+  float v[PER_LANE];
+  if constexpr (PER_LANE == 4) {
+    const float4 t = *reinterpret_cast<const float4*>(src);
+    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+  } else {
+    const float2 t = *reinterpret_cast<const float2*>(src);
+    v[0] = t.x; v[1] = t.y;
+  }
+  float a = 0.f;
+#pragma unroll
+  for (int i = 0; i < PER_LANE; ++i) a = fmaxf(a, fabsf(v[i]));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+
+  const float s = __fdiv_rn(a, 7.0f);
+  const __half sh = __float2half_rn(s);
+  const float sf = __half2float(sh);
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < PER_LANE; ++i) {
+    const int q = (sf == 0.f) ? 0 : clamp_q(__float2int_rn(__fdiv_rn(v[i], sf)));
+    packed |= (static_cast<uint32_t>(q) & 0xFu) << (4 * i);
+  }
+  uint8_t* dst = wq + row * (k / 2) + g * (GROUP / 2) + lane * (PER_LANE / 2);
+  if constexpr (PER_LANE == 4) {
+    *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(packed);
+  } else {
+    *dst = static_cast<uint8_t>(packed);
+  }
+  if (lane == 0) ws[row * groups_per_row + g] = __half_as_ushort(sh);
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) {
+  return __uint_as_float(bits16 << 16);
+}
+
+// One CTA per token row.  kPacked: write two nibbles per byte (the ABI
+// format); otherwise write one int8 per element (the layout the W4A4 GEMM
+// streams into its tensor-core operand tiles).
+template <bool kPacked>
+__global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restrict__ x,
+                                                        int64_t k, void* __restrict__ out,
+                                                        float* __restrict__ scales) {
+  __shared__ float red[8];
+  const int64_t row = blockIdx.x;
+  const uint16_t* xr = x + row * k;
+  const int tid = threadIdx.x;
+
+  float a = 0.f;
+  for (int64_t c = static_cast<int64_t>(tid) * 8; c < k; c += 256 * 8) {
+    const uint4 u = *reinterpret_cast<const uint4*>(xr + c);
+    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      a = fmaxf(a, fabsf(bf16_bits_to_float(w4[j] & 0xFFFFu)));
+      a = fmaxf(a, fabsf(bf16_bits_to_float(w4[j] >> 16)));
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+  if ((tid & 31) == 0) red[tid >> 5] = a;
+  __syncthreads();
+  a = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) a = fmaxf(a, red[i]);
+
+  const float s = __fdiv_rn(a, 7.0f);
+  const float inv = __fdiv_rn(7.0f, a);
+  if (tid == 0) scales[row] = s;
+
+  for (int64_t c = static_cast<int64_t>(tid) * 8; c < k; c += 256 * 8) {
+    const uint4 u = *reinterpret_cast<const uint4*>(xr + c);
+    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+    int q[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float lo = bf16_bits_to_float(w4[j] & 0xFFFFu);
+      const float hi = bf16_bits_to_float(w4[j] >> 16);
+      q[2 * j] = (a == 0.f) ? 0 : clamp_q(__float2int_rn(__fmul_rn(lo, inv)));
+      q[2 * j + 1] = (a == 0.f) ? 0 : clamp_q(__float2int_rn(__fmul_rn(hi, inv)));
+    }
+    if constexpr (kPacked) {
+      uint32_t p = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) p |= (static_cast<uint32_t>(q[j]) & 0xFu) << (4 * j);
+      *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(out) + row * (k / 2) + c / 2) = p;
+    } else {
+      uint32_t lo = 0, hi = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        lo |= (static_cast<uint32_t>(q[j]) & 0xFFu) << (8 * j);
+        hi |= (static_cast<uint32_t>(q[j + 4]) & 0xFFu) << (8 * j);
+      }
+      *reinterpret_cast<uint2*>(static_cast<int8_t*>(out) + row * k + c) = make_uint2(lo, hi);
+    }
+  }
+}
+
+}  // namespace qspec

@@ -1,0 +1,189 @@
+"""Python binding of libqspec.so (the C ABI in include/qspec.h).
+
+Argument marshalling only: every step of the hot path runs in the CUDA
+kernels of the library.  Importing this module loads the library and raises
+if it is missing; there is no fallback implementation.
+
+Functions take CUDA torch tensors (contiguous, on the current device) and
+launch on the current torch stream unless `stream` is given.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqspec.so")
+
+OK = 0
+STATUS_NAMES = {0: "ok", 1: "invalid argument", 2: "unsupported device", 3: "CUDA error",
+                4: "workspace too small", 5: "timeout", 6: "bad input"}
+OP_QUANTIZE_WEIGHTS, OP_QUANT_ACT, OP_GEMM_W4A4, OP_GEMM_W4A16, OP_SPEC_ACCEPT = range(5)
+
+EXPORTED = ("qspec_quantize_weights", "qspec_quant_act", "qspec_gemm_w4a4", "qspec_gemm_w4a16",
+            "qspec_spec_accept", "qspec_workspace_size", "qspec_workspace_status",
+            "qspec_status_string")
+
+
+class QSpecError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} (status {status})")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(
+            f"libqspec.so not found at {_LIB_PATH}; build it with "
+            "`python -m quantized_speculative_decoding_packed_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+    lib.qspec_quantize_weights.argtypes = [P, I64, I64, I32, P, P, P]
+    lib.qspec_quant_act.argtypes = [P, I64, I64, P, P, P]
+    lib.qspec_gemm_w4a4.argtypes = [P, I64, I64, P, P, I64, I32, P, P, SZ, P, P]
+    lib.qspec_gemm_w4a16.argtypes = [P, I64, I64, P, P, I64, I32, P, P, SZ, P]
+    lib.qspec_spec_accept.argtypes = [P, P, P, P, P, I32, I32, I32, P, P, P, SZ, P]
+    lib.qspec_workspace_size.argtypes = [I32, I64, I64, I64, I32, I32, I32, I32]
+    lib.qspec_workspace_size.restype = SZ
+    lib.qspec_workspace_status.argtypes = [P, P]
+    lib.qspec_status_string.argtypes = [I32]
+    lib.qspec_status_string.restype = ctypes.c_char_p
+    for name in ("qspec_quantize_weights", "qspec_quant_act", "qspec_gemm_w4a4",
+                 "qspec_gemm_w4a16", "qspec_spec_accept", "qspec_workspace_status"):
+        getattr(lib, name).restype = ctypes.c_int
+    return lib
+
+
+LIB = _load()
+LIB_PATH = _LIB_PATH
+
+
+def _check(status: int, what: str) -> None:
+    if status != OK:
+        raise QSpecError(status, what)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, dtype, name: str) -> None:
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+
+
+_WS_CACHE: dict = {}
+
+
+def workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A zero-initialised per-device scratch buffer of at least `nbytes` bytes.
+
+    The library leaves it ready for reuse after every call that completes.
+    Calls that run concurrently on different streams need separate buffers.
+    """
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    cur = _WS_CACHE.get(dev)
+    if cur is None or cur.numel() < nbytes:
+        cur = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=dev)
+        _WS_CACHE[dev] = cur
+    return cur
+
+
+def workspace_size(op: int, m: int = 0, n: int = 0, k: int = 0, group: int = 128,
+                   batch: int = 0, gamma: int = 0, vocab: int = 0) -> int:
+    return int(LIB.qspec_workspace_size(op, m, n, k, group, batch, gamma, vocab))
+
+
+def workspace_status(ws: torch.Tensor, stream=None) -> int:
+    return int(LIB.qspec_workspace_status(_ptr(ws), _stream(stream)))
+
+
+def quantize_weights(w: torch.Tensor, group: int = 128, wq: torch.Tensor | None = None,
+                     ws: torch.Tensor | None = None, stream=None):
+    """fp32 [N][K] -> (wq uint8 [N][K/2], ws fp16 [N][K/group])."""
+    _need(w, torch.float32, "w")
+    n, k = w.shape
+    if wq is None:
+        wq = torch.empty((n, k // 2), dtype=torch.uint8, device=w.device)
+    if ws is None:
+        ws = torch.empty((n, k // group), dtype=torch.float16, device=w.device)
+    _check(LIB.qspec_quantize_weights(_ptr(w), n, k, group, _ptr(wq), _ptr(ws), _stream(stream)),
+           "qspec_quantize_weights")
+    return wq, ws
+
+
+def quant_act(x: torch.Tensor, xq: torch.Tensor | None = None, xs: torch.Tensor | None = None,
+              stream=None):
+    """bf16 [M][K] -> (xq uint8 [M][K/2] packed INT4, xs fp32 [M] per-token scales)."""
+    _need(x, torch.bfloat16, "x")
+    m, k = x.shape
+    if xq is None:
+        xq = torch.empty((m, k // 2), dtype=torch.uint8, device=x.device)
+    if xs is None:
+        xs = torch.empty((m,), dtype=torch.float32, device=x.device)
+    _check(LIB.qspec_quant_act(_ptr(x), m, k, _ptr(xq), _ptr(xs), _stream(stream)),
+           "qspec_quant_act")
+    return xq, xs
+
+
+def gemm_w4a4(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor, group: int = 128,
+              y: torch.Tensor | None = None, work: torch.Tensor | None = None,
+              dbg_acc: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """W4A4 drafting GEMM: y[M][N] fp32 = quant(x) . deq(wq, ws)^T."""
+    _need(x, torch.bfloat16, "x")
+    m, k = x.shape
+    n = wq.shape[0]
+    if y is None:
+        y = torch.empty((m, n), dtype=torch.float32, device=x.device)
+    need = workspace_size(OP_GEMM_W4A4, m, n, k, group)
+    if work is None:
+        work = workspace(need, x.device)
+    _check(LIB.qspec_gemm_w4a4(_ptr(x), m, k, _ptr(wq), _ptr(ws), n, group, _ptr(y), _ptr(work),
+                               work.numel(), _ptr(dbg_acc), _stream(stream)), "qspec_gemm_w4a4")
+    return y
+
+
+def gemm_w4a16(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor, group: int = 128,
+               y: torch.Tensor | None = None, work: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """W4A16 verifying GEMM: y[M][N] fp32 = x . deq(wq, ws)^T."""
+    _need(x, torch.bfloat16, "x")
+    m, k = x.shape
+    n = wq.shape[0]
+    if y is None:
+        y = torch.empty((m, n), dtype=torch.float32, device=x.device)
+    need = workspace_size(OP_GEMM_W4A16, m, n, k, group)
+    if work is None:
+        work = workspace(need, x.device)
+    _check(LIB.qspec_gemm_w4a16(_ptr(x), m, k, _ptr(wq), _ptr(ws), n, group, _ptr(y), _ptr(work),
+                                work.numel(), _stream(stream)), "qspec_gemm_w4a16")
+    return y
+
+
+def spec_accept(p: torch.Tensor, q: torch.Tensor, draft: torch.Tensor, u_acc: torch.Tensor,
+                u_res: torch.Tensor, n_accepted: torch.Tensor | None = None,
+                tokens: torch.Tensor | None = None, work: torch.Tensor | None = None,
+                stream=None):
+    """Speculative accept / residual resample -> (n_accepted int32 [B], tokens int32 [B][gamma+1])."""
+    _need(p, torch.float32, "p")
+    _need(q, torch.float32, "q")
+    _need(draft, torch.int32, "draft")
+    _need(u_acc, torch.float32, "u_acc")
+    _need(u_res, torch.float32, "u_res")
+    b, g1, v = p.shape
+    gamma = g1 - 1
+    if n_accepted is None:
+        n_accepted = torch.empty((b,), dtype=torch.int32, device=p.device)
+    if tokens is None:
+        tokens = torch.empty((b, gamma + 1), dtype=torch.int32, device=p.device)
+    nbytes = 0 if work is None else work.numel()
+    _check(LIB.qspec_spec_accept(_ptr(p), _ptr(q), _ptr(draft), _ptr(u_acc), _ptr(u_res), b, gamma,
+                                 v, _ptr(n_accepted), _ptr(tokens), _ptr(work), nbytes,
+                                 _stream(stream)), "qspec_spec_accept")
+    return n_accepted, tokens

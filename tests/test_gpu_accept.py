@@ -1,0 +1,87 @@
+"""GPU parity of the speculative accept / residual resample kernel: accepted
+lengths and tokens identical to the oracle."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import qspec_oracle as orc
+from quantized_speculative_decoding_packed_b200 import synth
+
+from gpu_util import cuda_f32, cuda_i32
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def qs():
+    from quantized_speculative_decoding_packed_b200 import qspec
+    return qspec
+
+
+def _run(qs, ai, work=None):
+    n, tok = qs.spec_accept(cuda_f32(ai.p), cuda_f32(ai.q), cuda_i32(ai.draft),
+                            cuda_f32(ai.u_acc), cuda_f32(ai.u_res), work=work)
+    torch.cuda.synchronize()
+    return n.cpu().numpy(), tok.cpu().numpy()
+
+
+def near_ties(ai) -> int:
+    """Positions where |u - p/q| < 1e-6 (reported; the exact test makes them agree anyway)."""
+    b = np.arange(ai.draft.shape[0])[:, None]
+    i = np.arange(ai.draft.shape[1])[None, :]
+    ratio = ai.p[b, i, ai.draft].astype(np.float64) / ai.q[b, i, ai.draft].astype(np.float64)
+    return int((np.abs(ai.u_acc.astype(np.float64) - ratio) < 1e-6).sum())
+
+
+def test_tiny_config_identical(qs):
+    ai = synth.tiny_accept_inputs()
+    n, tok = _run(qs, ai)
+    n_ref, tok_ref = orc.spec_accept(ai.p, ai.q, ai.draft, ai.u_acc, ai.u_res)
+    assert np.array_equal(n, n_ref) and np.array_equal(tok, tok_ref)
+
+
+@pytest.mark.parametrize("sigma", synth.ACCEPT_SIGMAS)
+def test_vocab_128256_batch_64_identical(qs, sigma):
+    ai = synth.big_accept_inputs(sigma)
+    n, tok = _run(qs, ai)
+    n_ref, tok_ref = orc.spec_accept(ai.p, ai.q, ai.draft, ai.u_acc, ai.u_res)
+    print(f"sigma={sigma}: near ties {near_ties(ai)}, mean accepted {n.mean():.3f}")
+    assert np.array_equal(n, n_ref)
+    assert np.array_equal(tok, tok_ref)
+
+
+@pytest.mark.parametrize("b,g,v", [(1, 1, 4), (3, 16, 36), (5, 2, 1000), (130, 3, 2048)])
+def test_ragged_sizes_identical(qs, b, g, v):
+    ai = synth.accept_inputs(synth.rng_for("accept", 11, b, g, v), b, g, v, 1.0, 0.7)
+    n, tok = _run(qs, ai)
+    n_ref, tok_ref = orc.spec_accept(ai.p, ai.q, ai.draft, ai.u_acc, ai.u_res)
+    assert np.array_equal(n, n_ref) and np.array_equal(tok, tok_ref)
+
+
+def test_p_equals_q_accepts_all_and_draws_bonus(qs):
+    ai = synth.accept_inputs(synth.rng_for("accept", 12), 8, 5, 5000, 2.0, 0.5)
+    ai.q = ai.p[:, :5, :].copy()
+    n, tok = _run(qs, ai)
+    n_ref, tok_ref = orc.spec_accept(ai.p, ai.q, ai.draft, ai.u_acc, ai.u_res)
+    assert np.all(n == 5) and np.array_equal(tok, tok_ref)
+
+
+def test_empty_residual_falls_back_to_target_row(qs):
+    ai = synth.accept_inputs(synth.rng_for("accept", 13), 4, 4, 64, 1.0, 0.5)
+    ai.q = ai.p[:, :4, :].copy()
+    for b in range(4):
+        ai.p[b, b % 4, ai.draft[b, b % 4]] = 0.0    # forces a rejection with an empty residual
+    n, tok = _run(qs, ai)
+    n_ref, tok_ref = orc.spec_accept(ai.p, ai.q, ai.draft, ai.u_acc, ai.u_res)
+    assert np.array_equal(n, n_ref) and np.array_equal(tok, tok_ref)
+
+
+def test_out_of_range_draft_is_reported(qs):
+    ai = synth.tiny_accept_inputs()
+    ai.draft = ai.draft.copy()
+    ai.draft[1, 1] = 32                              # == vocab: invalid
+    work = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    n, tok = _run(qs, ai, work=work)
+    assert n[1] <= 1
+    assert qs.workspace_status(work) == 6
+    assert qs.workspace_status(work) == 0           # reading clears it

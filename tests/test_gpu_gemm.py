@@ -1,0 +1,159 @@
+"""GPU parity of the shared-INT4 GEMMs against the oracle.
+
+W4A4: per-group int32 accumulators bit-exact; outputs within 1e-3 relative.
+W4A16: outputs within 1e-3 relative Frobenius of the float64 oracle on the
+same dequantized weights (and bit-exact where every partial sum is an
+integer below 2^24).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import qspec_oracle as orc
+from quantized_speculative_decoding_packed_b200 import synth
+
+from gpu_util import assert_close_1e3, cuda_bf16, cuda_f32, rel_fro
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def qs():
+    from quantized_speculative_decoding_packed_b200 import qspec
+    return qspec
+
+
+def _prep(qs, gi):
+    wq, ws = qs.quantize_weights(cuda_f32(gi.w), gi.group)
+    q, s_h = orc.quantize_weights(gi.w, gi.group)
+    return wq, ws, q, s_h
+
+
+SHAPES = [  # (m, n, k, group): tiles, ragged tails, both group sizes, every token tile
+    (4, 256, 256, 64), (1, 256, 1024, 128), (3, 200, 256, 64), (16, 1000, 1024, 128),
+    (17, 384, 512, 128), (33, 256, 384, 64), (48, 130, 256, 128), (64, 512, 768, 128),
+    (80, 512, 1024, 128), (95, 256, 256, 64), (100, 256, 384, 128), (128, 384, 512, 128),
+    (130, 384, 512, 128), (257, 136, 256, 64),
+]
+
+
+@pytest.mark.parametrize("m,n,k,group", SHAPES)
+def test_w4a4_accumulators_exact_and_output(qs, m, n, k, group):
+    gi = synth.gemm_inputs("llama3_8b", m, n, k, group, stream=99)
+    wq, ws, q, s_h = _prep(qs, gi)
+    dbg = torch.zeros((m, n, k // group), dtype=torch.int32, device="cuda")
+    y = qs.gemm_w4a4(cuda_bf16(gi.x_bits), wq, ws, group, dbg_acc=dbg)
+    torch.cuda.synchronize()
+    y_ref, acc = orc.gemm_w4a4(gi.x, q, s_h, group, return_acc=True)
+    assert np.array_equal(dbg.cpu().numpy(), acc)
+    assert_close_1e3(y.cpu().numpy(), y_ref)
+
+
+@pytest.mark.parametrize("m,n,k,group", SHAPES)
+def test_w4a16_output(qs, m, n, k, group):
+    gi = synth.gemm_inputs("llama3_8b", m, n, k, group, stream=98)
+    wq, ws, q, s_h = _prep(qs, gi)
+    y = qs.gemm_w4a16(cuda_bf16(gi.x_bits), wq, ws, group)
+    torch.cuda.synchronize()
+    y_ref = orc.gemm_w4a16(gi.x, q, s_h, group)
+    assert_close_1e3(y.cpu().numpy(), y_ref)
+    assert rel_fro(y.cpu().numpy(), y_ref) < 1e-5      # fp32 accumulation only
+
+
+@pytest.mark.parametrize("mode", ["w4a4", "w4a16"])
+def test_integer_special_case_bit_exact(qs, mode):
+    """Scale 1 (absmax 7 per group) and integer activations with absmax 7:
+    every partial sum is an integer below 2^24, so both modes are exact."""
+    rng = np.random.default_rng(21)
+    m, n, k = 20, 384, 512
+    lv = rng.integers(-7, 8, size=(n, k))
+    lv[:, ::128] = 7
+    xi = rng.integers(-7, 8, size=(m, k)).astype(np.float32)
+    xi[:, 3] = -7
+    bits = synth.to_bf16_bits(xi)
+    wq, ws = qs.quantize_weights(cuda_f32(lv.astype(np.float32)), 128)
+    fn = qs.gemm_w4a4 if mode == "w4a4" else qs.gemm_w4a16
+    y = fn(cuda_bf16(bits), wq, ws, 128)
+    torch.cuda.synchronize()
+    assert np.array_equal(y.cpu().numpy().astype(np.float64), (xi.astype(np.int64) @ lv.T).astype(np.float64))
+
+
+def test_repeat_calls_are_deterministic(qs):
+    gi = synth.gemm_inputs("llama3_8b", 16, 4096, 4096, 128, stream=5)
+    wq, ws, q, s_h = _prep(qs, gi)
+    x = cuda_bf16(gi.x_bits)
+    for fn in (qs.gemm_w4a4, qs.gemm_w4a16):
+        y1 = fn(x, wq, ws, 128).clone()
+        y2 = fn(x, wq, ws, 128).clone()
+        torch.cuda.synchronize()
+        assert torch.equal(y1, y2)
+
+
+def _sampled_full_size(qs, mode, m, name, n, k):
+    gi = synth.gemm_inputs("llama2_7b", m, n, k, 128)
+    wq, ws = qs.quantize_weights(cuda_f32(gi.w), 128)
+    x = cuda_bf16(gi.x_bits)
+    cols = np.sort(synth.rng_for("llama2_7b", 9, n).choice(n, size=256, replace=False))
+    q, s_h = orc.quantize_weights(gi.w[cols], 128)
+    if mode == "w4a4":
+        dbg = torch.zeros((m, n, k // 128), dtype=torch.int32, device="cuda")
+        y = qs.gemm_w4a4(x, wq, ws, 128, dbg_acc=dbg)
+        torch.cuda.synchronize()
+        y_ref, acc = orc.gemm_w4a4(gi.x, q, s_h, 128, return_acc=True)
+        assert np.array_equal(dbg.cpu().numpy()[:, cols, :], acc)
+    else:
+        y = qs.gemm_w4a16(x, wq, ws, 128)
+        torch.cuda.synchronize()
+        y_ref = orc.gemm_w4a16(gi.x, q, s_h, 128)
+    assert_close_1e3(y.cpu().numpy()[:, cols], y_ref)
+
+
+@pytest.mark.parametrize("name,n,k", synth.LLAMA2_7B_LAYERS)
+def test_llama2_7b_decode_shapes_sampled(qs, name, n, k):
+    _sampled_full_size(qs, "w4a4", 16, name, n, k)
+    _sampled_full_size(qs, "w4a16", 80, name, n, k)
+
+
+@pytest.mark.parametrize("m", synth.LLAMA3_8B_M_SWEEP)
+def test_llama3_8b_sweep_sampled(qs, m):
+    n, k = 6144, 4096
+    gi = synth.gemm_inputs("llama3_8b", m, n, k, 128)
+    wq, ws = qs.quantize_weights(cuda_f32(gi.w), 128)
+    x = cuda_bf16(gi.x_bits)
+    cols = np.sort(synth.rng_for("llama3_8b", 9, m).choice(n, size=128, replace=False))
+    q, s_h = orc.quantize_weights(gi.w[cols], 128)
+    y4 = qs.gemm_w4a4(x, wq, ws, 128)
+    y16 = qs.gemm_w4a16(x, wq, ws, 128)
+    torch.cuda.synchronize()
+    assert_close_1e3(y4.cpu().numpy()[:, cols], orc.gemm_w4a4(gi.x, q, s_h, 128))
+    assert_close_1e3(y16.cpu().numpy()[:, cols], orc.gemm_w4a16(gi.x, q, s_h, 128))
+
+
+def test_llama2_70b_large_m_sampled(qs):
+    """M = 2048 on the 70B QKV shape; outputs checked on sampled rows and columns."""
+    m, n, k = 2048, 10240, 8192
+    gi = synth.gemm_inputs("llama2_70b", m, n, k, 128)
+    wq, ws = qs.quantize_weights(cuda_f32(gi.w), 128)
+    x = cuda_bf16(gi.x_bits)
+    rows = np.sort(synth.rng_for("llama2_70b", 9, 1).choice(m, size=64, replace=False))
+    cols = np.sort(synth.rng_for("llama2_70b", 9, 2).choice(n, size=64, replace=False))
+    q, s_h = orc.quantize_weights(gi.w[cols], 128)
+    y4 = qs.gemm_w4a4(x, wq, ws, 128)
+    y16 = qs.gemm_w4a16(x, wq, ws, 128)
+    torch.cuda.synchronize()
+    xs = gi.x[rows]
+    # the W4A4 reference quantizes each sampled row on its own, as the kernel does
+    assert_close_1e3(y4.cpu().numpy()[np.ix_(rows, cols)], orc.gemm_w4a4(xs, q, s_h, 128))
+    assert_close_1e3(y16.cpu().numpy()[np.ix_(rows, cols)], orc.gemm_w4a16(xs, q, s_h, 128))
+
+
+def test_shared_weights_are_one_buffer(qs):
+    """Both modes read the same wq/ws bytes; nothing is repacked per mode."""
+    gi = synth.gemm_inputs("llama3_8b", 16, 256, 256, 128, stream=3)
+    wq, ws = qs.quantize_weights(cuda_f32(gi.w), 128)
+    before = (wq.clone(), ws.clone())
+    x = cuda_bf16(gi.x_bits)
+    qs.gemm_w4a4(x, wq, ws, 128)
+    qs.gemm_w4a16(x, wq, ws, 128)
+    torch.cuda.synchronize()
+    assert torch.equal(before[0], wq) and torch.equal(before[1], ws)

@@ -1,0 +1,92 @@
+"""Host-side checks that need no GPU: the C ABI library loads, exports every
+symbol the header declares, and rejects bad arguments before launching."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qspec.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from quantized_speculative_decoding_packed_b200 import build
+    build.build()
+    from quantized_speculative_decoding_packed_b200 import qspec
+    return qspec
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:qspec_status|size_t|const char\*)\s+(qspec_\w+)\s*\(",
+                                 text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for name in ("qspec_quantize_weights", "qspec_quant_act", "qspec_gemm_w4a4",
+                 "qspec_gemm_w4a16", "qspec_spec_accept", "qspec_workspace_size",
+                 "qspec_workspace_status", "qspec_status_string"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    raw = ctypes.CDLL(lib.LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(raw, name), name
+
+
+def test_status_strings(lib):
+    for code, text in [(0, b"ok"), (1, b"invalid argument"), (4, b"workspace too small"),
+                       (5, b"kernel wait timed out")]:
+        assert lib.LIB.qspec_status_string(code) == text
+
+
+FAKE = ctypes.c_void_p(0x10000)      # 16-byte aligned, never dereferenced: validation fails first
+
+
+@pytest.mark.parametrize("args", [
+    (None, 4, 256, 64, FAKE, FAKE, None),            # null input
+    (FAKE, 4, 256, 32, FAKE, FAKE, None),            # unsupported group
+    (FAKE, 4, 200, 64, FAKE, FAKE, None),            # k not a multiple of group
+    (FAKE, 0, 256, 64, FAKE, FAKE, None),            # empty
+])
+def test_quantize_weights_rejects(lib, args):
+    assert lib.LIB.qspec_quantize_weights(*args) == 1
+
+
+@pytest.mark.parametrize("m,k,n,group", [(0, 256, 256, 64), (4, 200, 256, 64), (4, 256, 0, 64),
+                                         (4, 256, 256, 96), (4, 64, 256, 64)])
+def test_gemm_rejects_bad_shapes(lib, m, k, n, group):
+    assert lib.LIB.qspec_gemm_w4a4(FAKE, m, k, FAKE, FAKE, n, group, FAKE, FAKE, 1 << 30, None,
+                                   None) == 1
+    assert lib.LIB.qspec_gemm_w4a16(FAKE, m, k, FAKE, FAKE, n, group, FAKE, FAKE, 1 << 30,
+                                    None) == 1
+
+
+def test_gemm_rejects_misaligned_pointers(lib):
+    odd = ctypes.c_void_p(0x10008)
+    assert lib.LIB.qspec_gemm_w4a16(odd, 4, 256, FAKE, FAKE, 256, 64, FAKE, FAKE, 1 << 30, None) == 1
+    assert lib.LIB.qspec_gemm_w4a16(FAKE, 4, 256, odd, FAKE, 256, 64, FAKE, FAKE, 1 << 30, None) == 1
+    assert lib.LIB.qspec_gemm_w4a16(FAKE, 4, 256, FAKE, FAKE, 256, 64, FAKE, None, 1 << 30, None) == 1
+
+
+@pytest.mark.parametrize("b,g,v", [(0, 4, 32), (2, 0, 32), (2, 17, 32), (2, 4, 30), (2, 4, 0),
+                                   (2, 4, 409604)])
+def test_accept_rejects(lib, b, g, v):
+    assert lib.LIB.qspec_spec_accept(FAKE, FAKE, FAKE, FAKE, FAKE, b, g, v, FAKE, FAKE, None, 0,
+                                     None) == 1
+
+
+def test_quant_act_rejects(lib):
+    assert lib.LIB.qspec_quant_act(FAKE, 4, 12, FAKE, FAKE, None) == 1
+    assert lib.LIB.qspec_quant_act(FAKE, 0, 16, FAKE, FAKE, None) == 1
+    assert lib.LIB.qspec_quant_act(None, 4, 16, FAKE, FAKE, None) == 1
+
+
+def test_workspace_size_of_invalid_shapes_is_zero(lib):
+    assert lib.workspace_size(lib.OP_GEMM_W4A4, 4, 256, 200, 64) == 0
+    assert lib.workspace_size(lib.OP_QUANT_ACT, 4, 0, 256) == 0
+    assert lib.workspace_size(lib.OP_SPEC_ACCEPT, batch=2, gamma=4, vocab=32) == 256
