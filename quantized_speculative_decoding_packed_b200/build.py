@@ -30,12 +30,17 @@ def needs_build() -> bool:
     return any(os.path.getmtime(f) > t for f in DEPENDS)
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if not force and not needs_build() and not verbose_ptxas:
+def build(force: bool = False, verbose_ptxas: bool = False, trace: bool = False) -> str:
+    """trace=True builds libqspec_trace.so, a debug variant with per-warp
+    checkpoints and software alignment checks (never loaded by the package)."""
+    out = LIB.replace("libqspec.so", "libqspec_trace.so") if trace else LIB
+    if not force and not trace and not needs_build() and not verbose_ptxas:
         return LIB
     cmd = [nvcc(), "-std=c++17", "-O3", "-lineinfo", "--shared", "-Xcompiler", "-fPIC",
            "-gencode", "arch=compute_100a,code=sm_100a", "-I", INCLUDE, "-I", CSRC,
-           "-o", LIB] + SOURCES
+           "-o", out] + SOURCES
+    if trace:
+        cmd += ["-DQSPEC_TRACE", "-rdc=false"]
     if verbose_ptxas:
         cmd += ["-Xptxas", "-v"]
     res = subprocess.run(cmd, capture_output=True, text=True)
@@ -43,9 +48,8 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose_ptxas:
         sys.stdout.write(res.stdout + res.stderr)
-    return LIB
+    return out
 
 
 if __name__ == "__main__":
-    build(force=True, verbose_ptxas="--verbose-ptxas" in sys.argv)
-    print(LIB)
+    print(build(force=True, verbose_ptxas="--verbose-ptxas" in sys.argv, trace="--trace" in sys.argv))

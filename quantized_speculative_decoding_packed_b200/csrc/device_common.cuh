@@ -9,6 +9,29 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+// Debug builds (-DQSPEC_TRACE) record, per warp, the last checkpoint reached
+// into a host-mapped buffer that stays readable after a device fault, and
+// check operand alignment in software (record and skip instead of faulting).
+#ifdef QSPEC_TRACE
+static __device__ unsigned int* g_qspec_trace = nullptr;
+#define QSPEC_TRACE_AT(info)                                                            \
+  do {                                                                                  \
+    if (g_qspec_trace && (threadIdx.x & 31) == 0) {                                     \
+      volatile unsigned int* t_ = g_qspec_trace + (blockIdx.x * 64u + (threadIdx.x >> 5)); \
+      *t_ = (static_cast<unsigned>(__LINE__) << 16) | (static_cast<unsigned>(info) & 0xFFFFu); \
+      __threadfence_system();                                                           \
+    }                                                                                   \
+  } while (0)
+#define QSPEC_ALIGN_OK(addr, a)                                                          \
+  ((static_cast<unsigned long long>(addr) % (a)) == 0 ||                                 \
+   (g_qspec_trace && (g_qspec_trace[8191] = (0xA0000000u | __LINE__), __threadfence_system(), false)))
+#else
+#define QSPEC_TRACE_AT(info) \
+  do {                       \
+  } while (0)
+#define QSPEC_ALIGN_OK(addr, a) true
+#endif
+
 namespace qspec {
 
 // Device status bits written to the first word of a workspace.

@@ -24,7 +24,9 @@
 // units +-1, whatever the shape.  A CTA that covers a whole tile writes y
 // directly; partial tiles go to workspace slots and the last CTA to finish a
 // tile (an atomic ticket, no waiting) adds the slots in K order, so results
-// are deterministic.
+// are deterministic.  A split tile starts inside exactly one CTA's range and
+// at most one split tile starts in any CTA's range, so the ticket of a tile
+// is indexed by its first contributor; tickets return to zero after use.
 //
 // Warp roles (one CTA per SM):
 //   warp 0      TMA producer for packed weight tiles (8-stage ring, 8 KB each)
@@ -51,6 +53,7 @@ constexpr int kNumAcc = 4;                       // tensor-memory group ring
 constexpr int kConvWarps = 8;
 constexpr int kCtlWarps = 4;
 constexpr int kSmemLimit = 232448;               // sm_100 dynamic shared memory per CTA
+constexpr int kMaxGrid = 1024;                   // ticket slots in the workspace
 
 __host__ __device__ constexpr int pow2_at_least(int v) {
   int p = 32;
@@ -94,7 +97,7 @@ struct GemmArgs {
   float* y;                // [M][N]
   int32_t* dbg_acc;        // optional W4A4 per-group accumulators [M][N][K/group]
   uint32_t* status;        // device status word
-  uint32_t* counters;      // per-tile tickets [m_tiles * n_tiles]
+  uint32_t* counters;      // tickets [kMaxGrid], indexed by a split tile's first CTA
   float* partials;         // [2 * gridDim.x][MT][128]
 };
 
@@ -192,6 +195,8 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = misc[0];
+  QSPEC_TRACE_AT(tmem_base & 0xFFFF);
+  if (!QSPEC_ALIGN_OK(smem_u32(smem), 1024) || !QSPEC_ALIGN_OK(smem_u32(bars), 8)) *abort_flag = 1;
 
   if (warp == 0) {
     // ------------------------------------------------ packed-weight producer
@@ -204,6 +209,8 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
         const long long t = u / ku;
         const int kc = static_cast<int>(u - t * ku);
         const int n_tile = static_cast<int>(t / args.m_tiles);
+        QSPEC_TRACE_AT(i);
+        if (!QSPEC_ALIGN_OK(smem_u32(pk_buf + s * kPkBytes), 128)) break;
         mbar_arrive_expect_tx(smem_u32(&pk_full[s]), kPkBytes);
         tma_load_2d(smem_u32(pk_buf + s * kPkBytes), &tmap_w, smem_u32(&pk_full[s]),
                     kc * (kUnitK / 2), n_tile * kTileN);
@@ -224,6 +231,8 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
         const long long t = u / ku;
         const int kc = static_cast<int>(u - t * ku);
         const int m_tile = static_cast<int>(t % args.m_tiles);
+        QSPEC_TRACE_AT(i);
+        if (!QSPEC_ALIGN_OK(smem_u32(x_buf + s * C::kXBytes), 1024)) break;
         mbar_arrive_expect_tx(smem_u32(&x_full[s]), C::kXBytes);
 #pragma unroll
         for (int a = 0; a < C::kAtoms; ++a) {
@@ -249,6 +258,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
         if (!mbar_wait(smem_u32(&cv_full[s]), ph, abort_flag, args.status)) break;
         if (!mbar_wait(smem_u32(&x_full[s]), ph, abort_flag, args.status)) break;
         tc_fence_after();
+        QSPEC_TRACE_AT(i);
         const uint32_t a_base = smem_u32(cv_buf + s * C::kCvBytes);
         const uint32_t b_base = smem_u32(x_buf + s * C::kXBytes);
         for (int h = 0; h < gpu; ++h, ++j) {
@@ -264,10 +274,16 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
             const uint32_t atom = kbyte >> 7, within = kbyte & 127u;
             const uint64_t a_desc = smem_desc_sw128(a_base + atom * (kTileN * 128) + within);
             const uint64_t b_desc = smem_desc_sw128(b_base + atom * (MT * 128) + within);
+            QSPEC_TRACE_AT(0x8000 | (j << 4) | kk);
+            if (!QSPEC_ALIGN_OK(a_base + atom * (kTileN * 128) + within, 16) ||
+                !QSPEC_ALIGN_OK(b_base + atom * (MT * 128) + within, 16) ||
+                !QSPEC_ALIGN_OK(static_cast<uint32_t>(b * MT) & 0xFFFFu, 8))
+              continue;
             mma_ss<kInt8>(tmem_base + static_cast<uint32_t>(b * MT), a_desc, b_desc, idesc,
                           kk > 0 ? 1u : 0u);
           }
           mma_commit(smem_u32(&acc_full[b]));
+          QSPEC_TRACE_AT(0x4000 | j);
         }
         if (!ok) break;
         mma_commit(smem_u32(&cv_empty[s]));
@@ -291,9 +307,11 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       if (!__all_sync(0xffffffffu, ok)) break;
       const uint8_t* src = pk_buf + sp * kPkBytes;
       uint8_t* dst = cv_buf + sc * C::kCvBytes;
+      QSPEC_TRACE_AT(i);
 #pragma unroll
       for (int it = 0; it < kPkBytes / 16 / (kConvWarps * 32); ++it) {
         const int ch = ct + it * kConvWarps * 32;   // 16-byte chunk of the packed tile
+        if (!QSPEC_ALIGN_OK(smem_u32(src + ch * 16), 16)) continue;
         const uint4 v = *reinterpret_cast<const uint4*>(src + ch * 16);
         const int r = ch >> 2;                      // weight row within the tile
         const int p = ch & 3;                       // which 32 input channels of the row
@@ -313,6 +331,9 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
           }
           uint8_t* row = dst + r * 128;
           const int c0 = 2 * p, c1 = 2 * p + 1;
+          if (!QSPEC_ALIGN_OK(smem_u32(row + ((c0 ^ (r & 7)) << 4)), 16) ||
+              !QSPEC_ALIGN_OK(smem_u32(row + ((c1 ^ (r & 7)) << 4)), 16))
+            continue;
           *reinterpret_cast<uint4*>(row + ((c0 ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
           *reinterpret_cast<uint4*>(row + ((c1 ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
         } else {
@@ -329,19 +350,21 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
             const uint32_t b2 = bf16x2_minus_136(prmt(t1, 0x43434343u, 0x4140u));
             const uint32_t b3 = bf16x2_minus_136(prmt(t1, 0x43434343u, 0x4342u));
             const int c = 4 * (p & 1) + wi;
+            if (!QSPEC_ALIGN_OK(smem_u32(row + ((c ^ (r & 7)) << 4)), 16)) continue;
             *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = make_uint4(b0, b1, b2, b3);
           }
         }
       }
       fence_proxy_async_smem();
       __syncwarp();
+      QSPEC_TRACE_AT(0x4000 | i);
       if (lane == 0) {
         mbar_arrive(smem_u32(&pk_empty[sp]));
         mbar_arrive(smem_u32(&cv_full[sc]));
       }
     }
-  } else {
-    // ------------------------------------------------ epilogue
+  } else if (warp >= kCtlWarps + kConvWarps) {
+    // ------------------------------------------------ epilogue (warp 3 is idle and lands nowhere)
     const int ew = warp - (kCtlWarps + kConvWarps);
     const int quad = warp & 3;                 // tensor-memory lanes this warp may read
     const int team = ew >> 2;
@@ -387,10 +410,11 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
           if (!ok) break;
           tc_fence_after();
           const uint32_t taddr = lane_addr + static_cast<uint32_t>(b * MT + col0);
+          QSPEC_TRACE_AT(j);
 #pragma unroll
           for (int c = 0; c < C::kCols; c += 8) {
-            uint32_t v[8];
-            tmem_ld8(taddr + c, v);
+            uint32_t v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            if (QSPEC_ALIGN_OK((taddr + c) & 0xFFFFu, 8)) tmem_ld8(taddr + c, v);
             tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -411,12 +435,14 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
           }
           tc_fence_before();
           __syncwarp();
+          QSPEC_TRACE_AT(0x4000 | j);
           if (lane == 0) mbar_arrive(smem_u32(&acc_empty[b]));
         }
       }
       if (!ok) break;
 
       const bool full = (seg_start == tile_u0) && (seg_end == tile_u0 + ku);
+      QSPEC_TRACE_AT(full ? 0x2001 : 0x2000);
       bool write_out = full;
       if (!full) {
         // Publish this CTA's share of the tile, then take a ticket.
@@ -429,11 +455,12 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
         const long long c_lo = unit_owner(tile_u0, units, grid);
         const long long c_hi = unit_owner(tile_u0 + ku - 1, units, grid);
         if (et == 0) {
-          const uint32_t old = atomicAdd(&args.counters[t], 1u);
+          const uint32_t old = atomicAdd(&args.counters[c_lo], 1u);
           *reducer_flag = (old == static_cast<uint32_t>(c_hi - c_lo)) ? 1 : 0;
         }
         if (!epi_barrier()) break;
         write_out = (*reducer_flag != 0);
+        QSPEC_TRACE_AT(write_out ? 0x3001 : 0x3000);
         if (write_out) {
           __threadfence();
 #pragma unroll
@@ -444,7 +471,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
 #pragma unroll
             for (int c = 0; c < C::kCols; ++c) run[c] += __ldcg(src + (col0 + c) * kTileN + row);
           }
-          if (et == 0) args.counters[t] = 0u;   // ready for the next launch
+          if (et == 0) args.counters[c_lo] = 0u;   // ready for the next launch
         }
       }
       if (write_out && n < args.N) {
@@ -460,12 +487,14 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     }
   }
 
+  QSPEC_TRACE_AT(0xFFF0);
   tc_fence_before();
   __syncthreads();
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
+  QSPEC_TRACE_AT(0xFFFF);
 }
 
 }  // namespace qspec

@@ -126,10 +126,14 @@ GemmPlan plan_gemm(bool int8_mode, int64_t m, int64_t n, int64_t k, int sm_count
   p.n_tiles = static_cast<int>((n + kTileN - 1) / kTileN);
   p.ku = static_cast<int>(k / kUnitK);
   p.units = static_cast<long long>(p.m_tiles) * p.n_tiles * p.ku;
-  p.grid = static_cast<int>(p.units < sm_count ? p.units : sm_count);
+  const int max_grid = sm_count < kMaxGrid ? sm_count : kMaxGrid;
+  p.grid = static_cast<int>(p.units < max_grid ? p.units : max_grid);
+  // Fixed-position regions first, so that calls of any shape sharing one
+  // workspace never see each other's scratch data in their status word or
+  // ticket slots; shape-dependent scratch follows.
   size_t off = 256;                                  // status word(s)
   p.off_counters = off;
-  off += round_up(static_cast<size_t>(p.m_tiles) * p.n_tiles * 4, 256);
+  off += static_cast<size_t>(kMaxGrid) * 4;
   p.off_partials = off;
   off += round_up(static_cast<size_t>(2) * p.grid * p.mt * kTileN * 4, 256);
   if (int8_mode) {
@@ -234,6 +238,12 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
 }  // namespace qspec
 
 using namespace qspec;
+
+#ifdef QSPEC_TRACE
+extern "C" int qspec_debug_set_trace(void* host_mapped) {
+  return cudaMemcpyToSymbol(g_qspec_trace, &host_mapped, sizeof(void*)) == cudaSuccess ? 0 : 1;
+}
+#endif
 
 extern "C" {
 

@@ -11,6 +11,8 @@
 #include <cuda_fp16.h>
 #include <cstdint>
 
+#include "device_common.cuh"
+
 namespace qspec {
 
 __device__ __forceinline__ int clamp_q(int v) { return v < -8 ? -8 : (v > 7 ? 7 : v); }
@@ -77,6 +79,10 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
   const int64_t row = blockIdx.x;
   const uint16_t* xr = x + row * k;
   const int tid = threadIdx.x;
+  QSPEC_TRACE_AT(1);
+  if (!QSPEC_ALIGN_OK(reinterpret_cast<uintptr_t>(xr), 16) ||
+      !QSPEC_ALIGN_OK(reinterpret_cast<uintptr_t>(out), 8))
+    return;
 
   float a = 0.f;
   for (int64_t c = static_cast<int64_t>(tid) * 8; c < k; c += 256 * 8) {

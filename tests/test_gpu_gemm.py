@@ -157,3 +157,23 @@ def test_shared_weights_are_one_buffer(qs):
     qs.gemm_w4a16(x, wq, ws, 128)
     torch.cuda.synchronize()
     assert torch.equal(before[0], wq) and torch.equal(before[1], ws)
+
+
+def test_one_workspace_shared_across_shapes(qs):
+    """Scratch left by a call of one shape must not disturb a call of another."""
+    shapes = [(4, 256, 256, 64), (16, 12288, 4096, 128), (80, 4096, 11008, 128), (3, 200, 256, 64),
+              (16, 12288, 4096, 128)]
+    need = max(qs.workspace_size(qs.OP_GEMM_W4A4, m, n, k, g) for (m, n, k, g) in shapes)
+    work = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for i, (m, n, k, g) in enumerate(shapes):
+        gi = synth.gemm_inputs("llama3_8b", m, n, k, g, stream=40 + i)
+        wq, ws = qs.quantize_weights(cuda_f32(gi.w), g)
+        x = cuda_bf16(gi.x_bits)
+        y4 = qs.gemm_w4a4(x, wq, ws, g, work=work)
+        y16 = qs.gemm_w4a16(x, wq, ws, g, work=work)
+        torch.cuda.synchronize()
+        cols = np.arange(0, n, max(1, n // 64))
+        q, s_h = orc.quantize_weights(gi.w[cols], g)
+        assert_close_1e3(y4.cpu().numpy()[:, cols], orc.gemm_w4a4(gi.x, q, s_h, g))
+        assert_close_1e3(y16.cpu().numpy()[:, cols], orc.gemm_w4a16(gi.x, q, s_h, g))
+        assert qs.workspace_status(work) == 0

@@ -90,3 +90,18 @@ def test_workspace_size_of_invalid_shapes_is_zero(lib):
     assert lib.workspace_size(lib.OP_GEMM_W4A4, 4, 256, 200, 64) == 0
     assert lib.workspace_size(lib.OP_QUANT_ACT, 4, 0, 256) == 0
     assert lib.workspace_size(lib.OP_SPEC_ACCEPT, batch=2, gamma=4, vocab=32) == 256
+
+
+def test_stream_k_schedule_invariants(tmp_path):
+    """Compile the scheduling helpers of the GEMM for the host and check the
+    partition, ticket and partial-slot invariants over many shapes."""
+    import subprocess
+    from quantized_speculative_decoding_packed_b200 import build as b
+    exe = tmp_path / "schedule_check"
+    src = os.path.join(ROOT, "tests", "schedule_check.cu")
+    cmd = [b.nvcc(), "-std=c++17", "-O1", "-gencode", "arch=compute_100a,code=sm_100a",
+           "-I", b.INCLUDE, "-I", b.CSRC, "-o", str(exe), src]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert run.returncode == 0 and run.stdout.startswith("ok"), run.stdout
