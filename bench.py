@@ -1,0 +1,465 @@
+#!/usr/bin/env python
+"""Benchmark of the shared-INT4 QSpec hot path on B200.
+
+One step = one draft-verify round over the linear layers of a
+Llama-2-7B-shaped decoder (32 layers x {fused QKV 12288x4096, o_proj
+4096x4096, gate+up 22016x4096, down 4096x11008}, group 128), all served from
+ONE packed INT4 weight set:
+  * gamma = 4 drafting passes, W4A4 at M = 16 (batch 16, one token each),
+  * one verifying pass, W4A16 at M = 80 (batch 16 x (gamma + 1)),
+  * the accept / residual-resample step for batch 16, gamma 4, vocab 32000.
+The step is captured once as a CUDA graph and replayed.  Weights (3.3 GB
+packed per pass) exceed the 126 MB L2 many times over, so every pass streams
+them from HBM.  Synthetic, seeded inputs; random-init weights.
+
+Prints ONE JSON line (rank 0).  `--impl reference` times the CPU oracle on a
+bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "shared-INT4-weight GEMM TOPS/GB/s (W4A4 draft, W4A16 verify) vs roofline"
+LAYERS = (("qkv", 12288, 4096), ("o_proj", 4096, 4096), ("gate_up", 22016, 4096),
+          ("down", 4096, 11008))
+GROUP = 128
+GAMMA = 4
+BATCH = 16
+M_DRAFT = BATCH
+M_VERIFY = BATCH * (GAMMA + 1)
+VOCAB = 32000
+N_LAYERS = 32
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("qspec", "reference"), default="qspec")
+    ap.add_argument("--layers", type=int, default=N_LAYERS,
+                    help="decoder layers (32 = the full model; smaller only for profiling)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- algorithmic bytes / ops
+def gemm_bytes(m, n, k, mode):
+    """Compulsory HBM bytes of one GEMM call: packed weights + fp16 scales +
+    activations as the kernel reads them + fp32 output."""
+    w = n * k // 2 + n * (k // GROUP) * 2
+    x = m * k * (1 if mode == "w4a4" else 2)
+    return w + x + m * n * 4
+
+
+def packed_bytes(n, k):
+    return n * k // 2 + n * (k // GROUP) * 2
+
+
+def accept_bytes(n_acc, gamma, vocab):
+    """Per sequence: 2 gathered elements per tested position, then one row of
+    p and q (rejection) or one row of p (bonus), plus the outputs."""
+    total = 0
+    for n in n_acc:
+        tested = min(int(n) + 1, gamma)
+        total += tested * 2 * 4 + (2 * vocab * 4 if n < gamma else vocab * 4) + (gamma + 2) * 4
+    return total
+
+
+def step_work(layers):
+    b = 0
+    ops = 0
+    for (_, n, k) in LAYERS:
+        b += layers * (GAMMA * gemm_bytes(M_DRAFT, n, k, "w4a4") + gemm_bytes(M_VERIFY, n, k, "w4a16"))
+        ops += layers * (GAMMA * 2 * M_DRAFT * n * k + 2 * M_VERIFY * n * k)
+    return b, ops
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running (read only)."""
+
+    def __init__(self, index):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        names = {getattr(nv, k): k for k in dir(nv) if k.startswith("nvmlClocksEventReason") or
+                 k.startswith("nvmlClocksThrottleReason")}
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                try:
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except Exception:
+                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                for bit, name in names.items():
+                    if isinstance(bit, int) and bit and (r & bit) == bit and bit != 0xFFFFFFFFFFFFFFFF:
+                        self.reasons.add(name.replace("nvmlClocksEventReason", "").replace(
+                            "nvmlClocksThrottleReason", ""))
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self._nv:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        reasons = sorted(r for r in self.reasons if r not in ("None", "All", "GpuIdle",
+                                                              "ApplicationsClocksSetting"))
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+def oracle_sample(columns=2048, seed=0):
+    """Time the oracle on `columns` output columns of every layer shape (both
+    modes) plus the full accept step; return (seconds per full step scaled
+    to the bench workload, description)."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import qspec_oracle as orc
+    from quantized_speculative_decoding_packed_b200 import synth
+
+    with threadpool_limits(limits=1):
+        t_step = 0.0
+        for si, (name, n, k) in enumerate(LAYERS):
+            c = min(columns, n)
+            rng = synth.rng_for("llama2_7b", 50 + seed, si)
+            w = synth.weights(rng, c, k)
+            outl = synth.outlier_channels(synth.rng_for("llama2_7b", 2, k), k)
+            x16 = synth.bf16_bits_to_f32(synth.activations(rng, M_DRAFT, k, outl))
+            x80 = synth.bf16_bits_to_f32(synth.activations(rng, M_VERIFY, k, outl))
+            q, s_h = orc.quantize_weights(w, GROUP)
+            t0 = time.perf_counter()
+            orc.gemm_w4a4(x16, q, s_h, GROUP)
+            t1 = time.perf_counter()
+            orc.gemm_w4a16(x80, q, s_h, GROUP)
+            t2 = time.perf_counter()
+            scale = n / c
+            t_step += N_LAYERS * scale * (GAMMA * (t1 - t0) + (t2 - t1))
+        ai = synth.accept_inputs(synth.rng_for("llama2_7b", 60 + seed), BATCH, GAMMA, VOCAB, 2.0, 0.5)
+        t0 = time.perf_counter()
+        n_acc, _ = orc.spec_accept(ai.p, ai.q, ai.draft, ai.u_acc, ai.u_res)
+        t_step += time.perf_counter() - t0
+    desc = (f"oracle on {columns} output columns of each of the 4 layer shapes (W4A4 at M=16, "
+            f"W4A16 at M=80) plus the full accept step, scaled by N/{columns} x 32 layers x "
+            f"({GAMMA}+1) passes; single thread")
+    return t_step, desc, n_acc
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    bytes_step, ops_step = step_work(N_LAYERS)
+    times = []
+    n_acc = None
+    for i in range(args.warmup + args.steps):
+        t, desc, n_acc = oracle_sample(columns=256, seed=i)
+        if i >= args.warmup:
+            times.append(t)
+    acc_b = accept_bytes(n_acc, GAMMA, VOCAB)
+    t = sum(times) / len(times)
+    value = (bytes_step + acc_b) / t / 1e9
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "impl": "reference", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64/f64",
+            "data": "synthetic", "config": workload_config(N_LAYERS),
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": desc.replace("2048", "256")},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def workload_config(layers):
+    return {"workload": "Llama-2-7B-shaped decode GEMMs, one QSpec round per step: "
+                        f"{layers} layers x (qkv 12288x4096, o_proj 4096x4096, gate_up 22016x4096, "
+                        f"down 4096x11008), gamma={GAMMA} W4A4 draft passes at M={M_DRAFT}, one W4A16 "
+                        f"verify pass at M={M_VERIFY}, accept B={BATCH} V={VOCAB}",
+            "layers": layers, "group": GROUP, "gamma": GAMMA, "draft_m": M_DRAFT,
+            "verify_m": M_VERIFY, "accept": {"batch": BATCH, "gamma": GAMMA, "vocab": VOCAB},
+            "l2": "inputs larger than L2 (packed weights of all layers streamed every pass)",
+            "parallelism": "replicas" }
+
+
+# ---------------------------------------------------------------- GPU arm
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    from quantized_speculative_decoding_packed_b200 import qspec
+
+    L = args.layers
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(20241015 + 1000 * rank)
+
+    # ---- one packed INT4 weight set, shared by both modes
+    wq = [[None] * len(LAYERS) for _ in range(L)]
+    ws = [[None] * len(LAYERS) for _ in range(L)]
+    for li in range(L):
+        for si, (_, n, k) in enumerate(LAYERS):
+            w = torch.randn((n, k), generator=gen, device=dev, dtype=torch.float32) * 0.02
+            wq[li][si], ws[li][si] = qspec.quantize_weights(w, GROUP)
+            del w
+    torch.cuda.synchronize()
+
+    def acts(m, k):
+        x = torch.randn((m, k), generator=gen, device=dev, dtype=torch.float32)
+        idx = torch.randperm(k, generator=gen, device=dev)[: round(0.01 * k)]
+        x[:, idx] *= 20.0
+        return x.to(torch.bfloat16)
+
+    x16 = [acts(M_DRAFT, k) for (_, n, k) in LAYERS]
+    x80 = [acts(M_VERIFY, k) for (_, n, k) in LAYERS]
+    y16 = [torch.empty((M_DRAFT, n), device=dev) for (_, n, k) in LAYERS]
+    y80 = [torch.empty((M_VERIFY, n), device=dev) for (_, n, k) in LAYERS]
+    need = max(max(qspec.workspace_size(qspec.OP_GEMM_W4A4, M_DRAFT, n, k, GROUP),
+                   qspec.workspace_size(qspec.OP_GEMM_W4A16, M_VERIFY, n, k, GROUP))
+               for (_, n, k) in LAYERS)
+    work = torch.zeros(need, dtype=torch.uint8, device=dev)
+    acc_work = torch.zeros(256, dtype=torch.uint8, device=dev)
+
+    # accept inputs: p, q softmaxes of N(0, 2^2) logits, q = p-logits + N(0, 0.5^2)
+    lp = torch.randn((BATCH, GAMMA + 1, VOCAB), generator=gen, device=dev, dtype=torch.float64) * 2
+    lq = lp[:, :GAMMA] + torch.randn((BATCH, GAMMA, VOCAB), generator=gen, device=dev,
+                                     dtype=torch.float64) * 0.5
+    p = torch.softmax(lp, -1).float().contiguous()
+    q = torch.softmax(lq, -1).float().contiguous()
+    draft = torch.multinomial(q.reshape(-1, VOCAB).double(), 1, generator=gen).reshape(
+        BATCH, GAMMA).to(torch.int32)
+    u_acc = (torch.randint(0, 1 << 24, (BATCH, GAMMA), generator=gen, device=dev).double()
+             / (1 << 24)).float()
+    u_res = (torch.randint(0, 1 << 24, (BATCH,), generator=gen, device=dev).double()
+             / (1 << 24)).float()
+    n_acc = torch.empty((BATCH,), dtype=torch.int32, device=dev)
+    tokens = torch.empty((BATCH, GAMMA + 1), dtype=torch.int32, device=dev)
+
+    # events bracketing a sample of launches inside the graph (layer 0 of each pass)
+    ev = {}
+
+    def mark(key):
+        e = ev.setdefault(key, torch.cuda.Event(enable_timing=True, external=True))
+        e.record()
+
+    def step(with_events):
+        for pss in range(GAMMA):
+            for li in range(L):
+                for si, (_, n, k) in enumerate(LAYERS):
+                    t = with_events and li == 0
+                    if t:
+                        mark(("w4a4", pss, si, 0))
+                    qspec.gemm_w4a4(x16[si], wq[li][si], ws[li][si], GROUP, y=y16[si], work=work)
+                    if t:
+                        mark(("w4a4", pss, si, 1))
+        for li in range(L):
+            for si, (_, n, k) in enumerate(LAYERS):
+                t = with_events and li == 0
+                if t:
+                    mark(("w4a16", 0, si, 0))
+                qspec.gemm_w4a16(x80[si], wq[li][si], ws[li][si], GROUP, y=y80[si], work=work)
+                if t:
+                    mark(("w4a16", 0, si, 1))
+        if with_events:
+            mark(("accept", 0, 0, 0))
+        qspec.spec_accept(p, q, draft, u_acc, u_res, n_accepted=n_acc, tokens=tokens, work=acc_work)
+        if with_events:
+            mark(("accept", 0, 0, 1))
+
+    launches_per_step = GAMMA * L * len(LAYERS) * 2 + L * len(LAYERS) + 1
+    stream = torch.cuda.Stream(device=dev)
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        step(False)                                  # eager first call: per-kernel setup
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream, capture_error_mode="thread_local"):
+            step(True)
+        for _ in range(max(args.warmup, 3)):
+            graph.replay()
+        stream.synchronize()
+        if qspec.workspace_status(work, stream) != 0:
+            raise RuntimeError("device status reported a fault during warm-up")
+
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        with ClockSampler(local) as clk:
+            start.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            end.record(stream)
+            end.synchronize()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        ms_total = start.elapsed_time(end)
+    ms_step = ms_total / args.steps
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+        ms_step = ms_total / args.steps
+
+    # per-kernel durations from the last timed step
+    def dur(kind, pss, si):
+        return ev[(kind, pss, si, 0)].elapsed_time(ev[(kind, pss, si, 1)])
+
+    kern = {}
+    w4a4_b = w4a4_t = 0.0
+    for si, (name, n, k) in enumerate(LAYERS):
+        t4 = [dur("w4a4", pss, si) for pss in range(GAMMA)]
+        t16 = dur("w4a16", 0, si)
+        b4, b16 = gemm_bytes(M_DRAFT, n, k, "w4a4"), gemm_bytes(M_VERIFY, n, k, "w4a16")
+        kern[name] = {"w4a4_us": 1e3 * statistics.mean(t4), "w4a4_gbs": b4 / (statistics.mean(t4) * 1e-3) / 1e9,
+                      "w4a4_tops": 2 * M_DRAFT * n * k / (statistics.mean(t4) * 1e-3) / 1e12,
+                      "w4a16_us": 1e3 * t16, "w4a16_gbs": b16 / (t16 * 1e-3) / 1e9,
+                      "w4a16_tflops": 2 * M_VERIFY * n * k / (t16 * 1e-3) / 1e12}
+        w4a4_b += b4 * GAMMA
+        w4a4_t += sum(t4)
+    t_acc = dur("accept", 0, 0)
+    acc_b = accept_bytes(n_acc.cpu().numpy(), GAMMA, VOCAB)
+    kern["accept"] = {"us": 1e3 * t_acc, "gbs": acc_b / (t_acc * 1e-3) / 1e9}
+
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+    except Exception:
+        pass
+    hbm_peak = peaks.get("hbm_gbs", 6650.0)
+    achieved = w4a4_b / (w4a4_t * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": traffic_from_profile(),
+                "kernel": "W4A4 drafting GEMM call (per-token quant pre-pass + qgemm_kernel<int8,16>)",
+                "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)" if "hbm_gbs" in peaks
+                else "fallback 6650 GB/s"}
+
+    bytes_step, ops_step = step_work(L)
+    bytes_step += acc_b
+    value = world * bytes_step / (ms_step * 1e-3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(torch, stream, graph, [x16, x80], [p, q, draft, u_acc, u_res],
+                          [n_acc, tokens], args.steps, bytes_step)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t_cpu, desc, _ = oracle_sample()
+        cpu = {"value": bytes_step / t_cpu / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": desc}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "s8/bf16", "data": "synthetic (seeded), random-init weights",
+                "config": workload_config(L),
+                "tops": world * ops_step / (ms_step * 1e-3) / 1e12,
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches_per_step * args.steps,
+                "clocks": clk.summary(), "kernels": kern}
+        print(json.dumps(line))
+    if world > 1:
+        del graph
+        dist.destroy_process_group()
+
+
+def measure_e2e(torch, stream, graph, acts, accept_in, outs, steps, bytes_step):
+    """Same step through the public API with host buffers: every step copies the
+    step's inputs from pinned host memory and reads the result back."""
+    host_in = [t.detach().cpu().pin_memory() for group in acts for t in group] + \
+              [t.detach().cpu().pin_memory() for t in accept_in]
+    dev_in = [t for group in acts for t in group] + list(accept_in)
+    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        torch.cuda.synchronize()
+        start.record(stream)
+        for _ in range(steps):
+            for d, h in zip(dev_in, host_in):
+                d.copy_(h, non_blocking=True)
+            graph.replay()
+            for h, d in zip(host_out, outs):
+                h.copy_(d, non_blocking=True)
+        end.record(stream)
+        end.synchronize()
+    ms = start.elapsed_time(end) / steps
+    return {"value": bytes_step / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def traffic_from_profile():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current GEMM source; else null."""
+    path = os.path.join(ROOT, "profiles", "qgemm_w4a4_llama2_7b_gate_up_m16.json")
+    src = os.path.join(ROOT, "quantized_speculative_decoding_packed_b200", "csrc", "gemm.cuh")
+    try:
+        with open(path) as f:
+            prof = json.load(f)
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        if prof.get("gemm_source_sha256") == sha:
+            return prof.get("dram_bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+if __name__ == "__main__":
+    main()

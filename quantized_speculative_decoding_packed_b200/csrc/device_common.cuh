@@ -22,6 +22,26 @@ static __device__ unsigned int* g_qspec_trace = nullptr;
       __threadfence_system();                                                           \
     }                                                                                   \
   } while (0)
+// Timeline stamps (SM clock, low 32 bits) per event and unit, kept in shared
+// memory (one st.shared each) and copied to [cta][16][64] at kernel exit.
+static __device__ unsigned long long* g_qspec_timeline = nullptr;
+#define QSPEC_STAMP_DECL __shared__ unsigned int s_qspec_stamps[16 * 64];
+#define QSPEC_STAMP(ev, unit)                                                           \
+  do {                                                                                  \
+    if ((unit) < 64) s_qspec_stamps[(ev) * 64 + (unit)] = static_cast<unsigned>(clock64()); \
+  } while (0)
+#define QSPEC_STAMP_FLUSH()                                                             \
+  do {                                                                                  \
+    if (g_qspec_timeline)                                                               \
+      for (int q_ = threadIdx.x; q_ < 16 * 64; q_ += blockDim.x)                        \
+        g_qspec_timeline[blockIdx.x * 1024u + q_] = s_qspec_stamps[q_];                 \
+  } while (0)
+// Coarse phase stamps (global timer, ns, comparable across SMs): [cta][16].
+static __device__ unsigned long long* g_qspec_phases = nullptr;
+#define QSPEC_PHASE(ev)                                                                 \
+  do {                                                                                  \
+    if (g_qspec_phases) g_qspec_phases[blockIdx.x * 16u + (ev)] = global_timer_ns();    \
+  } while (0)
 #define QSPEC_ALIGN_OK(addr, a)                                                          \
   ((static_cast<unsigned long long>(addr) % (a)) == 0 ||                                 \
    (g_qspec_trace && (g_qspec_trace[8191] = (0xA0000000u | __LINE__), __threadfence_system(), false)))
@@ -30,6 +50,16 @@ static __device__ unsigned int* g_qspec_trace = nullptr;
   do {                       \
   } while (0)
 #define QSPEC_ALIGN_OK(addr, a) true
+#define QSPEC_STAMP(ev, unit) \
+  do {                        \
+  } while (0)
+#define QSPEC_PHASE(ev) \
+  do {                  \
+  } while (0)
+#define QSPEC_STAMP_DECL
+#define QSPEC_STAMP_FLUSH() \
+  do {                      \
+  } while (0)
 #endif
 
 namespace qspec {
@@ -82,27 +112,55 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread sleeps in hardware until the
+// phase completes or the hint (ns) expires, instead of spinning on shared
+// memory and stealing issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete.  Returns false (and
 // raises the CTA-wide abort flag and the device status word) if the wait
 // runs past kWaitLimitNs or another thread of the CTA has already aborted.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           uint32_t* status) {
   if (mbar_try_wait(bar, parity)) return true;
-  uint64_t start = 0;
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0u) {
-      if (*abort_flag) return false;
-      const uint64_t now = global_timer_ns();
-      if (start == 0) {
-        start = now;
-      } else if (now - start > kWaitLimitNs) {
-        *abort_flag = 1;
-        if (status) atomicOr(status, kDevTimeout);
-        return false;
-      }
+  const uint64_t start = global_timer_ns();
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;   // sleeps <= 0.2 ms
+    if (*abort_flag) return false;
+    if (global_timer_ns() - start > kWaitLimitNs) {
+      *abort_flag = 1;
+      if (status) atomicOr(status, kDevTimeout);
+      return false;
     }
   }
+}
+
+// Warp-level wait: every lane polls (one warp-wide instruction per poll, no
+// divergent region -- a lane-0-only branch costs far more than the poll) and
+// the warp agrees on the outcome.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          uint32_t* status) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status));
+}
+
+// True in exactly one lane of a converged warp.
+__device__ __forceinline__ bool elect_one_lane() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
 }
 
 // Short bounded wait used while draining copies on the abort path.

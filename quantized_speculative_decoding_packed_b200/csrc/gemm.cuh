@@ -29,12 +29,16 @@
 // is indexed by its first contributor; tickets return to zero after use.
 //
 // Warp roles (one CTA per SM):
-//   warp 0      TMA producer for packed weight tiles (8-stage ring, 8 KB each)
-//   warp 1      TMA producer for activation tiles (128-byte swizzled)
+//   warp 0      TMA producer for packed weight tiles (ring of up to 16 x 8 KB)
+//   warp 1      TMA producer for activation tiles (128-byte swizzled ring)
 //   warp 2      tensor-memory allocation and the single MMA-issuing thread
 //   warp 3      idle
 //   8 warps     converters: packed nibbles -> int8 / bf16 operand tiles
 //   4..16 warps epilogue: tensor memory -> registers, group scales, output
+//
+// Three independent rings decouple the latencies: packed weights (HBM
+// latency), widened weights (converter -> tensor core) and activations (L2
+// latency); a 4-deep tensor-memory ring decouples the MMAs from the epilogue.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -48,18 +52,19 @@ namespace qspec {
 constexpr int kTileN = 128;                      // weight rows per tile (MMA M)
 constexpr int kUnitK = 128;                      // input channels per unit
 constexpr int kPkBytes = kTileN * kUnitK / 2;    // packed bytes per unit
-constexpr int kNumPk = 8;                        // packed-weight ring depth
 constexpr int kNumAcc = 4;                       // tensor-memory group ring
 constexpr int kConvWarps = 8;
 constexpr int kCtlWarps = 4;
 constexpr int kSmemLimit = 232448;               // sm_100 dynamic shared memory per CTA
 constexpr int kMaxGrid = 1024;                   // ticket slots in the workspace
+constexpr int kMaxPk = 16, kMaxCv = 4, kMaxX = 8;
 
 __host__ __device__ constexpr int pow2_at_least(int v) {
   int p = 32;
   while (p < v) p <<= 1;
   return p;
 }
+__host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 
 template <bool kInt8, int MT>
 struct GemmCfg {
@@ -76,12 +81,16 @@ struct GemmCfg {
   static_assert(kCols % 8 == 0, "epilogue columns must be a multiple of 8");
   static constexpr int kWarps = kCtlWarps + kConvWarps + kEpiWarps;
   static constexpr int kThreads = 32 * kWarps;
-  static constexpr int kBarBytes = 512;
-  static constexpr int kRingBytes = kCvBytes + kXBytes;
-  static constexpr int kNumCvRaw = (kSmemLimit - 1024 - kBarBytes - kNumPk * kPkBytes) / kRingBytes;
-  static constexpr int kNumCv = kNumCvRaw > 4 ? 4 : kNumCvRaw;
-  static_assert(kNumCv >= 2, "shared memory too small for a double-buffered operand ring");
-  static constexpr int kSmemBytes = 1024 + kNumPk * kPkBytes + kNumCv * kRingBytes + kBarBytes;
+  static constexpr int kBarBytes = 1024;
+  // ring depths from the shared-memory budget
+  static constexpr int kNumCv = (!kInt8 && MT >= 64) ? 2 : 4;
+  static constexpr int kAvail = kSmemLimit - 1024 - kBarBytes - kNumCv * kCvBytes;
+  static constexpr int kNumX = cmin(kMaxX, (kAvail - 6 * kPkBytes) / kXBytes);
+  static constexpr int kNumPk = cmin(kMaxPk, (kAvail - kNumX * kXBytes) / kPkBytes);
+  static_assert(kNumX >= 2 && kNumPk >= 6, "shared memory too small for the rings");
+  static constexpr int kSmemBytes =
+      1024 + kNumPk * kPkBytes + kNumCv * kCvBytes + kNumX * kXBytes + kBarBytes;
+  static_assert(kSmemBytes <= kSmemLimit, "shared memory overflow");
   static constexpr int kTmemCols = pow2_at_least(kNumAcc * MT);
   static_assert(kTmemCols <= 512, "tensor memory overflow");
 };
@@ -128,24 +137,57 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* v) {
       : "memory");
 }
 
+// Coordinates of a unit, advanced without divisions inside the hot loops
+// (64-bit integer division is a long software sequence on the GPU).
+struct UnitCursor {
+  int kc, m_tile, n_tile;
+  __device__ __forceinline__ void init(long long u, int ku, int m_tiles) {
+    const long long t = u / ku;
+    kc = static_cast<int>(u - t * ku);
+    n_tile = static_cast<int>(t / m_tiles);
+    m_tile = static_cast<int>(t - static_cast<long long>(n_tile) * m_tiles);
+  }
+  __device__ __forceinline__ void next(int ku, int m_tiles) {
+    if (++kc == ku) {
+      kc = 0;
+      if (++m_tile == m_tiles) {
+        m_tile = 0;
+        ++n_tile;
+      }
+    }
+  }
+};
+
+// Programmatic dependent launch: wait for the grid this one depends on (a
+// no-op when launched without the attribute); let dependents start early.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 template <bool kInt8, int MT>
 __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     qgemm_kernel(const __grid_constant__ CUtensorMap tmap_w,
                  const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args) {
   using C = GemmCfg<kInt8, MT>;
+  constexpr int NPK = C::kNumPk, NCV = C::kNumCv, NX = C::kNumX;
   extern __shared__ uint8_t smem_raw[];
+  QSPEC_STAMP_DECL
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* pk_buf = smem;
-  uint8_t* cv_buf = pk_buf + kNumPk * kPkBytes;
-  uint8_t* x_buf = cv_buf + C::kNumCv * C::kCvBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(x_buf + C::kNumCv * C::kXBytes);
+  uint8_t* cv_buf = pk_buf + NPK * kPkBytes;
+  uint8_t* x_buf = cv_buf + NCV * C::kCvBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(x_buf + NX * C::kXBytes);
   uint64_t* pk_full = bars;
-  uint64_t* pk_empty = pk_full + kNumPk;
-  uint64_t* cv_full = pk_empty + kNumPk;
-  uint64_t* x_full = cv_full + 4;
-  uint64_t* cv_empty = x_full + 4;
-  uint64_t* acc_full = cv_empty + 4;
+  uint64_t* pk_empty = pk_full + kMaxPk;
+  uint64_t* cv_full = pk_empty + kMaxPk;
+  uint64_t* cv_empty = cv_full + kMaxCv;
+  uint64_t* x_full = cv_empty + kMaxCv;
+  uint64_t* x_empty = x_full + kMaxX;
+  uint64_t* acc_full = x_empty + kMaxX;
   uint64_t* acc_empty = acc_full + kNumAcc;
   uint64_t* mma_done = acc_empty + kNumAcc;
   uint64_t* epi_sync = mma_done + 1;
@@ -163,15 +205,19 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   const int ku = args.ku;
   const int gpu = args.groups_per_unit;
 
+  if (threadIdx.x == 0) QSPEC_PHASE(0);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kNumPk; ++s) {
+    for (int s = 0; s < NPK; ++s) {
       mbar_init(smem_u32(&pk_full[s]), 1);
       mbar_init(smem_u32(&pk_empty[s]), kConvWarps);
     }
-    for (int s = 0; s < C::kNumCv; ++s) {
+    for (int s = 0; s < NCV; ++s) {
       mbar_init(smem_u32(&cv_full[s]), kConvWarps);
-      mbar_init(smem_u32(&x_full[s]), 1);
       mbar_init(smem_u32(&cv_empty[s]), 1);
+    }
+    for (int s = 0; s < NX; ++s) {
+      mbar_init(smem_u32(&x_full[s]), 1);
+      mbar_init(smem_u32(&x_empty[s]), 1);
     }
     for (int b = 0; b < kNumAcc; ++b) {
       mbar_init(smem_u32(&acc_full[b]), 1);
@@ -196,122 +242,129 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = misc[0];
   QSPEC_TRACE_AT(tmem_base & 0xFFFF);
-  if (!QSPEC_ALIGN_OK(smem_u32(smem), 1024) || !QSPEC_ALIGN_OK(smem_u32(bars), 8)) *abort_flag = 1;
+  if (threadIdx.x == 0) QSPEC_PHASE(1);
 
   if (warp == 0) {
     // ------------------------------------------------ packed-weight producer
-    if (lane == 0) {
-      int i = 0;
-      for (long long u = u_begin; u < u_end; ++u, ++i) {
-        const int s = i % kNumPk;
-        const uint32_t ph = (i / kNumPk) & 1;
-        if (!mbar_wait(smem_u32(&pk_empty[s]), ph ^ 1, abort_flag, args.status)) break;
-        const long long t = u / ku;
-        const int kc = static_cast<int>(u - t * ku);
-        const int n_tile = static_cast<int>(t / args.m_tiles);
-        QSPEC_TRACE_AT(i);
-        if (!QSPEC_ALIGN_OK(smem_u32(pk_buf + s * kPkBytes), 128)) break;
+    // (the whole warp walks the loop; an elected lane issues the copies)
+    int i = 0;
+    UnitCursor cur;
+    cur.init(u_begin, ku, args.m_tiles);
+    for (long long u = u_begin; u < u_end; ++u, ++i, cur.next(ku, args.m_tiles)) {
+      const int s = i % NPK;
+      const uint32_t ph = (i / NPK) & 1;
+      if (!warp_wait(smem_u32(&pk_empty[s]), ph ^ 1, abort_flag, args.status)) break;
+      if (elect_one_lane()) {
         mbar_arrive_expect_tx(smem_u32(&pk_full[s]), kPkBytes);
         tma_load_2d(smem_u32(pk_buf + s * kPkBytes), &tmap_w, smem_u32(&pk_full[s]),
-                    kc * (kUnitK / 2), n_tile * kTileN);
+                    cur.kc * (kUnitK / 2), cur.n_tile * kTileN);
       }
-      if (*abort_flag) {
-        for (int j = (i > kNumPk ? i - kNumPk : 0); j < i; ++j)
-          mbar_wait_drain(smem_u32(&pk_full[j % kNumPk]), (j / kNumPk) & 1);
-      }
+      __syncwarp();
+      QSPEC_STAMP(0, i);
+    }
+    if (*abort_flag) {
+      for (int j = (i > NPK ? i - NPK : 0); j < i; ++j)
+        mbar_wait_drain(smem_u32(&pk_full[j % NPK]), (j / NPK) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ activation producer
-    if (lane == 0) {
-      int i = 0;
-      for (long long u = u_begin; u < u_end; ++u, ++i) {
-        const int s = i % C::kNumCv;
-        const uint32_t ph = (i / C::kNumCv) & 1;
-        if (!mbar_wait(smem_u32(&cv_empty[s]), ph ^ 1, abort_flag, args.status)) break;
-        const long long t = u / ku;
-        const int kc = static_cast<int>(u - t * ku);
-        const int m_tile = static_cast<int>(t % args.m_tiles);
-        QSPEC_TRACE_AT(i);
-        if (!QSPEC_ALIGN_OK(smem_u32(x_buf + s * C::kXBytes), 1024)) break;
+    grid_dependency_wait();   // activations may come from the preceding kernel
+    int i = 0;
+    UnitCursor cur;
+    cur.init(u_begin, ku, args.m_tiles);
+    for (long long u = u_begin; u < u_end; ++u, ++i, cur.next(ku, args.m_tiles)) {
+      const int s = i % NX;
+      const uint32_t ph = (i / NX) & 1;
+      if (!warp_wait(smem_u32(&x_empty[s]), ph ^ 1, abort_flag, args.status)) break;
+      if (elect_one_lane()) {
         mbar_arrive_expect_tx(smem_u32(&x_full[s]), C::kXBytes);
 #pragma unroll
         for (int a = 0; a < C::kAtoms; ++a) {
           tma_load_2d(smem_u32(x_buf + s * C::kXBytes + a * MT * 128), &tmap_x,
-                      smem_u32(&x_full[s]), kc * kUnitK + a * (128 / C::kElem), m_tile * MT);
+                      smem_u32(&x_full[s]), cur.kc * kUnitK + a * (128 / C::kElem),
+                      cur.m_tile * MT);
         }
       }
-      if (*abort_flag) {
-        for (int j = (i > C::kNumCv ? i - C::kNumCv : 0); j < i; ++j)
-          mbar_wait_drain(smem_u32(&x_full[j % C::kNumCv]), (j / C::kNumCv) & 1);
-      }
+      __syncwarp();
+      QSPEC_STAMP(7, i);
+    }
+    if (*abort_flag) {
+      for (int j = (i > NX ? i - NX : 0); j < i; ++j)
+        mbar_wait_drain(smem_u32(&x_full[j % NX]), (j / NX) & 1);
     }
   } else if (warp == 2) {
     // ------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = kInt8 ? idesc_i8(MT) : idesc_bf16(MT);
-      const int per_group = C::kMmas / gpu;
-      int i = 0, j = 0;
-      bool ok = true;
-      for (long long u = u_begin; u < u_end && ok; ++u, ++i) {
-        const int s = i % C::kNumCv;
-        const uint32_t ph = (i / C::kNumCv) & 1;
-        if (!mbar_wait(smem_u32(&cv_full[s]), ph, abort_flag, args.status)) break;
-        if (!mbar_wait(smem_u32(&x_full[s]), ph, abort_flag, args.status)) break;
+    // The whole warp walks the loop (waits are warp-uniform); one elected lane
+    // issues each tcgen05 instruction, which is cheaper than a lone lane.
+    constexpr uint32_t idesc = kInt8 ? idesc_i8(MT) : idesc_bf16(MT);
+    const int per_group = C::kMmas / gpu;
+    int i = 0, j = 0;
+    bool ok = true;
+    for (long long u = u_begin; u < u_end && ok; ++u, ++i) {
+      const int sc = i % NCV;
+      const int sx = i % NX;
+      QSPEC_STAMP(13, i);
+      ok = warp_wait(smem_u32(&cv_full[sc]), (i / NCV) & 1, abort_flag, args.status);
+      QSPEC_STAMP(14, i);
+      ok = ok && warp_wait(smem_u32(&x_full[sx]), (i / NX) & 1, abort_flag, args.status);
+      if (!ok) break;
+      QSPEC_STAMP(3, i);
+      tc_fence_after();
+      const uint32_t a_base = smem_u32(cv_buf + sc * C::kCvBytes);
+      const uint32_t b_base = smem_u32(x_buf + sx * C::kXBytes);
+      for (int h = 0; h < gpu; ++h, ++j) {
+        const int b = j % kNumAcc;
+        const uint32_t pha = (j / kNumAcc) & 1;
+        ok = warp_wait(smem_u32(&acc_empty[b]), pha ^ 1, abort_flag, args.status);
+        if (!ok) break;
         tc_fence_after();
-        QSPEC_TRACE_AT(i);
-        const uint32_t a_base = smem_u32(cv_buf + s * C::kCvBytes);
-        const uint32_t b_base = smem_u32(x_buf + s * C::kXBytes);
-        for (int h = 0; h < gpu; ++h, ++j) {
-          const int b = j % kNumAcc;
-          const uint32_t pha = (j / kNumAcc) & 1;
-          if (!mbar_wait(smem_u32(&acc_empty[b]), pha ^ 1, abort_flag, args.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          for (int kk = 0; kk < per_group; ++kk) {
-            const uint32_t kbyte = static_cast<uint32_t>(h * per_group + kk) * 32u;
-            const uint32_t atom = kbyte >> 7, within = kbyte & 127u;
-            const uint64_t a_desc = smem_desc_sw128(a_base + atom * (kTileN * 128) + within);
-            const uint64_t b_desc = smem_desc_sw128(b_base + atom * (MT * 128) + within);
-            QSPEC_TRACE_AT(0x8000 | (j << 4) | kk);
-            if (!QSPEC_ALIGN_OK(a_base + atom * (kTileN * 128) + within, 16) ||
-                !QSPEC_ALIGN_OK(b_base + atom * (MT * 128) + within, 16) ||
-                !QSPEC_ALIGN_OK(static_cast<uint32_t>(b * MT) & 0xFFFFu, 8))
-              continue;
+        if (h == 0) QSPEC_STAMP(8, i);
+        for (int kk = 0; kk < per_group; ++kk) {
+          const uint32_t kbyte = static_cast<uint32_t>(h * per_group + kk) * 32u;
+          const uint32_t atom = kbyte >> 7, within = kbyte & 127u;
+          const uint64_t a_desc = smem_desc_sw128(a_base + atom * (kTileN * 128) + within);
+          const uint64_t b_desc = smem_desc_sw128(b_base + atom * (MT * 128) + within);
+          if (elect_one_lane())
             mma_ss<kInt8>(tmem_base + static_cast<uint32_t>(b * MT), a_desc, b_desc, idesc,
                           kk > 0 ? 1u : 0u);
-          }
-          mma_commit(smem_u32(&acc_full[b]));
-          QSPEC_TRACE_AT(0x4000 | j);
+          __syncwarp();
+          if (h == 0 && (kk == 0 || kk == per_group - 1)) QSPEC_STAMP(kk == 0 ? 9 : 11, i);
         }
-        if (!ok) break;
-        mma_commit(smem_u32(&cv_empty[s]));
+        if (elect_one_lane()) mma_commit(smem_u32(&acc_full[b]));
+        __syncwarp();
+        if (h == 0) QSPEC_STAMP(12, i);
       }
-      // All MMAs this thread issued have finished once mma_done completes.
-      mma_commit(smem_u32(mma_done));
-      mbar_wait_drain(smem_u32(mma_done), 0);
+      if (!ok) break;
+      if (elect_one_lane()) {
+        mma_commit(smem_u32(&cv_empty[sc]));
+        mma_commit(smem_u32(&x_empty[sx]));
+      }
+      __syncwarp();
+      QSPEC_STAMP(4, i);
+      if (i == 0 && lane == 0) QSPEC_PHASE(3);
     }
+    // All MMAs this warp issued have finished once mma_done completes.
+    if (elect_one_lane()) mma_commit(smem_u32(mma_done));
+    __syncwarp();
+    mbar_wait_drain(smem_u32(mma_done), 0);
     __syncwarp();
   } else if (warp >= kCtlWarps && warp < kCtlWarps + kConvWarps) {
     // ------------------------------------------------ converters
     const int ct = threadIdx.x - kCtlWarps * 32;
     int i = 0;
     for (long long u = u_begin; u < u_end; ++u, ++i) {
-      const int sp = i % kNumPk;
-      const uint32_t php = (i / kNumPk) & 1;
-      const int sc = i % C::kNumCv;
-      const uint32_t phc = (i / C::kNumCv) & 1;
-      bool ok = mbar_wait(smem_u32(&pk_full[sp]), php, abort_flag, args.status);
-      ok = ok && mbar_wait(smem_u32(&cv_empty[sc]), phc ^ 1, abort_flag, args.status);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      const int sp = i % NPK;
+      const int sc = i % NCV;
+      bool ok = warp_wait(smem_u32(&pk_full[sp]), (i / NPK) & 1, abort_flag, args.status);
+      ok = ok && warp_wait(smem_u32(&cv_empty[sc]), ((i / NCV) & 1) ^ 1, abort_flag, args.status);
+      if (!ok) break;
+      if (warp == kCtlWarps) QSPEC_STAMP(1, i);
+      if (i == 0 && ct == 0) QSPEC_PHASE(2);
       const uint8_t* src = pk_buf + sp * kPkBytes;
       uint8_t* dst = cv_buf + sc * C::kCvBytes;
-      QSPEC_TRACE_AT(i);
 #pragma unroll
       for (int it = 0; it < kPkBytes / 16 / (kConvWarps * 32); ++it) {
         const int ch = ct + it * kConvWarps * 32;   // 16-byte chunk of the packed tile
-        if (!QSPEC_ALIGN_OK(smem_u32(src + ch * 16), 16)) continue;
         const uint4 v = *reinterpret_cast<const uint4*>(src + ch * 16);
         const int r = ch >> 2;                      // weight row within the tile
         const int p = ch & 3;                       // which 32 input channels of the row
@@ -331,9 +384,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
           }
           uint8_t* row = dst + r * 128;
           const int c0 = 2 * p, c1 = 2 * p + 1;
-          if (!QSPEC_ALIGN_OK(smem_u32(row + ((c0 ^ (r & 7)) << 4)), 16) ||
-              !QSPEC_ALIGN_OK(smem_u32(row + ((c1 ^ (r & 7)) << 4)), 16))
-            continue;
           *reinterpret_cast<uint4*>(row + ((c0 ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
           *reinterpret_cast<uint4*>(row + ((c1 ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
         } else {
@@ -350,18 +400,18 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
             const uint32_t b2 = bf16x2_minus_136(prmt(t1, 0x43434343u, 0x4140u));
             const uint32_t b3 = bf16x2_minus_136(prmt(t1, 0x43434343u, 0x4342u));
             const int c = 4 * (p & 1) + wi;
-            if (!QSPEC_ALIGN_OK(smem_u32(row + ((c ^ (r & 7)) << 4)), 16)) continue;
             *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = make_uint4(b0, b1, b2, b3);
           }
         }
       }
       fence_proxy_async_smem();
       __syncwarp();
-      QSPEC_TRACE_AT(0x4000 | i);
-      if (lane == 0) {
+      if (elect_one_lane()) {
         mbar_arrive(smem_u32(&pk_empty[sp]));
         mbar_arrive(smem_u32(&cv_full[sc]));
       }
+      __syncwarp();
+      if (warp == kCtlWarps) QSPEC_STAMP(2, i);
     }
   } else if (warp >= kCtlWarps + kConvWarps) {
     // ------------------------------------------------ epilogue (warp 3 is idle and lands nowhere)
@@ -373,6 +423,33 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     const int et = ew * 32 + lane;             // 0 .. kEpiWarps*32-1
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     volatile int* reducer_flag = reinterpret_cast<volatile int*>(&misc[2]);
+
+    // Group scales are read from global memory four groups ahead of use; a
+    // second cursor walks the CTA's groups for the prefetch.
+    const int groups_total = static_cast<int>(u_end - u_begin) * gpu;
+    UnitCursor pf;
+    pf.init(u_begin, ku, args.m_tiles);
+    int pf_h = 0, pf_j = 0;
+    auto next_scale = [&]() -> float {
+      float v = 0.f;
+      if (pf_j < groups_total) {
+        const int nn = pf.n_tile * kTileN + row;
+        if (nn < args.N)
+          v = __half2float(__ushort_as_half(
+              __ldg(args.ws + static_cast<long long>(nn) * args.groups_per_row + pf.kc * gpu + pf_h)));
+        ++pf_j;
+        if (++pf_h == gpu) {
+          pf_h = 0;
+          pf.next(ku, args.m_tiles);
+        }
+      }
+      return v;
+    };
+    float sq0 = next_scale();
+    float sq1 = next_scale();
+    float sq2 = next_scale();
+    float sq3 = next_scale();
+
     float run[C::kCols];
     int j = 0;
     bool ok = true;
@@ -380,69 +457,80 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     // All epilogue warps meet here; bounded, unlike a hardware named barrier.
     auto epi_barrier = [&]() -> bool {
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(epi_sync));
-      const bool fine = __all_sync(0xffffffffu, mbar_wait(smem_u32(epi_sync), epi_phase, abort_flag, args.status));
+      if (elect_one_lane()) mbar_arrive(smem_u32(epi_sync));
+      __syncwarp();
+      const bool fine = warp_wait(smem_u32(epi_sync), epi_phase, abort_flag, args.status);
       epi_phase ^= 1u;
       return fine;
     };
     long long u = u_begin;
+    UnitCursor cur;
+    cur.init(u_begin, ku, args.m_tiles);
     while (u < u_end && ok) {
-      const long long t = u / ku;
+      const long long t = static_cast<long long>(cur.n_tile) * args.m_tiles + cur.m_tile;
       const long long seg_start = u;
       const long long tile_u0 = t * ku;
       const long long seg_end = (u_end < tile_u0 + ku) ? u_end : tile_u0 + ku;
-      const int n_tile = static_cast<int>(t / args.m_tiles);
-      const int m_tile = static_cast<int>(t - static_cast<long long>(n_tile) * args.m_tiles);
-      const int n = n_tile * kTileN + row;
-      const int m0 = m_tile * MT + col0;
+      const int n = cur.n_tile * kTileN + row;
+      const int m0 = cur.m_tile * MT + col0;
 #pragma unroll
       for (int c = 0; c < C::kCols; ++c) run[c] = 0.f;
-      for (; u < seg_end && ok; ++u) {
-        const int kc = static_cast<int>(u - tile_u0);
+      for (; u < seg_end && ok; ++u, cur.next(ku, args.m_tiles)) {
+        const int kc = cur.kc;
         for (int h = 0; h < gpu; ++h, ++j) {
           const int b = j % kNumAcc;
           const uint32_t pha = (j / kNumAcc) & 1;
           const int g = kc * gpu + h;
-          const float sc = (n < args.N)
-                               ? __half2float(__ushort_as_half(args.ws[static_cast<long long>(n) * args.groups_per_row + g]))
-                               : 0.f;
-          ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_full[b]), pha, abort_flag, args.status));
+          const float sc = sq0;
+          sq0 = sq1;
+          sq1 = sq2;
+          sq2 = sq3;
+          sq3 = next_scale();
+          ok = warp_wait(smem_u32(&acc_full[b]), pha, abort_flag, args.status);
           if (!ok) break;
+          if (ew == 0) QSPEC_STAMP(5, j);
           tc_fence_after();
           const uint32_t taddr = lane_addr + static_cast<uint32_t>(b * MT + col0);
-          QSPEC_TRACE_AT(j);
 #pragma unroll
-          for (int c = 0; c < C::kCols; c += 8) {
-            uint32_t v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            if (QSPEC_ALIGN_OK((taddr + c) & 0xFFFFu, 8)) tmem_ld8(taddr + c, v);
+          for (int c0 = 0; c0 < C::kCols; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld8(taddr + c0, v);
+            if (c0 + 8 < C::kCols) tmem_ld8(taddr + c0 + 8, v + 8);
             tmem_ld_wait();
+            if (c0 + 16 >= C::kCols) {
+              // all columns of this group are in registers: hand the buffer back
+              tc_fence_before();
+              __syncwarp();
+              if (elect_one_lane()) mbar_arrive(smem_u32(&acc_empty[b]));
+              __syncwarp();
+              if (ew == 0) QSPEC_STAMP(6, j);
+              if (et == 0 && j == 0) QSPEC_PHASE(4);
+            }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float a = kInt8 ? static_cast<float>(static_cast<int>(v[e])) : __uint_as_float(v[e]);
-              run[c + e] = fmaf(sc, a, run[c + e]);
+            for (int e = 0; e < 16; ++e) {
+              if (c0 + e < C::kCols) {
+                const float a = kInt8 ? static_cast<float>(static_cast<int>(v[e])) : __uint_as_float(v[e]);
+                run[c0 + e] = fmaf(sc, a, run[c0 + e]);
+              }
             }
             if constexpr (kInt8) {
               if (args.dbg_acc != nullptr && n < args.N) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                  const int m = m0 + c + e;
-                  if (m < args.M)
+                for (int e = 0; e < 16; ++e) {
+                  const int m = m0 + c0 + e;
+                  if (c0 + e < C::kCols && m < args.M)
                     args.dbg_acc[(static_cast<long long>(m) * args.N + n) * args.groups_per_row + g] =
                         static_cast<int>(v[e]);
                 }
               }
             }
           }
-          tc_fence_before();
-          __syncwarp();
-          QSPEC_TRACE_AT(0x4000 | j);
-          if (lane == 0) mbar_arrive(smem_u32(&acc_empty[b]));
         }
       }
       if (!ok) break;
+      if (et == 0) QSPEC_PHASE(u >= u_end ? 5 : 7);
 
       const bool full = (seg_start == tile_u0) && (seg_end == tile_u0 + ku);
-      QSPEC_TRACE_AT(full ? 0x2001 : 0x2000);
       bool write_out = full;
       if (!full) {
         // Publish this CTA's share of the tile, then take a ticket.
@@ -460,7 +548,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
         }
         if (!epi_barrier()) break;
         write_out = (*reducer_flag != 0);
-        QSPEC_TRACE_AT(write_out ? 0x3001 : 0x3000);
         if (write_out) {
           __threadfence();
 #pragma unroll
@@ -475,6 +562,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
         }
       }
       if (write_out && n < args.N) {
+        if constexpr (kInt8) grid_dependency_wait();   // s_a comes from the preceding kernel
 #pragma unroll
         for (int c = 0; c < C::kCols; ++c) {
           const int m = m0 + c;
@@ -488,13 +576,16 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   }
 
   QSPEC_TRACE_AT(0xFFF0);
+  if (warp >= kCtlWarps + kConvWarps && (threadIdx.x & 31) == 0 && warp == kCtlWarps + kConvWarps)
+    QSPEC_PHASE(6);
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) QSPEC_PHASE(8);
+  QSPEC_STAMP_FLUSH();
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
-  QSPEC_TRACE_AT(0xFFFF);
 }
 
 }  // namespace qspec

@@ -159,7 +159,21 @@ qspec_status launch_qgemm_t(const CUtensorMap& tw, const CUtensorMap& tx, const 
     }
     attr_set[dev] = true;
   }
-  qgemm_kernel<kInt8, MT><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tw, tx, a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  // W4A4 follows its own activation-quantization kernel: overlap with it.
+  cfg.attrs = attr;
+  cfg.numAttrs = kInt8 ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, qgemm_kernel<kInt8, MT>, tw, tx, a) != cudaSuccess) {
+    cudaGetLastError();
+    return QSPEC_ERR_CUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? QSPEC_OK : QSPEC_ERR_CUDA;
 }
 
@@ -242,6 +256,12 @@ using namespace qspec;
 #ifdef QSPEC_TRACE
 extern "C" int qspec_debug_set_trace(void* host_mapped) {
   return cudaMemcpyToSymbol(g_qspec_trace, &host_mapped, sizeof(void*)) == cudaSuccess ? 0 : 1;
+}
+extern "C" int qspec_debug_set_phases(void* dev_buffer) {
+  return cudaMemcpyToSymbol(g_qspec_phases, &dev_buffer, sizeof(void*)) == cudaSuccess ? 0 : 1;
+}
+extern "C" int qspec_debug_set_timeline(void* dev_buffer) {
+  return cudaMemcpyToSymbol(g_qspec_timeline, &dev_buffer, sizeof(void*)) == cudaSuccess ? 0 : 1;
 }
 #endif
 

@@ -80,6 +80,10 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
   const uint16_t* xr = x + row * k;
   const int tid = threadIdx.x;
   QSPEC_TRACE_AT(1);
+  // The GEMM that consumes this kernel's output is launched as a programmatic
+  // dependent: it may start streaming weights now and waits for our results
+  // (griddepcontrol.wait) only where it reads them.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (!QSPEC_ALIGN_OK(reinterpret_cast<uintptr_t>(xr), 16) ||
       !QSPEC_ALIGN_OK(reinterpret_cast<uintptr_t>(out), 8))
     return;
