@@ -153,6 +153,34 @@ qspec_status qspec_spec_accept(const float* p, const float* q, const int32_t* dr
                                int32_t* tokens, void* workspace, size_t workspace_bytes,
                                void* stream);
 
+/*
+ * W4A16 verifying GEMM that allocates nothing and takes no workspace.
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory at the point of the call -- e.g. code
+ * running where the CUDA runtime may not be entered to allocate, such as a
+ * host function enqueued with cudaLaunchHostFunc, or a plugin hosted by an
+ * application that owns all device memory and permits no allocation outside
+ * its own pools.
+ * Computes exactly what qspec_gemm_w4a16 computes, with its scratch held in a
+ * file-scope device array of QSPEC_STATIC_SCRATCH_BYTES (16 MiB) that every
+ * GPU loading this library keeps until the process exits.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture.
+ *  - Every call shares the one array: calls that overlap on the GPU (on
+ *    different streams, or from different threads) race and must not be
+ *    issued.  Each call clears the status word and split-tile tickets with an
+ *    asynchronous memset on `stream`; nothing else needs to start at zero.
+ *  - Shapes whose scratch would exceed the array (for example m > 96 on a
+ *    148-SM B200) return QSPEC_ERR_WORKSPACE_TOO_SMALL and launch nothing.
+ *  - Calls no cudaMalloc, cudaFree or other allocating routine.
+ * Arguments as for qspec_gemm_w4a16, without workspace.
+ */
+#define QSPEC_STATIC_SCRATCH_BYTES (16u << 20)
+qspec_status qspec_gemm_w4a16_noalloc(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
+                                      const uint16_t* ws, int64_t n, int32_t group, float* y,
+                                      void* stream);
+
 /* Bytes of workspace an operation needs on the current device (0 = none).
  * Unused size arguments are ignored.  Returns 0 for invalid arguments too. */
 size_t qspec_workspace_size(int32_t op, int64_t m, int64_t n, int64_t k, int32_t group,

@@ -388,6 +388,59 @@ qspec_status qspec_workspace_status(void* workspace, void* stream) {
   return (word & kDevTimeout) ? QSPEC_ERR_TIMEOUT : QSPEC_ERR_BAD_INPUT;
 }
 
+// ---------------------------------------------------------------- no-allocation variant
+// Built-in scratch for callers that cannot allocate device memory: code that
+// runs where the CUDA runtime may not be entered to allocate (for example a
+// host function enqueued with cudaLaunchHostFunc), or a plugin inside a host
+// application that owns all device memory and allows no allocation beyond
+// its own pools.  Every GPU that loads this library holds the array until
+// the process exits.
+static __device__ __align__(256) unsigned char g_qspec_static_scratch[QSPEC_STATIC_SCRATCH_BYTES];
+
+namespace {
+void* g_static_scratch_ptr[kMaxDevices] = {};
+std::mutex g_static_scratch_mutex;
+}  // namespace
+
+qspec_status qspec_gemm_w4a16_noalloc(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
+                                      const uint16_t* ws, int64_t n, int32_t group, float* y,
+                                      void* stream) {
+  if (!x || !wq || !ws || !y) return QSPEC_ERR_INVALID_ARG;
+  if (!gemm_shape_ok(m, n, k, group)) return QSPEC_ERR_INVALID_ARG;
+  int dev = 0;
+  DeviceInfo info;
+  qspec_status st = current_device(&dev, &info);
+  if (st != QSPEC_OK) return st;
+  // The scratch needed by this shape must fit in the built-in array.
+  if (plan_gemm(false, m, n, k, info.sm_count).total > QSPEC_STATIC_SCRATCH_BYTES)
+    return QSPEC_ERR_WORKSPACE_TOO_SMALL;
+  void* scratch = nullptr;
+  {
+    // One-time set-up per device, with that device current: host code must
+    // ask the runtime for the array's device address (the symbol's name is
+    // only a host-side stand-in).
+    std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
+    if (!g_static_scratch_ptr[dev]) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_qspec_static_scratch) != cudaSuccess || p == nullptr) {
+        cudaGetLastError();
+        return QSPEC_ERR_CUDA;
+      }
+      g_static_scratch_ptr[dev] = p;
+    }
+    scratch = g_static_scratch_ptr[dev];
+  }
+  // The array keeps whatever the previous call left: reset the status word and
+  // the split-tile tickets, the only parts that must start at zero.
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(scratch, 0, 256 + static_cast<size_t>(kMaxGrid) * 4, s) != cudaSuccess) {
+    cudaGetLastError();
+    return QSPEC_ERR_CUDA;
+  }
+  return run_gemm<false>(x, m, k, wq, ws, n, group, y, scratch, QSPEC_STATIC_SCRATCH_BYTES, nullptr,
+                         stream);
+}
+
 const char* qspec_status_string(qspec_status status) {
   switch (status) {
     case QSPEC_OK: return "ok";

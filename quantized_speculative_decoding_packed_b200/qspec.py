@@ -23,7 +23,7 @@ OP_QUANTIZE_WEIGHTS, OP_QUANT_ACT, OP_GEMM_W4A4, OP_GEMM_W4A16, OP_SPEC_ACCEPT =
 
 EXPORTED = ("qspec_quantize_weights", "qspec_quant_act", "qspec_gemm_w4a4", "qspec_gemm_w4a16",
             "qspec_spec_accept", "qspec_workspace_size", "qspec_workspace_status",
-            "qspec_status_string")
+            "qspec_status_string", "qspec_gemm_w4a16_noalloc")
 
 
 class QSpecError(RuntimeError):
@@ -43,6 +43,7 @@ def _load() -> ctypes.CDLL:
     lib.qspec_quant_act.argtypes = [P, I64, I64, P, P, P]
     lib.qspec_gemm_w4a4.argtypes = [P, I64, I64, P, P, I64, I32, P, P, SZ, P, P]
     lib.qspec_gemm_w4a16.argtypes = [P, I64, I64, P, P, I64, I32, P, P, SZ, P]
+    lib.qspec_gemm_w4a16_noalloc.argtypes = [P, I64, I64, P, P, I64, I32, P, P]
     lib.qspec_spec_accept.argtypes = [P, P, P, P, P, I32, I32, I32, P, P, P, SZ, P]
     lib.qspec_workspace_size.argtypes = [I32, I64, I64, I64, I32, I32, I32, I32]
     lib.qspec_workspace_size.restype = SZ
@@ -50,7 +51,8 @@ def _load() -> ctypes.CDLL:
     lib.qspec_status_string.argtypes = [I32]
     lib.qspec_status_string.restype = ctypes.c_char_p
     for name in ("qspec_quantize_weights", "qspec_quant_act", "qspec_gemm_w4a4",
-                 "qspec_gemm_w4a16", "qspec_spec_accept", "qspec_workspace_status"):
+                 "qspec_gemm_w4a16", "qspec_spec_accept", "qspec_workspace_status",
+                 "qspec_gemm_w4a16_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -163,6 +165,23 @@ def gemm_w4a16(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor, group: int =
         work = workspace(need, x.device)
     _check(LIB.qspec_gemm_w4a16(_ptr(x), m, k, _ptr(wq), _ptr(ws), n, group, _ptr(y), _ptr(work),
                                 work.numel(), _stream(stream)), "qspec_gemm_w4a16")
+    return y
+
+
+def gemm_w4a16_noalloc(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor, group: int = 128,
+                       y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """W4A16 verifying GEMM using the library's built-in scratch (no workspace).
+
+    For callers that cannot allocate device memory where they call; the
+    output buffer is still the caller's.  Calls must not overlap on the GPU.
+    """
+    _need(x, torch.bfloat16, "x")
+    m, k = x.shape
+    n = wq.shape[0]
+    if y is None:
+        y = torch.empty((m, n), dtype=torch.float32, device=x.device)
+    _check(LIB.qspec_gemm_w4a16_noalloc(_ptr(x), m, k, _ptr(wq), _ptr(ws), n, group, _ptr(y),
+                                        _stream(stream)), "qspec_gemm_w4a16_noalloc")
     return y
 
 
