@@ -88,6 +88,27 @@ def step_work(layers):
     return b, ops
 
 
+# ---------------------------------------------------------------- multi-rank plumbing
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank float over all ranks (the job time is the slowest rank's)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_rank_step: float, world: int, ms_step: float) -> float:
+    """Whole-job GB/s: every rank processes its own replica of the step (weak scaling)."""
+    return world * bytes_per_rank_step / (ms_step * 1e-3) / 1e9
+
+
+def rank_seed(rank: int) -> int:
+    return 20241015 + 1000 * rank
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     """Samples SM clock and clock-event reasons through NVML while running (read only)."""
@@ -242,7 +263,7 @@ def main():
 
     L = args.layers
     gen = torch.Generator(device=dev)
-    gen.manual_seed(20241015 + 1000 * rank)
+    gen.manual_seed(rank_seed(rank))
 
     # ---- one packed INT4 weight set, shared by both modes
     wq = [[None] * len(LAYERS) for _ in range(L)]
@@ -348,9 +369,7 @@ def main():
         ms_total = start.elapsed_time(end)
     ms_step = ms_total / args.steps
     if world > 1:
-        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+        ms_total = max_over_ranks(ms_total, dev)
         ms_step = ms_total / args.steps
 
     # per-kernel durations from the last timed step
@@ -359,6 +378,7 @@ def main():
 
     kern = {}
     w4a4_b = w4a4_t = 0.0
+    gu_b = gu_t = 0.0
     for si, (name, n, k) in enumerate(LAYERS):
         t4 = [dur("w4a4", pss, si) for pss in range(GAMMA)]
         t16 = dur("w4a16", 0, si)
@@ -369,6 +389,8 @@ def main():
                       "w4a16_tflops": 2 * M_VERIFY * n * k / (t16 * 1e-3) / 1e12}
         w4a4_b += b4 * GAMMA
         w4a4_t += sum(t4)
+        if name == "gate_up":
+            gu_b, gu_t = b4 * GAMMA, sum(t4)
     t_acc = dur("accept", 0, 0)
     acc_b = accept_bytes(n_acc.cpu().numpy(), GAMMA, VOCAB)
     kern["accept"] = {"us": 1e3 * t_acc, "gbs": acc_b / (t_acc * 1e-3) / 1e9}
@@ -380,16 +402,22 @@ def main():
     except Exception:
         pass
     hbm_peak = peaks.get("hbm_gbs", 6650.0)
-    achieved = w4a4_b / (w4a4_t * 1e-3) / 1e9
+    # Dominant kernel: the W4A4 drafting GEMM.  The roofline object describes its
+    # largest launch (gate+up, 46.5 MB packed), timed live over the 4 draft passes
+    # of each step's layer 0; the all-shape figure is kept beside it.
+    achieved = gu_b / (gu_t * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "traffic": traffic_from_profile(),
-                "kernel": "W4A4 drafting GEMM call (per-token quant pre-pass + qgemm_kernel<int8,16>)",
+                "kernel": "W4A4 drafting GEMM call on gate_up N=22016 K=4096 M=16 "
+                          "(per-token quant pre-pass + qgemm_kernel<int8,16>)",
+                "bytes_per_launch": gemm_bytes(M_DRAFT, 22016, 4096, "w4a4"),
+                "all_shapes_achieved": w4a4_b / (w4a4_t * 1e-3) / 1e9,
                 "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)" if "hbm_gbs" in peaks
                 else "fallback 6650 GB/s"}
 
     bytes_step, ops_step = step_work(L)
     bytes_step += acc_b
-    value = world * bytes_step / (ms_step * 1e-3) / 1e9
+    value = job_throughput(bytes_step, world, ms_step)
 
     e2e = None
     if not args.no_e2e:
