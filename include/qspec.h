@@ -96,7 +96,8 @@ qspec_status qspec_quant_act(const uint16_t* x, int64_t m, int64_t k, uint8_t* x
  * is computed exactly on the int8 tensor cores (int32), and
  *   y[m][n] = s_a[m] * sum_g s_h[n][g] * acc[m][n][g]   (fp32 arithmetic).
  *  x        [m][k] bf16.
- *  wq, ws   as produced by qspec_quantize_weights for [n][k] weights.
+ *  wq, ws   as produced by qspec_quantize_weights for [n][k] weights; wq
+ *           16-byte aligned, ws 4-byte aligned (scales are fetched as words).
  *  y        [m][n] fp32 out.
  *  workspace  device scratch of at least
  *           qspec_workspace_size(QSPEC_OP_GEMM_W4A4, m, n, k, group, 0, 0, 0)

@@ -24,15 +24,17 @@
 // units +-1, whatever the shape.  A CTA that covers a whole tile writes y
 // directly; partial tiles go to workspace slots and the last CTA to finish a
 // tile (an atomic ticket, no waiting) adds the slots in K order, so results
-// are deterministic.  A split tile starts inside exactly one CTA's range and
+// are deterministic.  The ticket of a CTA's first split tile is taken by the
+// weight producer, so the epilogue goes straight on to the next tile.  A split tile starts inside exactly one CTA's range and
 // at most one split tile starts in any CTA's range, so the ticket of a tile
 // is indexed by its first contributor; tickets return to zero after use.
 //
 // Warp roles (one CTA per SM):
 //   warp 0      TMA producer for packed weight tiles (ring of up to 16 x 8 KB)
 //   warp 1      TMA producer for activation tiles (128-byte swizzled ring)
-//   warp 2      tensor-memory allocation and the single MMA-issuing thread
-//   warp 3      idle
+//   warps 2, 3  MMA issuers for even / odd units (warp 2 also owns the
+//               tensor-memory allocation); two issuers halve the exposed
+//               per-instruction issue latency of the small decode MMAs
 //   8 warps     converters: packed nibbles -> int8 / bf16 operand tiles
 //   4..16 warps epilogue: tensor memory -> registers, group scales, output
 //
@@ -79,17 +81,22 @@ struct GemmCfg {
   static constexpr int kEpiWarps = 4 * kTeams;
   static constexpr int kCols = MT / kTeams;                      // token columns per epilogue thread
   static_assert(kCols % 8 == 0, "epilogue columns must be a multiple of 8");
+  static constexpr int kEpiThreads = 32 * kEpiWarps;
   static constexpr int kWarps = kCtlWarps + kConvWarps + kEpiWarps;
   static constexpr int kThreads = 32 * kWarps;
   static constexpr int kBarBytes = 1024;
+  // group scales travel global -> shared by cp.async, kScaleAhead groups ahead
+  static constexpr int kScaleAhead = 4;
+  static constexpr int kScaleSlots = kScaleAhead + 1;
+  static constexpr int kScaleBytes = kScaleSlots * kEpiThreads * 4;
   // ring depths from the shared-memory budget
   static constexpr int kNumCv = (!kInt8 && MT >= 64) ? 2 : 4;
-  static constexpr int kAvail = kSmemLimit - 1024 - kBarBytes - kNumCv * kCvBytes;
+  static constexpr int kAvail = kSmemLimit - 1024 - kBarBytes - kScaleBytes - kNumCv * kCvBytes;
   static constexpr int kNumX = cmin(kMaxX, (kAvail - 6 * kPkBytes) / kXBytes);
   static constexpr int kNumPk = cmin(kMaxPk, (kAvail - kNumX * kXBytes) / kPkBytes);
   static_assert(kNumX >= 2 && kNumPk >= 6, "shared memory too small for the rings");
   static constexpr int kSmemBytes =
-      1024 + kNumPk * kPkBytes + kNumCv * kCvBytes + kNumX * kXBytes + kBarBytes;
+      1024 + kNumPk * kPkBytes + kNumCv * kCvBytes + kNumX * kXBytes + kScaleBytes + kBarBytes;
   static_assert(kSmemBytes <= kSmemLimit, "shared memory overflow");
   static constexpr int kTmemCols = pow2_at_least(kNumAcc * MT);
   static_assert(kTmemCols <= 512, "tensor memory overflow");
@@ -167,10 +174,24 @@ __device__ __forceinline__ void grid_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Ticket of split tile t after this CTA published its share (one thread).
+// Returns true for the tile's last contributor, which then adds the shares.
+__device__ __forceinline__ bool take_tile_ticket(const GemmArgs& args, long long t,
+                                                 long long units, long long grid) {
+  const long long tile_u0 = t * args.ku;
+  const long long c_lo = unit_owner(tile_u0, units, grid);
+  const long long c_hi = unit_owner(tile_u0 + args.ku - 1, units, grid);
+  __threadfence();   // the share, seen through an mbarrier, before the ticket
+  const uint32_t old = atomicAdd(&args.counters[c_lo], 1u);
+  const bool last = (old == static_cast<uint32_t>(c_hi - c_lo));
+  if (last) __threadfence();   // every share, before the reads of the reduction
+  return last;
+}
+
 template <bool kInt8, int MT>
 __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     qgemm_kernel(const __grid_constant__ CUtensorMap tmap_w,
-                 const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args) {
+                 const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ GemmArgs args) {
   using C = GemmCfg<kInt8, MT>;
   constexpr int NPK = C::kNumPk, NCV = C::kNumCv, NX = C::kNumX;
   extern __shared__ uint8_t smem_raw[];
@@ -180,7 +201,8 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   uint8_t* pk_buf = smem;
   uint8_t* cv_buf = pk_buf + NPK * kPkBytes;
   uint8_t* x_buf = cv_buf + NCV * C::kCvBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(x_buf + NX * C::kXBytes);
+  uint32_t* scale_ring = reinterpret_cast<uint32_t*>(x_buf + NX * C::kXBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(scale_ring + C::kScaleSlots * C::kEpiThreads);
   uint64_t* pk_full = bars;
   uint64_t* pk_empty = pk_full + kMaxPk;
   uint64_t* cv_full = pk_empty + kMaxPk;
@@ -190,9 +212,12 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   uint64_t* acc_full = x_empty + kMaxX;
   uint64_t* acc_empty = acc_full + kNumAcc;
   uint64_t* mma_done = acc_empty + kNumAcc;
-  uint64_t* epi_sync = mma_done + 1;
+  uint64_t* flush_bar = mma_done + 1;   // the head split tile's share is published
+  uint64_t* ticket_bar = flush_bar + 1; // ... and its ticket taken (result in misc[3])
+  uint64_t* epi_sync = ticket_bar + 1;
   uint32_t* misc = reinterpret_cast<uint32_t*>(epi_sync + 1);
-  // misc[0]: tensor-memory base; misc[1]: abort flag; misc[2]: reducer flag
+  // misc[0]: tensor-memory base; misc[1]: abort flag; misc[2]: reducer flag;
+  // misc[3]: this CTA is the last contributor of its head split tile
   volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[1]);
 
   const int warp = threadIdx.x >> 5;
@@ -223,7 +248,10 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       mbar_init(smem_u32(&acc_full[b]), 1);
       mbar_init(smem_u32(&acc_empty[b]), C::kEpiWarps);
     }
-    mbar_init(smem_u32(mma_done), 1);
+    mbar_init(smem_u32(mma_done), 2);
+    mbar_init(smem_u32(flush_bar), C::kEpiWarps);
+    mbar_init(smem_u32(ticket_bar), 1);
+    misc[3] = 0;
     mbar_init(smem_u32(epi_sync), C::kEpiWarps);
     misc[1] = 0;
     misc[2] = 0;
@@ -247,6 +275,14 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------ packed-weight producer
     // (the whole warp walks the loop; an elected lane issues the copies)
+    // This warp also takes the ticket of the CTA's first tile when that tile
+    // is split and more tiles follow (the epilogue handles a split last tile
+    // itself); it probes for the published share once per unit, having run
+    // far enough ahead that the ticket's latency costs the pipeline nothing,
+    // and leaves any reduction to the epilogue's many threads.
+    const long long t_head = u_begin / ku;
+    const long long head_end = (u_end < (t_head + 1) * ku) ? u_end : (t_head + 1) * ku;
+    bool head_pending = (u_begin < u_end) && head_end < u_end && u_begin != t_head * ku;
     int i = 0;
     UnitCursor cur;
     cur.init(u_begin, ku, args.m_tiles);
@@ -261,6 +297,21 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       }
       __syncwarp();
       QSPEC_STAMP(0, i);
+      if (head_pending && __all_sync(0xffffffffu, mbar_test_wait(smem_u32(flush_bar), 0))) {
+        if (lane == 0) {
+          misc[3] = take_tile_ticket(args, t_head, units, grid) ? 1u : 0u;
+          mbar_arrive(smem_u32(ticket_bar));
+        }
+        __syncwarp();
+        head_pending = false;
+      }
+    }
+    if (head_pending && warp_wait(smem_u32(flush_bar), 0, abort_flag, args.status)) {
+      if (lane == 0) {
+        misc[3] = take_tile_ticket(args, t_head, units, grid) ? 1u : 0u;
+        mbar_arrive(smem_u32(ticket_bar));
+      }
+      __syncwarp();
     }
     if (*abort_flag) {
       for (int j = (i > NPK ? i - NPK : 0); j < i; ++j)
@@ -292,15 +343,17 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       for (int j = (i > NX ? i - NX : 0); j < i; ++j)
         mbar_wait_drain(smem_u32(&x_full[j % NX]), (j / NX) & 1);
     }
-  } else if (warp == 2) {
-    // ------------------------------------------------ MMA issuer
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------ MMA issuers (even / odd units)
     // The whole warp walks the loop (waits are warp-uniform); one elected lane
     // issues each tcgen05 instruction, which is cheaper than a lone lane.
     constexpr uint32_t idesc = kInt8 ? idesc_i8(MT) : idesc_bf16(MT);
     const int per_group = C::kMmas / gpu;
-    int i = 0, j = 0;
+    const int parity = warp - 2;
+    int i = parity;
     bool ok = true;
-    for (long long u = u_begin; u < u_end && ok; ++u, ++i) {
+    for (long long u = u_begin + parity; u < u_end && ok; u += 2, i += 2) {
+      int j = i * gpu;
       const int sc = i % NCV;
       const int sx = i % NX;
       QSPEC_STAMP(13, i);
@@ -319,18 +372,18 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         if (h == 0) QSPEC_STAMP(8, i);
-        for (int kk = 0; kk < per_group; ++kk) {
-          const uint32_t kbyte = static_cast<uint32_t>(h * per_group + kk) * 32u;
-          const uint32_t atom = kbyte >> 7, within = kbyte & 127u;
-          const uint64_t a_desc = smem_desc_sw128(a_base + atom * (kTileN * 128) + within);
-          const uint64_t b_desc = smem_desc_sw128(b_base + atom * (MT * 128) + within);
-          if (elect_one_lane())
+        // One elected lane issues the group's MMAs and its commit back to back.
+        if (elect_one_lane()) {
+          for (int kk = 0; kk < per_group; ++kk) {
+            const uint32_t kbyte = static_cast<uint32_t>(h * per_group + kk) * 32u;
+            const uint32_t atom = kbyte >> 7, within = kbyte & 127u;
+            const uint64_t a_desc = smem_desc_sw128(a_base + atom * (kTileN * 128) + within);
+            const uint64_t b_desc = smem_desc_sw128(b_base + atom * (MT * 128) + within);
             mma_ss<kInt8>(tmem_base + static_cast<uint32_t>(b * MT), a_desc, b_desc, idesc,
                           kk > 0 ? 1u : 0u);
-          __syncwarp();
-          if (h == 0 && (kk == 0 || kk == per_group - 1)) QSPEC_STAMP(kk == 0 ? 9 : 11, i);
+          }
+          mma_commit(smem_u32(&acc_full[b]));
         }
-        if (elect_one_lane()) mma_commit(smem_u32(&acc_full[b]));
         __syncwarp();
         if (h == 0) QSPEC_STAMP(12, i);
       }
@@ -414,45 +467,93 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       if (warp == kCtlWarps) QSPEC_STAMP(2, i);
     }
   } else if (warp >= kCtlWarps + kConvWarps) {
-    // ------------------------------------------------ epilogue (warp 3 is idle and lands nowhere)
+    // ------------------------------------------------ epilogue
     const int ew = warp - (kCtlWarps + kConvWarps);
     const int quad = warp & 3;                 // tensor-memory lanes this warp may read
     const int team = ew >> 2;
     const int col0 = team * C::kCols;
     const int row = quad * 32 + lane;
-    const int et = ew * 32 + lane;             // 0 .. kEpiWarps*32-1
+    const int et = ew * 32 + lane;             // 0 .. kEpiThreads-1
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
-    volatile int* reducer_flag = reinterpret_cast<volatile int*>(&misc[2]);
 
-    // Group scales are read from global memory four groups ahead of use; a
-    // second cursor walks the CTA's groups for the prefetch.
+    // Group scales.  Each thread copies the aligned 32-bit word holding its
+    // row's fp16 scale of group j + kScaleAhead into a private shared-memory
+    // slot with cp.async (nothing waits on a register) and reads group j's
+    // scale once that copy has landed: the load latency hides behind
+    // kScaleAhead groups of work.  A word that would end past the last
+    // scale is copied as its first half only.
     const int groups_total = static_cast<int>(u_end - u_begin) * gpu;
+    const long long ws_elems = static_cast<long long>(args.N) * args.groups_per_row;
+    const uint32_t slot0 = smem_u32(scale_ring + et);
+    constexpr uint32_t kSlotStride = C::kEpiThreads * 4;
     UnitCursor pf;
     pf.init(u_begin, ku, args.m_tiles);
-    int pf_h = 0, pf_j = 0;
-    auto next_scale = [&]() -> float {
-      float v = 0.f;
+    int pf_h = 0, pf_j = 0, pf_slot = 0;
+    auto issue_scale = [&]() {
       if (pf_j < groups_total) {
         const int nn = pf.n_tile * kTileN + row;
-        if (nn < args.N)
-          v = __half2float(__ushort_as_half(
-              __ldg(args.ws + static_cast<long long>(nn) * args.groups_per_row + pf.kc * gpu + pf_h)));
-        ++pf_j;
+        if (nn < args.N) {
+          const long long idx =
+              static_cast<long long>(nn) * args.groups_per_row + pf.kc * gpu + pf_h;
+          const long long w0 = idx & ~1ll;
+          cp_async_4(slot0 + pf_slot * kSlotStride, args.ws + w0, (w0 + 1 < ws_elems) ? 4u : 2u);
+        }
         if (++pf_h == gpu) {
           pf_h = 0;
           pf.next(ku, args.m_tiles);
         }
       }
-      return v;
+      ++pf_j;
+      if (++pf_slot == C::kScaleSlots) pf_slot = 0;
+      cp_async_commit();   // one group per scale, possibly empty, keeps the count uniform
     };
-    float sq0 = next_scale();
-    float sq1 = next_scale();
-    float sq2 = next_scale();
-    float sq3 = next_scale();
+#pragma unroll
+    for (int a = 0; a < C::kScaleAhead; ++a) issue_scale();
 
     float run[C::kCols];
-    int j = 0;
+    // y rows m0 .. m0+kCols-1 of output column n from run[]
+    auto write_y = [&](int n, int m0) {
+      if (n >= args.N) return;
+      if constexpr (kInt8) grid_dependency_wait();   // s_a comes from the preceding kernel
+#pragma unroll
+      for (int c = 0; c < C::kCols; ++c) {
+        const int m = m0 + c;
+        if (m < args.M) {
+          const float v = kInt8 ? args.s_a[m] * run[c] : run[c];
+          args.y[static_cast<long long>(m) * args.N + n] = v;
+        }
+      }
+    };
+    // As the last contributor of split tile t: add every share in K order
+    // (the CTA owning the tile's first unit first) and write y.  Contributor
+    // c_lo wrote its head slot if its range starts at the tile, else its tail
+    // slot; every later contributor starts inside the tile.
+    auto reduce_tile = [&](long long t) {
+      const long long tile_u0 = t * ku;
+      const long long c_lo = unit_owner(tile_u0, units, grid);
+      const long long c_hi = unit_owner(tile_u0 + ku - 1, units, grid);
+      const int lo_k = (unit_begin(c_lo, units, grid) == tile_u0) ? 0 : 1;
+      const float* src = args.partials + (2 * c_lo + lo_k) * static_cast<long long>(MT * kTileN);
+#pragma unroll
+      for (int c = 0; c < C::kCols; ++c) run[c] = __ldcg(src + (col0 + c) * kTileN + row);
+      for (long long cc = c_lo + 1; cc <= c_hi; ++cc) {
+        src = args.partials + 2 * cc * static_cast<long long>(MT * kTileN);
+#pragma unroll
+        for (int c = 0; c < C::kCols; ++c) run[c] += __ldcg(src + (col0 + c) * kTileN + row);
+      }
+      if (et == 0) args.counters[c_lo] = 0u;   // ready for the next launch
+      const int n_tile = static_cast<int>(t / args.m_tiles);
+      const int m_tile = static_cast<int>(t - static_cast<long long>(n_tile) * args.m_tiles);
+      write_y(n_tile * kTileN + row, m_tile * MT + col0);
+    };
+    const long long t_head = u_begin / ku;
+    const long long head_end = (u_end < (t_head + 1) * ku) ? u_end : (t_head + 1) * ku;
+    const bool head_handoff = (u_begin < u_end) && head_end < u_end && u_begin != t_head * ku;
+    long long to_reduce[2];
+    int n_reduce = 0;
+    int j = 0, rd_slot = 0;
     bool ok = true;
+    volatile int* reducer_flag = reinterpret_cast<volatile int*>(&misc[2]);
     uint32_t epi_phase = 0;
     // All epilogue warps meet here; bounded, unlike a hardware named barrier.
     auto epi_barrier = [&]() -> bool {
@@ -473,6 +574,8 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       const long long seg_end = (u_end < tile_u0 + ku) ? u_end : tile_u0 + ku;
       const int n = cur.n_tile * kTileN + row;
       const int m0 = cur.m_tile * MT + col0;
+      // scale (n, g) sits in the upper half of its word when n * G + g is odd
+      const uint32_t row_par = static_cast<uint32_t>(n & args.groups_per_row & 1);
 #pragma unroll
       for (int c = 0; c < C::kCols; ++c) run[c] = 0.f;
       for (; u < seg_end && ok; ++u, cur.next(ku, args.m_tiles)) {
@@ -481,11 +584,13 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
           const int b = j % kNumAcc;
           const uint32_t pha = (j / kNumAcc) & 1;
           const int g = kc * gpu + h;
-          const float sc = sq0;
-          sq0 = sq1;
-          sq1 = sq2;
-          sq2 = sq3;
-          sq3 = next_scale();
+          cp_async_wait<C::kScaleAhead - 1>();   // this thread's copy for group j has landed
+          uint32_t sw;
+          asm volatile("ld.shared.b32 %0, [%1];" : "=r"(sw) : "r"(slot0 + rd_slot * kSlotStride));
+          if (++rd_slot == C::kScaleSlots) rd_slot = 0;
+          const uint32_t hbits = ((row_par ^ static_cast<uint32_t>(g)) & 1u) ? (sw >> 16) : (sw & 0xFFFFu);
+          const float sc = __half2float(__ushort_as_half(static_cast<unsigned short>(hbits)));
+          issue_scale();   // refills the slot read one group ago
           ok = warp_wait(smem_u32(&acc_full[b]), pha, abort_flag, args.status);
           if (!ok) break;
           if (ew == 0) QSPEC_STAMP(5, j);
@@ -531,48 +636,36 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       if (et == 0) QSPEC_PHASE(u >= u_end ? 5 : 7);
 
       const bool full = (seg_start == tile_u0) && (seg_end == tile_u0 + ku);
-      bool write_out = full;
-      if (!full) {
-        // Publish this CTA's share of the tile, then take a ticket.
-        const int slot = static_cast<int>(2 * cta + (seg_start == u_begin ? 0 : 1));
-        float* mine = args.partials + static_cast<long long>(slot) * MT * kTileN;
+      if (full) {
+        write_y(n, m0);
+      } else {
+        const int k = (seg_start == u_begin) ? 0 : 1;
+        float* mine = args.partials + static_cast<long long>(2 * cta + k) * MT * kTileN;
 #pragma unroll
         for (int c = 0; c < C::kCols; ++c) mine[(col0 + c) * kTileN + row] = run[c];
-        __threadfence();
-        if (!epi_barrier()) break;
-        const long long c_lo = unit_owner(tile_u0, units, grid);
-        const long long c_hi = unit_owner(tile_u0 + ku - 1, units, grid);
-        if (et == 0) {
-          const uint32_t old = atomicAdd(&args.counters[c_lo], 1u);
-          *reducer_flag = (old == static_cast<uint32_t>(c_hi - c_lo)) ? 1 : 0;
-        }
-        if (!epi_barrier()) break;
-        write_out = (*reducer_flag != 0);
-        if (write_out) {
-          __threadfence();
-#pragma unroll
-          for (int c = 0; c < C::kCols; ++c) run[c] = 0.f;
-          for (long long cc = c_lo; cc <= c_hi; ++cc) {
-            const int s2 = static_cast<int>(2 * cc + (unit_begin(cc, units, grid) >= tile_u0 ? 0 : 1));
-            const float* src = args.partials + static_cast<long long>(s2) * MT * kTileN;
-#pragma unroll
-            for (int c = 0; c < C::kCols; ++c) run[c] += __ldcg(src + (col0 + c) * kTileN + row);
-          }
-          if (et == 0) args.counters[c_lo] = 0u;   // ready for the next launch
-        }
-      }
-      if (write_out && n < args.N) {
-        if constexpr (kInt8) grid_dependency_wait();   // s_a comes from the preceding kernel
-#pragma unroll
-        for (int c = 0; c < C::kCols; ++c) {
-          const int m = m0 + c;
-          if (m < args.M) {
-            const float v = kInt8 ? args.s_a[m] * run[c] : run[c];
-            args.y[static_cast<long long>(m) * args.N + n] = v;
-          }
+        if (seg_end < u_end) {
+          // The CTA's first tile with more to follow: publish the share and go
+          // on; the weight producer takes the ticket.
+          __syncwarp();
+          if (elect_one_lane()) mbar_arrive(smem_u32(flush_bar));
+          __syncwarp();
+        } else {
+          // The CTA's last tile: take the ticket here.
+          if (!epi_barrier()) break;
+          if (et == 0) *reducer_flag = take_tile_ticket(args, t, units, grid) ? 1 : 0;
+          if (!epi_barrier()) break;
+          if (*reducer_flag != 0) to_reduce[n_reduce++] = t;
         }
       }
     }
+    // The split tiles whose last ticket came to this CTA are added up here,
+    // after the CTA's own tiles: the last one and possibly the head one.
+    if (ok && head_handoff) {
+      ok = warp_wait(smem_u32(ticket_bar), 0, abort_flag, args.status);
+      if (ok && misc[3] != 0u) to_reduce[n_reduce++] = t_head;
+    }
+    for (int r = 0; ok && r < n_reduce; ++r) reduce_tile(to_reduce[r]);
+    cp_async_wait<0>();
   }
 
   QSPEC_TRACE_AT(0xFFF0);

@@ -198,7 +198,7 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
                       size_t workspace_bytes, int32_t* dbg_acc, void* stream_v) {
   if (!x || !wq || !ws || !y || !workspace) return QSPEC_ERR_INVALID_ARG;
   if (!gemm_shape_ok(m, n, k, group)) return QSPEC_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(wq, 16) || !aligned(ws, 2) || !aligned(y, 4) ||
+  if (!aligned(x, 16) || !aligned(wq, 16) || !aligned(ws, 4) || !aligned(y, 4) ||
       !aligned(workspace, 16) || (dbg_acc && !aligned(dbg_acc, 4)))
     return QSPEC_ERR_INVALID_ARG;
   int dev = 0;
