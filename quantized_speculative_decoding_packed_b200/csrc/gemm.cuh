@@ -5,10 +5,12 @@
 // notes that the modes differ mainly in how activations are handled.  This
 // one kernel template serves both from the same `wq`/`ws` bytes:
 //
-//   W4A4  (kInt8 = true):  nibbles widened to int8 in shared memory,
-//         tcgen05.mma kind::i8 (s8 x s8 -> s32 in tensor memory), one exact
-//         int32 accumulator per weight group; epilogue
-//         y = s_a[m] * sum_g s_h[n,g] * acc_g.
+//   W4A4  (kInt8 = true):  nibbles widened to int8 (as 16 q: two masks and
+//         two byte permutes per 8 weights) in shared memory, tcgen05.mma
+//         kind::i8 (s8 x s8 -> s32 in tensor memory), one exact int32
+//         accumulator per weight group (16 acc_g); epilogue
+//         y = (s_a[m] / 16) * sum_g s_h[n,g] * (16 acc_g), bit-identical to
+//         s_a[m] * sum_g s_h[n,g] * acc_g since only powers of two differ.
 //   W4A16 (kInt8 = false): nibbles widened to exact bf16 integers in shared
 //         memory, tcgen05.mma kind::f16 (bf16 x bf16 -> f32), one fp32 partial
 //         per group; epilogue y = sum_g s_h[n,g] * partial_g, i.e. exactly
@@ -77,8 +79,12 @@ struct GemmCfg {
   static constexpr int kXBytes = MT * 128 * kAtoms;              // activation tile
   static constexpr int kMmaK = kInt8 ? 32 : 16;
   static constexpr int kMmas = kUnitK / kMmaK;                   // MMAs per unit
-  static constexpr int kTeams = (MT <= 48) ? 1 : (MT <= 96 ? 2 : 4);
-  static constexpr int kEpiWarps = 4 * kTeams;
+  static constexpr int kTeams = (MT <= 48) ? 1 : (MT <= 96 ? 2 : 4);   // column teams
+  // Group teams: with few tokens the epilogue's cost is per group, not per
+  // column, so two teams take alternate groups and add up at tile ends.
+  static constexpr int kTeamsG = (MT <= 32) ? 2 : 1;
+  static constexpr int kTeamWarps = 4 * kTeams;                  // warps of one group team
+  static constexpr int kEpiWarps = kTeamWarps * kTeamsG;
   static constexpr int kCols = MT / kTeams;                      // token columns per epilogue thread
   static_assert(kCols % 8 == 0, "epilogue columns must be a multiple of 8");
   static constexpr int kEpiThreads = 32 * kEpiWarps;
@@ -89,14 +95,21 @@ struct GemmCfg {
   static constexpr int kScaleAhead = 4;
   static constexpr int kScaleSlots = kScaleAhead + 1;
   static constexpr int kScaleBytes = kScaleSlots * kEpiThreads * 4;
+  static constexpr int kXchgBytes = (kTeamsG > 1) ? MT * kTileN * 4 : 0;   // team sums
   // ring depths from the shared-memory budget
   static constexpr int kNumCv = (!kInt8 && MT >= 64) ? 2 : 4;
-  static constexpr int kAvail = kSmemLimit - 1024 - kBarBytes - kScaleBytes - kNumCv * kCvBytes;
+  // Converter teams take alternate units (fewer hand-offs per unit) when the
+  // widened-tile ring is deep enough for two units in conversion at once.
+  static constexpr int kConvTeams = (kNumCv >= 4) ? 2 : 1;
+  static constexpr int kConvTeamWarps = kConvWarps / kConvTeams;
+  static constexpr int kAvail =
+      kSmemLimit - 1024 - kBarBytes - kScaleBytes - kXchgBytes - kNumCv * kCvBytes;
   static constexpr int kNumX = cmin(kMaxX, (kAvail - 6 * kPkBytes) / kXBytes);
   static constexpr int kNumPk = cmin(kMaxPk, (kAvail - kNumX * kXBytes) / kPkBytes);
   static_assert(kNumX >= 2 && kNumPk >= 6, "shared memory too small for the rings");
   static constexpr int kSmemBytes =
-      1024 + kNumPk * kPkBytes + kNumCv * kCvBytes + kNumX * kXBytes + kScaleBytes + kBarBytes;
+      1024 + kNumPk * kPkBytes + kNumCv * kCvBytes + kNumX * kXBytes + kScaleBytes + kXchgBytes +
+      kBarBytes;
   static_assert(kSmemBytes <= kSmemLimit, "shared memory overflow");
   static constexpr int kTmemCols = pow2_at_least(kNumAcc * MT);
   static_assert(kTmemCols <= 512, "tensor memory overflow");
@@ -181,11 +194,14 @@ __device__ __forceinline__ bool take_tile_ticket(const GemmArgs& args, long long
   const long long tile_u0 = t * args.ku;
   const long long c_lo = unit_owner(tile_u0, units, grid);
   const long long c_hi = unit_owner(tile_u0 + args.ku - 1, units, grid);
-  __threadfence();   // the share, seen through an mbarrier, before the ticket
-  const uint32_t old = atomicAdd(&args.counters[c_lo], 1u);
-  const bool last = (old == static_cast<uint32_t>(c_hi - c_lo));
-  if (last) __threadfence();   // every share, before the reads of the reduction
-  return last;
+  // Release: this CTA's share (seen by this thread through an mbarrier) is
+  // published with the ticket.  Acquire: the last contributor sees every share.
+  uint32_t old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;"
+               : "=r"(old)
+               : "l"(args.counters + c_lo)
+               : "memory");
+  return old == static_cast<uint32_t>(c_hi - c_lo);
 }
 
 template <bool kInt8, int MT>
@@ -202,7 +218,8 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   uint8_t* cv_buf = pk_buf + NPK * kPkBytes;
   uint8_t* x_buf = cv_buf + NCV * C::kCvBytes;
   uint32_t* scale_ring = reinterpret_cast<uint32_t*>(x_buf + NX * C::kXBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(scale_ring + C::kScaleSlots * C::kEpiThreads);
+  float* xchg = reinterpret_cast<float*>(scale_ring + C::kScaleSlots * C::kEpiThreads);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(xchg) + C::kXchgBytes);
   uint64_t* pk_full = bars;
   uint64_t* pk_empty = pk_full + kMaxPk;
   uint64_t* cv_full = pk_empty + kMaxPk;
@@ -234,10 +251,10 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NPK; ++s) {
       mbar_init(smem_u32(&pk_full[s]), 1);
-      mbar_init(smem_u32(&pk_empty[s]), kConvWarps);
+      mbar_init(smem_u32(&pk_empty[s]), C::kConvTeamWarps);
     }
     for (int s = 0; s < NCV; ++s) {
-      mbar_init(smem_u32(&cv_full[s]), kConvWarps);
+      mbar_init(smem_u32(&cv_full[s]), C::kConvTeamWarps);
       mbar_init(smem_u32(&cv_empty[s]), 1);
     }
     for (int s = 0; s < NX; ++s) {
@@ -246,10 +263,10 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     }
     for (int b = 0; b < kNumAcc; ++b) {
       mbar_init(smem_u32(&acc_full[b]), 1);
-      mbar_init(smem_u32(&acc_empty[b]), C::kEpiWarps);
+      mbar_init(smem_u32(&acc_empty[b]), C::kTeamWarps);
     }
     mbar_init(smem_u32(mma_done), 2);
-    mbar_init(smem_u32(flush_bar), C::kEpiWarps);
+    mbar_init(smem_u32(flush_bar), C::kTeamWarps);
     mbar_init(smem_u32(ticket_bar), 1);
     misc[3] = 0;
     mbar_init(smem_u32(epi_sync), C::kEpiWarps);
@@ -271,6 +288,9 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   const uint32_t tmem_base = misc[0];
   QSPEC_TRACE_AT(tmem_base & 0xFFFF);
   if (threadIdx.x == 0) QSPEC_PHASE(1);
+  // The next grid may be scheduled as SMs free up; it waits for this one to
+  // complete before it reads inputs or writes anything.
+  if (threadIdx.x == 0) grid_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------ packed-weight producer
@@ -283,6 +303,10 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     const long long t_head = u_begin / ku;
     const long long head_end = (u_end < (t_head + 1) * ku) ? u_end : (t_head + 1) * ku;
     bool head_pending = (u_begin < u_end) && head_end < u_end && u_begin != t_head * ku;
+    // W4A16: the weights may come from the preceding grid.  W4A4 always runs
+    // behind its own activation quantization, which launched this grid only
+    // after the grid before it had completed.
+    if constexpr (!kInt8) grid_dependency_wait();
     int i = 0;
     UnitCursor cur;
     cur.init(u_begin, ku, args.m_tiles);
@@ -403,9 +427,12 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     __syncwarp();
   } else if (warp >= kCtlWarps && warp < kCtlWarps + kConvWarps) {
     // ------------------------------------------------ converters
-    const int ct = threadIdx.x - kCtlWarps * 32;
-    int i = 0;
-    for (long long u = u_begin; u < u_end; ++u, ++i) {
+    // With two teams of four warps taking alternate units, each unit pays the
+    // hand-off (waits, proxy fence, arrivals) four times, not eight.
+    const int cteam = (warp - kCtlWarps) / C::kConvTeamWarps;
+    const int ct = threadIdx.x - (kCtlWarps + cteam * C::kConvTeamWarps) * 32;
+    int i = cteam;
+    for (long long u = u_begin + cteam; u < u_end; u += C::kConvTeams, i += C::kConvTeams) {
       const int sp = i % NPK;
       const int sc = i % NCV;
       bool ok = warp_wait(smem_u32(&pk_full[sp]), (i / NPK) & 1, abort_flag, args.status);
@@ -416,8 +443,8 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       const uint8_t* src = pk_buf + sp * kPkBytes;
       uint8_t* dst = cv_buf + sc * C::kCvBytes;
 #pragma unroll
-      for (int it = 0; it < kPkBytes / 16 / (kConvWarps * 32); ++it) {
-        const int ch = ct + it * kConvWarps * 32;   // 16-byte chunk of the packed tile
+      for (int it = 0; it < kPkBytes / 16 / (C::kConvTeamWarps * 32); ++it) {
+        const int ch = ct + it * C::kConvTeamWarps * 32;   // 16-byte chunk of the packed tile
         const uint4 v = *reinterpret_cast<const uint4*>(src + ch * 16);
         const int r = ch >> 2;                      // weight row within the tile
         const int p = ch & 3;                       // which 32 input channels of the row
@@ -426,14 +453,14 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
           uint32_t o[8];
 #pragma unroll
           for (int wi = 0; wi < 4; ++wi) {
-            // offset-binary q + 8 per byte: even k in e, odd k in od
-            const uint32_t e = (wv[wi] & 0x0F0F0F0Fu) ^ 0x08080808u;
-            const uint32_t od = ((wv[wi] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
-            const uint32_t t0 = prmt(e, od, 0x5140u);   // k0 k1 k2 k3
-            const uint32_t t1 = prmt(e, od, 0x7362u);   // k4 k5 k6 k7
-            // q + 8 in [0,15] -> signed byte q, no carries between bytes
-            o[2 * wi] = (t0 + 0x78787878u) ^ 0x80808080u;
-            o[2 * wi + 1] = (t1 + 0x78787878u) ^ 0x80808080u;
+            // A two's-complement nibble in the high half of a byte is the
+            // signed byte 16 q, so masking alone widens: odd k are already
+            // there, even k move up by 4 bits.  The accumulators come out
+            // as 16 x the exact sums; the epilogue divides by 16 exactly.
+            const uint32_t od = wv[wi] & 0xF0F0F0F0u;          // 16 q of k1 k3 k5 k7
+            const uint32_t ev = (wv[wi] << 4) & 0xF0F0F0F0u;   // 16 q of k0 k2 k4 k6
+            o[2 * wi] = prmt(ev, od, 0x5140u);                 // k0 k1 k2 k3
+            o[2 * wi + 1] = prmt(ev, od, 0x7362u);             // k4 k5 k6 k7
           }
           uint8_t* row = dst + r * 128;
           const int c0 = 2 * p, c1 = 2 * p + 1;
@@ -470,10 +497,13 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     // ------------------------------------------------ epilogue
     const int ew = warp - (kCtlWarps + kConvWarps);
     const int quad = warp & 3;                 // tensor-memory lanes this warp may read
-    const int team = ew >> 2;
+    const int team = (ew >> 2) % C::kTeams;    // column team
+    const int gteam = (ew >> 2) / C::kTeams;   // group team: groups j with j % kTeamsG == gteam
+    const bool writer = (gteam == 0);          // group team 0 writes the tile results
     const int col0 = team * C::kCols;
     const int row = quad * 32 + lane;
     const int et = ew * 32 + lane;             // 0 .. kEpiThreads-1
+    grid_dependency_wait();   // no global write before the preceding grid is done
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
 
     // Group scales.  Each thread copies the aligned 32-bit word holding its
@@ -489,21 +519,37 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     UnitCursor pf;
     pf.init(u_begin, ku, args.m_tiles);
     int pf_h = 0, pf_j = 0, pf_slot = 0;
-    auto issue_scale = [&]() {
-      if (pf_j < groups_total) {
-        const int nn = pf.n_tile * kTileN + row;
-        if (nn < args.N) {
-          const long long idx =
-              static_cast<long long>(nn) * args.groups_per_row + pf.kc * gpu + pf_h;
-          const long long w0 = idx & ~1ll;
-          cp_async_4(slot0 + pf_slot * kSlotStride, args.ws + w0, (w0 + 1 < ws_elems) ? 4u : 2u);
-        }
-        if (++pf_h == gpu) {
-          pf_h = 0;
-          pf.next(ku, args.m_tiles);
+    // scale index of the prefetch cursor's group; groups of a tile are consecutive
+    bool pf_row_ok = pf.n_tile * kTileN + row < args.N;
+    long long pf_idx = static_cast<long long>(pf.n_tile * kTileN + row) * args.groups_per_row +
+                       static_cast<long long>(pf.kc) * gpu;
+    auto pf_advance = [&]() {
+      ++pf_j;
+      ++pf_idx;
+      if (++pf_h == gpu) {
+        pf_h = 0;
+        if (++pf.kc == ku) {   // next tile: scales restart at the row's group 0
+          pf.kc = 0;
+          if (++pf.m_tile == args.m_tiles) {
+            pf.m_tile = 0;
+            ++pf.n_tile;
+          }
+          const int nn = pf.n_tile * kTileN + row;
+          pf_row_ok = nn < args.N;
+          pf_idx = static_cast<long long>(nn) * args.groups_per_row;
         }
       }
-      ++pf_j;
+    };
+    // copy the scale of this team's next group
+    auto issue_scale = [&]() {
+      while (pf_j < groups_total && (pf_j % C::kTeamsG) != gteam) pf_advance();
+      if (pf_j < groups_total) {
+        if (pf_row_ok) {
+          const long long w0 = pf_idx & ~1ll;
+          cp_async_4(slot0 + pf_slot * kSlotStride, args.ws + w0, (w0 + 1 < ws_elems) ? 4u : 2u);
+        }
+        pf_advance();
+      }
       if (++pf_slot == C::kScaleSlots) pf_slot = 0;
       cp_async_commit();   // one group per scale, possibly empty, keeps the count uniform
     };
@@ -519,7 +565,9 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       for (int c = 0; c < C::kCols; ++c) {
         const int m = m0 + c;
         if (m < args.M) {
-          const float v = kInt8 ? args.s_a[m] * run[c] : run[c];
+          // int8 mode: run holds 16 x the sums; s_a / 16 is exact and so is
+          // the product's rounding relative to the unscaled one
+          const float v = kInt8 ? (args.s_a[m] * 0.0625f) * run[c] : run[c];
           args.y[static_cast<long long>(m) * args.N + n] = v;
         }
       }
@@ -581,6 +629,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       for (; u < seg_end && ok; ++u, cur.next(ku, args.m_tiles)) {
         const int kc = cur.kc;
         for (int h = 0; h < gpu; ++h, ++j) {
+          if ((j % C::kTeamsG) != gteam) continue;   // the other group team's group
           const int b = j % kNumAcc;
           const uint32_t pha = (j / kNumAcc) & 1;
           const int g = kc * gpu + h;
@@ -625,7 +674,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
                   const int m = m0 + c0 + e;
                   if (c0 + e < C::kCols && m < args.M)
                     args.dbg_acc[(static_cast<long long>(m) * args.N + n) * args.groups_per_row + g] =
-                        static_cast<int>(v[e]);
+                        static_cast<int>(v[e]) >> 4;   // exact: a multiple of 16
                 }
               }
             }
@@ -635,20 +684,38 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       if (!ok) break;
       if (et == 0) QSPEC_PHASE(u >= u_end ? 5 : 7);
 
+      if constexpr (C::kTeamsG > 1) {
+        // group team 1 hands its sums to team 0 through shared memory
+        float* xc = xchg + (col0 * kTileN + row);
+        if (!writer) {
+#pragma unroll
+          for (int c = 0; c < C::kCols; ++c) xc[c * kTileN] = run[c];
+        }
+        if (!epi_barrier()) break;
+        if (writer) {
+#pragma unroll
+          for (int c = 0; c < C::kCols; ++c) run[c] += xc[c * kTileN];
+        }
+        if (!epi_barrier()) break;   // the exchange buffer is free again
+      }
       const bool full = (seg_start == tile_u0) && (seg_end == tile_u0 + ku);
       if (full) {
-        write_y(n, m0);
+        if (writer) write_y(n, m0);
       } else {
         const int k = (seg_start == u_begin) ? 0 : 1;
         float* mine = args.partials + static_cast<long long>(2 * cta + k) * MT * kTileN;
+        if (writer) {
 #pragma unroll
-        for (int c = 0; c < C::kCols; ++c) mine[(col0 + c) * kTileN + row] = run[c];
+          for (int c = 0; c < C::kCols; ++c) mine[(col0 + c) * kTileN + row] = run[c];
+        }
         if (seg_end < u_end) {
           // The CTA's first tile with more to follow: publish the share and go
           // on; the weight producer takes the ticket.
-          __syncwarp();
-          if (elect_one_lane()) mbar_arrive(smem_u32(flush_bar));
-          __syncwarp();
+          if (writer) {
+            __syncwarp();
+            if (elect_one_lane()) mbar_arrive(smem_u32(flush_bar));
+            __syncwarp();
+          }
         } else {
           // The CTA's last tile: take the ticket here.
           if (!epi_barrier()) break;
@@ -664,7 +731,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       ok = warp_wait(smem_u32(ticket_bar), 0, abort_flag, args.status);
       if (ok && misc[3] != 0u) to_reduce[n_reduce++] = t_head;
     }
-    for (int r = 0; ok && r < n_reduce; ++r) reduce_tile(to_reduce[r]);
+    for (int r = 0; ok && writer && r < n_reduce; ++r) reduce_tile(to_reduce[r]);
     cp_async_wait<0>();
   }
 

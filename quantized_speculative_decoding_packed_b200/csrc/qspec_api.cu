@@ -164,12 +164,15 @@ qspec_status launch_qgemm_t(const CUtensorMap& tw, const CUtensorMap& tx, const 
   cfg.blockDim = dim3(C::kThreads);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
+  // Programmatic dependent launch: the GEMM's set-up overlaps the end of the
+  // preceding kernel (its activation quantization, or the previous GEMM) and,
+  // in W4A4 mode, so does its weight stream; it waits for that grid before it
+  // reads activations or writes anything.
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
-  // W4A4 follows its own activation-quantization kernel: overlap with it.
   cfg.attrs = attr;
-  cfg.numAttrs = kInt8 ? 1 : 0;
+  cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, qgemm_kernel<kInt8, MT>, tw, tx, a) != cudaSuccess) {
     cudaGetLastError();
     return QSPEC_ERR_CUDA;
@@ -234,8 +237,22 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
   if constexpr (kInt8) {
     int8_t* xq = reinterpret_cast<int8_t*>(wsp + p.off_xq);
     float* sa = reinterpret_cast<float*>(wsp + p.off_sa);
-    quant_act_kernel<false><<<static_cast<unsigned>(m), 256, 0, stream>>>(x, k, xq, sa);
-    if (cudaGetLastError() != cudaSuccess) return QSPEC_ERR_CUDA;
+    // Also a programmatic dependent: it waits for the preceding grid itself.
+    cudaLaunchConfig_t qc = {};
+    qc.gridDim = dim3(static_cast<unsigned>(m));
+    qc.blockDim = dim3(256);
+    qc.stream = stream;
+    cudaLaunchAttribute qa[1];
+    qa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    qa[0].val.programmaticStreamSerializationAllowed = 1;
+    qc.attrs = qa;
+    qc.numAttrs = 1;
+    void* qout = xq;
+    if (cudaLaunchKernelEx(&qc, quant_act_kernel<false>, x, static_cast<int64_t>(k), qout, sa) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return QSPEC_ERR_CUDA;
+    }
     a.s_a = sa;
     if (!make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, xq, m, k, p.mt, 128,
                    CU_TENSOR_MAP_SWIZZLE_128B))

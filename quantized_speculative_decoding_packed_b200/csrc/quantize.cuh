@@ -80,9 +80,12 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
   const uint16_t* xr = x + row * k;
   const int tid = threadIdx.x;
   QSPEC_TRACE_AT(1);
-  // The GEMM that consumes this kernel's output is launched as a programmatic
-  // dependent: it may start streaming weights now and waits for our results
-  // (griddepcontrol.wait) only where it reads them.
+  // This kernel may be launched as a programmatic dependent of the previous
+  // grid: wait for it (complete, memory flushed; a no-op otherwise), then let
+  // the GEMM that consumes our output launch.  That GEMM can then stream its
+  // weights at once, since whatever wrote them has finished, and waits for
+  // this kernel (griddepcontrol.wait) only where it reads x and s_a.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (!QSPEC_ALIGN_OK(reinterpret_cast<uintptr_t>(xr), 16) ||
       !QSPEC_ALIGN_OK(reinterpret_cast<uintptr_t>(out), 8))

@@ -177,3 +177,57 @@ def test_one_workspace_shared_across_shapes(qs):
         assert_close_1e3(y4.cpu().numpy()[:, cols], orc.gemm_w4a4(gi.x, q, s_h, g))
         assert_close_1e3(y16.cpu().numpy()[:, cols], orc.gemm_w4a16(gi.x, q, s_h, g))
         assert qs.workspace_status(work) == 0
+
+
+def test_back_to_back_calls_overlap_safely(qs):
+    """Calls are launched so that each may start while the previous finishes.
+
+    A chain of W4A4 and W4A16 calls on one stream, with no synchronisation,
+    shares one workspace (split-tile shares and tickets, quantized
+    activations) and rewrites the same outputs; run eagerly and as a CUDA
+    graph, every output must be bit-identical to a standalone call.
+    """
+    shapes = [(16, 12288, 4096), (80, 4096, 11008), (16, 4096, 11008), (80, 12288, 4096)]
+    ops, want = [], []
+    need = 0
+    for i, (m, n, k) in enumerate(shapes):
+        gi = synth.gemm_inputs("llama2_7b", m, n, k, 128, stream=60 + i)
+        wq, ws = qs.quantize_weights(cuda_f32(gi.w), 128)
+        x = cuda_bf16(gi.x_bits)
+        mode = "w4a4" if m == 16 else "w4a16"
+        fn = qs.gemm_w4a4 if mode == "w4a4" else qs.gemm_w4a16
+        want.append(fn(x, wq, ws, 128).clone())            # standalone reference
+        ops.append((fn, x, wq, ws, m, n))
+        need = max(need, qs.workspace_size(qs.OP_GEMM_W4A4, m, n, k, 128))
+    torch.cuda.synchronize()
+    work = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    outs = {}                                              # one output buffer per (m, n)
+    for (fn, x, wq, ws, m, n) in ops:
+        outs.setdefault((m, n), torch.empty((m, n), dtype=torch.float32, device="cuda"))
+
+    def chain():
+        for _ in range(3):
+            for (fn, x, wq, ws, m, n) in ops:
+                fn(x, wq, ws, 128, y=outs[(m, n)], work=work)
+
+    for y in outs.values():
+        y.fill_(float("nan"))
+    chain()
+    torch.cuda.synchronize()
+    for (fn, x, wq, ws, m, n), ref in zip(ops, want):
+        assert torch.equal(outs[(m, n)], ref)
+    assert qs.workspace_status(work) == 0
+
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        chain()
+    for y in outs.values():
+        y.fill_(float("nan"))
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    for (fn, x, wq, ws, m, n), ref in zip(ops, want):
+        assert torch.equal(outs[(m, n)], ref)
+    assert qs.workspace_status(work) == 0
