@@ -5,8 +5,9 @@
 // notes that the modes differ mainly in how activations are handled.  This
 // one kernel template serves both from the same `wq`/`ws` bytes:
 //
-//   W4A4  (kInt8 = true):  nibbles widened to int8 (as 16 q: two masks and
-//         two byte permutes per 8 weights) in shared memory, tcgen05.mma
+//   W4A4  (kInt8 = true):  nibbles widened to int8 (as 16 q, three integer
+//         ops per 8 weights, each 8 channels in the order 0,2,4,6,1,3,5,7,
+//         which the activation quantizer matches) in shared memory, tcgen05.mma
 //         kind::i8 (s8 x s8 -> s32 in tensor memory), one exact int32
 //         accumulator per weight group (16 acc_g); epilogue
 //         y = (s_a[m] / 16) * sum_g s_h[n,g] * (16 acc_g), bit-identical to
@@ -56,27 +57,32 @@ namespace qspec {
 constexpr int kTileN = 128;                      // weight rows per tile (MMA M)
 constexpr int kUnitK = 128;                      // input channels per unit
 constexpr int kPkBytes = kTileN * kUnitK / 2;    // packed bytes per unit
-constexpr int kNumAcc = 4;                       // tensor-memory group ring
-constexpr int kConvWarps = 8;
+constexpr int kConvWarps = 8;                    // two teams of four (one per lane quadrant)
+constexpr int kConvTeams = 2;                    // the teams take alternate units
+constexpr int kConvTeamWarps = kConvWarps / kConvTeams;
 constexpr int kCtlWarps = 4;
 constexpr int kSmemLimit = 232448;               // sm_100 dynamic shared memory per CTA
 constexpr int kMaxGrid = 1024;                   // ticket slots in the workspace
-constexpr int kMaxPk = 16, kMaxCv = 4, kMaxX = 8;
+constexpr int kMaxPk = 24, kMaxA = 8, kMaxAcc = 8, kMaxX = 8;
+constexpr int kTmemCols = 512;                   // all of tensor memory: one CTA per SM
 
-__host__ __device__ constexpr int pow2_at_least(int v) {
-  int p = 32;
-  while (p < v) p <<= 1;
-  return p;
-}
 __host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
+__host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
 
 template <bool kInt8, int MT>
 struct GemmCfg {
   static_assert(MT % 16 == 0 && MT >= 16 && MT <= 128, "token tile must be 16..128, step 16");
   static constexpr int kElem = kInt8 ? 1 : 2;                    // bytes per widened element
   static constexpr int kAtoms = kUnitK * kElem / 128;            // 128-byte K atoms per row
-  static constexpr int kCvBytes = kTileN * kUnitK * kElem;       // widened weight tile
   static constexpr int kXBytes = MT * 128 * kAtoms;              // activation tile
+  // Widened weight units live in tensor memory (lane = weight row, 32-bit
+  // columns along K): 32 columns of int8 or 64 of bf16 per unit, then the
+  // per-group accumulators (MT columns each) in what is left.
+  static constexpr int kACols = kUnitK * kElem / 4;
+  static constexpr int kNumA = (kInt8 && MT <= 32) ? kMaxA : 4;
+  static constexpr int kAccCol0 = kNumA * kACols;
+  static constexpr int kNumAcc = cmin(kMaxAcc, (kTmemCols - kAccCol0) / MT);
+  static_assert(kNumAcc >= 2, "tensor memory too small for two accumulators");
   static constexpr int kMmaK = kInt8 ? 32 : 16;
   static constexpr int kMmas = kUnitK / kMmaK;                   // MMAs per unit
   static constexpr int kTeams = (MT <= 48) ? 1 : (MT <= 96 ? 2 : 4);   // column teams
@@ -96,23 +102,15 @@ struct GemmCfg {
   static constexpr int kScaleSlots = kScaleAhead + 1;
   static constexpr int kScaleBytes = kScaleSlots * kEpiThreads * 4;
   static constexpr int kXchgBytes = (kTeamsG > 1) ? MT * kTileN * 4 : 0;   // team sums
-  // ring depths from the shared-memory budget
-  static constexpr int kNumCv = (!kInt8 && MT >= 64) ? 2 : 4;
-  // Converter teams take alternate units (fewer hand-offs per unit) when the
-  // widened-tile ring is deep enough for two units in conversion at once.
-  static constexpr int kConvTeams = (kNumCv >= 4) ? 2 : 1;
-  static constexpr int kConvTeamWarps = kConvWarps / kConvTeams;
-  static constexpr int kAvail =
-      kSmemLimit - 1024 - kBarBytes - kScaleBytes - kXchgBytes - kNumCv * kCvBytes;
-  static constexpr int kNumX = cmin(kMaxX, (kAvail - 6 * kPkBytes) / kXBytes);
+  // Ring depths from the shared-memory budget: packed weights first (they
+  // cover HBM latency), activations (an L2 hit) with what is left.
+  static constexpr int kAvail = kSmemLimit - 1024 - kBarBytes - kScaleBytes - kXchgBytes;
+  static constexpr int kNumX = cmin(kMaxX, cmax(3, (kAvail - 16 * kPkBytes) / kXBytes));
   static constexpr int kNumPk = cmin(kMaxPk, (kAvail - kNumX * kXBytes) / kPkBytes);
-  static_assert(kNumX >= 2 && kNumPk >= 6, "shared memory too small for the rings");
+  static_assert(kNumX >= 3 && kNumPk >= 8, "shared memory too small for the rings");
   static constexpr int kSmemBytes =
-      1024 + kNumPk * kPkBytes + kNumCv * kCvBytes + kNumX * kXBytes + kScaleBytes + kXchgBytes +
-      kBarBytes;
+      1024 + kNumPk * kPkBytes + kNumX * kXBytes + kScaleBytes + kXchgBytes + kBarBytes;
   static_assert(kSmemBytes <= kSmemLimit, "shared memory overflow");
-  static constexpr int kTmemCols = pow2_at_least(kNumAcc * MT);
-  static_assert(kTmemCols <= 512, "tensor memory overflow");
 };
 
 struct GemmArgs {
@@ -209,26 +207,25 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     qgemm_kernel(const __grid_constant__ CUtensorMap tmap_w,
                  const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ GemmArgs args) {
   using C = GemmCfg<kInt8, MT>;
-  constexpr int NPK = C::kNumPk, NCV = C::kNumCv, NX = C::kNumX;
+  constexpr int NPK = C::kNumPk, NA = C::kNumA, NX = C::kNumX, NACC = C::kNumAcc;
   extern __shared__ uint8_t smem_raw[];
   QSPEC_STAMP_DECL
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* pk_buf = smem;
-  uint8_t* cv_buf = pk_buf + NPK * kPkBytes;
-  uint8_t* x_buf = cv_buf + NCV * C::kCvBytes;
+  uint8_t* x_buf = pk_buf + NPK * kPkBytes;
   uint32_t* scale_ring = reinterpret_cast<uint32_t*>(x_buf + NX * C::kXBytes);
   float* xchg = reinterpret_cast<float*>(scale_ring + C::kScaleSlots * C::kEpiThreads);
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(xchg) + C::kXchgBytes);
   uint64_t* pk_full = bars;
   uint64_t* pk_empty = pk_full + kMaxPk;
-  uint64_t* cv_full = pk_empty + kMaxPk;
-  uint64_t* cv_empty = cv_full + kMaxCv;
-  uint64_t* x_full = cv_empty + kMaxCv;
+  uint64_t* a_full = pk_empty + kMaxPk;    // widened unit in tensor memory
+  uint64_t* a_empty = a_full + kMaxA;
+  uint64_t* x_full = a_empty + kMaxA;
   uint64_t* x_empty = x_full + kMaxX;
   uint64_t* acc_full = x_empty + kMaxX;
-  uint64_t* acc_empty = acc_full + kNumAcc;
-  uint64_t* mma_done = acc_empty + kNumAcc;
+  uint64_t* acc_empty = acc_full + kMaxAcc;
+  uint64_t* mma_done = acc_empty + kMaxAcc;
   uint64_t* flush_bar = mma_done + 1;   // the head split tile's share is published
   uint64_t* ticket_bar = flush_bar + 1; // ... and its ticket taken (result in misc[3])
   uint64_t* epi_sync = ticket_bar + 1;
@@ -251,17 +248,17 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NPK; ++s) {
       mbar_init(smem_u32(&pk_full[s]), 1);
-      mbar_init(smem_u32(&pk_empty[s]), C::kConvTeamWarps);
+      mbar_init(smem_u32(&pk_empty[s]), kConvTeamWarps);
     }
-    for (int s = 0; s < NCV; ++s) {
-      mbar_init(smem_u32(&cv_full[s]), C::kConvTeamWarps);
-      mbar_init(smem_u32(&cv_empty[s]), 1);
+    for (int s = 0; s < NA; ++s) {
+      mbar_init(smem_u32(&a_full[s]), kConvTeamWarps);
+      mbar_init(smem_u32(&a_empty[s]), 1);
     }
     for (int s = 0; s < NX; ++s) {
       mbar_init(smem_u32(&x_full[s]), 1);
       mbar_init(smem_u32(&x_empty[s]), 1);
     }
-    for (int b = 0; b < kNumAcc; ++b) {
+    for (int b = 0; b < NACC; ++b) {
       mbar_init(smem_u32(&acc_full[b]), 1);
       mbar_init(smem_u32(&acc_empty[b]), C::kTeamWarps);
     }
@@ -279,7 +276,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     prefetch_tensormap(&tmap_x);
   }
   if (warp == 2) {
-    tmem_alloc(smem_u32(&misc[0]), C::kTmemCols);
+    tmem_alloc(smem_u32(&misc[0]), kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -370,7 +367,8 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   } else if (warp == 2 || warp == 3) {
     // ------------------------------------------------ MMA issuers (even / odd units)
     // The whole warp walks the loop (waits are warp-uniform); one elected lane
-    // issues each tcgen05 instruction, which is cheaper than a lone lane.
+    // issues the tcgen05 instructions.  A (the widened weights) is read from
+    // tensor memory, B (the activations) from shared memory.
     constexpr uint32_t idesc = kInt8 ? idesc_i8(MT) : idesc_bf16(MT);
     const int per_group = C::kMmas / gpu;
     const int parity = warp - 2;
@@ -378,46 +376,41 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     bool ok = true;
     for (long long u = u_begin + parity; u < u_end && ok; u += 2, i += 2) {
       int j = i * gpu;
-      const int sc = i % NCV;
+      const int sa = i % NA;
       const int sx = i % NX;
-      QSPEC_STAMP(13, i);
-      ok = warp_wait(smem_u32(&cv_full[sc]), (i / NCV) & 1, abort_flag, args.status);
-      QSPEC_STAMP(14, i);
+      ok = warp_wait(smem_u32(&a_full[sa]), (i / NA) & 1, abort_flag, args.status);
       ok = ok && warp_wait(smem_u32(&x_full[sx]), (i / NX) & 1, abort_flag, args.status);
       if (!ok) break;
-      QSPEC_STAMP(3, i);
       tc_fence_after();
-      const uint32_t a_base = smem_u32(cv_buf + sc * C::kCvBytes);
+      const uint32_t a_col = tmem_base + static_cast<uint32_t>(sa * C::kACols);
       const uint32_t b_base = smem_u32(x_buf + sx * C::kXBytes);
       for (int h = 0; h < gpu; ++h, ++j) {
-        const int b = j % kNumAcc;
-        const uint32_t pha = (j / kNumAcc) & 1;
+        const int b = j % NACC;
+        const uint32_t pha = (j / NACC) & 1;
         ok = warp_wait(smem_u32(&acc_empty[b]), pha ^ 1, abort_flag, args.status);
         if (!ok) break;
         tc_fence_after();
-        if (h == 0) QSPEC_STAMP(8, i);
         // One elected lane issues the group's MMAs and its commit back to back.
         if (elect_one_lane()) {
+          const uint32_t d = tmem_base + static_cast<uint32_t>(C::kAccCol0 + b * MT);
           for (int kk = 0; kk < per_group; ++kk) {
-            const uint32_t kbyte = static_cast<uint32_t>(h * per_group + kk) * 32u;
+            const int step = h * per_group + kk;            // 32 bytes of K per step
+            const uint32_t kbyte = static_cast<uint32_t>(step) * 32u;
             const uint32_t atom = kbyte >> 7, within = kbyte & 127u;
-            const uint64_t a_desc = smem_desc_sw128(a_base + atom * (kTileN * 128) + within);
             const uint64_t b_desc = smem_desc_sw128(b_base + atom * (MT * 128) + within);
-            mma_ss<kInt8>(tmem_base + static_cast<uint32_t>(b * MT), a_desc, b_desc, idesc,
+            mma_ts<kInt8>(d, a_col + static_cast<uint32_t>(step * 8), b_desc, idesc,
                           kk > 0 ? 1u : 0u);
           }
           mma_commit(smem_u32(&acc_full[b]));
         }
         __syncwarp();
-        if (h == 0) QSPEC_STAMP(12, i);
       }
       if (!ok) break;
       if (elect_one_lane()) {
-        mma_commit(smem_u32(&cv_empty[sc]));
+        mma_commit(smem_u32(&a_empty[sa]));
         mma_commit(smem_u32(&x_empty[sx]));
       }
       __syncwarp();
-      QSPEC_STAMP(4, i);
       if (i == 0 && lane == 0) QSPEC_PHASE(3);
     }
     // All MMAs this warp issued have finished once mma_done completes.
@@ -427,47 +420,60 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     __syncwarp();
   } else if (warp >= kCtlWarps && warp < kCtlWarps + kConvWarps) {
     // ------------------------------------------------ converters
-    // With two teams of four warps taking alternate units, each unit pays the
-    // hand-off (waits, proxy fence, arrivals) four times, not eight.
-    const int cteam = (warp - kCtlWarps) / C::kConvTeamWarps;
-    const int ct = threadIdx.x - (kCtlWarps + cteam * C::kConvTeamWarps) * 32;
+    // Two teams of four warps (one per tensor-memory lane quadrant) take
+    // alternate units.  Thread = weight row = tensor-memory lane: it reads the
+    // row's 64 packed bytes (the TMA's 64-byte swizzle puts 16-byte chunk c of
+    // row r at c ^ ((r >> 1) & 3), so a quarter warp hits eight distinct bank
+    // groups), widens them in registers and stores them to its own lane.
+    const int cteam = (warp - kCtlWarps) / kConvTeamWarps;
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const uint32_t swz = static_cast<uint32_t>((r >> 1) & 3);
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     int i = cteam;
-    for (long long u = u_begin + cteam; u < u_end; u += C::kConvTeams, i += C::kConvTeams) {
+    for (long long u = u_begin + cteam; u < u_end; u += kConvTeams, i += kConvTeams) {
       const int sp = i % NPK;
-      const int sc = i % NCV;
+      const int sa = i % NA;
       bool ok = warp_wait(smem_u32(&pk_full[sp]), (i / NPK) & 1, abort_flag, args.status);
-      ok = ok && warp_wait(smem_u32(&cv_empty[sc]), ((i / NCV) & 1) ^ 1, abort_flag, args.status);
+      ok = ok && warp_wait(smem_u32(&a_empty[sa]), ((i / NA) & 1) ^ 1, abort_flag, args.status);
       if (!ok) break;
-      if (warp == kCtlWarps) QSPEC_STAMP(1, i);
-      if (i == 0 && ct == 0) QSPEC_PHASE(2);
-      const uint8_t* src = pk_buf + sp * kPkBytes;
-      uint8_t* dst = cv_buf + sc * C::kCvBytes;
+      if (i == 0 && r == 0) QSPEC_PHASE(2);
+      const uint8_t* rowp = pk_buf + sp * kPkBytes + r * (kUnitK / 2);
+      uint4 v[4];
 #pragma unroll
-      for (int it = 0; it < kPkBytes / 16 / (C::kConvTeamWarps * 32); ++it) {
-        const int ch = ct + it * C::kConvTeamWarps * 32;   // 16-byte chunk of the packed tile
-        const uint4 v = *reinterpret_cast<const uint4*>(src + ch * 16);
-        const int r = ch >> 2;                      // weight row within the tile
-        const int p = ch & 3;                       // which 32 input channels of the row
-        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-        if constexpr (kInt8) {
-          uint32_t o[8];
+      for (int c = 0; c < 4; ++c)
+        v[c] = *reinterpret_cast<const uint4*>(rowp + ((static_cast<uint32_t>(c) ^ swz) << 4));
+      // The packed slot may be refilled (by the async proxy) once every
+      // lane's reads are done.
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (elect_one_lane()) mbar_arrive(smem_u32(&pk_empty[sp]));
+      __syncwarp();
+      const uint32_t a_col = lane_base + static_cast<uint32_t>(sa * C::kACols);
+      if constexpr (kInt8) {
+        // A two's-complement nibble in the high half of a byte is the signed
+        // byte 16 q, so masking alone widens: odd k are already there, even k
+        // move up by 4 bits.  The accumulators come out as 16 x the exact
+        // sums; the epilogue divides by 16 exactly.  Each 8 channels land in
+        // the order (0,2,4,6,1,3,5,7), the order in which the activation
+        // quantizer stores them for this GEMM.
+        uint32_t o[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t wv[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
 #pragma unroll
           for (int wi = 0; wi < 4; ++wi) {
-            // A two's-complement nibble in the high half of a byte is the
-            // signed byte 16 q, so masking alone widens: odd k are already
-            // there, even k move up by 4 bits.  The accumulators come out
-            // as 16 x the exact sums; the epilogue divides by 16 exactly.
-            const uint32_t od = wv[wi] & 0xF0F0F0F0u;          // 16 q of k1 k3 k5 k7
-            const uint32_t ev = (wv[wi] << 4) & 0xF0F0F0F0u;   // 16 q of k0 k2 k4 k6
-            o[2 * wi] = prmt(ev, od, 0x5140u);                 // k0 k1 k2 k3
-            o[2 * wi + 1] = prmt(ev, od, 0x7362u);             // k4 k5 k6 k7
+            o[8 * c + 2 * wi] = (wv[wi] << 4) & 0xF0F0F0F0u;   // 16 q of k0 k2 k4 k6
+            o[8 * c + 2 * wi + 1] = wv[wi] & 0xF0F0F0F0u;      // 16 q of k1 k3 k5 k7
           }
-          uint8_t* row = dst + r * 128;
-          const int c0 = 2 * p, c1 = 2 * p + 1;
-          *reinterpret_cast<uint4*>(row + ((c0 ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-          *reinterpret_cast<uint4*>(row + ((c1 ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
-        } else {
-          uint8_t* row = dst + (p >> 1) * (kTileN * 128) + r * 128;
+        }
+        tmem_st16(a_col, o);
+        tmem_st16(a_col + 16, o + 16);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t wv[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+          uint32_t o[16];
 #pragma unroll
           for (int wi = 0; wi < 4; ++wi) {
             const uint32_t e = (wv[wi] & 0x0F0F0F0Fu) ^ 0x08080808u;
@@ -475,23 +481,19 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
             const uint32_t t0 = prmt(e, od, 0x5140u);   // k0 k1 k2 k3 (offset binary)
             const uint32_t t1 = prmt(e, od, 0x7362u);   // k4 k5 k6 k7
             // bf16 bit pattern 0x43uu is the value 128 + u
-            const uint32_t b0 = bf16x2_minus_136(prmt(t0, 0x43434343u, 0x4140u));
-            const uint32_t b1 = bf16x2_minus_136(prmt(t0, 0x43434343u, 0x4342u));
-            const uint32_t b2 = bf16x2_minus_136(prmt(t1, 0x43434343u, 0x4140u));
-            const uint32_t b3 = bf16x2_minus_136(prmt(t1, 0x43434343u, 0x4342u));
-            const int c = 4 * (p & 1) + wi;
-            *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = make_uint4(b0, b1, b2, b3);
+            o[4 * wi] = bf16x2_minus_136(prmt(t0, 0x43434343u, 0x4140u));
+            o[4 * wi + 1] = bf16x2_minus_136(prmt(t0, 0x43434343u, 0x4342u));
+            o[4 * wi + 2] = bf16x2_minus_136(prmt(t1, 0x43434343u, 0x4140u));
+            o[4 * wi + 3] = bf16x2_minus_136(prmt(t1, 0x43434343u, 0x4342u));
           }
+          tmem_st16(a_col + 16 * c, o);   // k = 32c .. 32c+31, two per column
         }
       }
-      fence_proxy_async_smem();
+      tmem_st_wait();
+      tc_fence_before();
       __syncwarp();
-      if (elect_one_lane()) {
-        mbar_arrive(smem_u32(&pk_empty[sp]));
-        mbar_arrive(smem_u32(&cv_full[sc]));
-      }
+      if (elect_one_lane()) mbar_arrive(smem_u32(&a_full[sa]));
       __syncwarp();
-      if (warp == kCtlWarps) QSPEC_STAMP(2, i);
     }
   } else if (warp >= kCtlWarps + kConvWarps) {
     // ------------------------------------------------ epilogue
@@ -630,8 +632,8 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
         const int kc = cur.kc;
         for (int h = 0; h < gpu; ++h, ++j) {
           if ((j % C::kTeamsG) != gteam) continue;   // the other group team's group
-          const int b = j % kNumAcc;
-          const uint32_t pha = (j / kNumAcc) & 1;
+          const int b = j % NACC;
+          const uint32_t pha = (j / NACC) & 1;
           const int g = kc * gpu + h;
           cp_async_wait<C::kScaleAhead - 1>();   // this thread's copy for group j has landed
           uint32_t sw;
@@ -644,7 +646,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
           if (!ok) break;
           if (ew == 0) QSPEC_STAMP(5, j);
           tc_fence_after();
-          const uint32_t taddr = lane_addr + static_cast<uint32_t>(b * MT + col0);
+          const uint32_t taddr = lane_addr + static_cast<uint32_t>(C::kAccCol0 + b * MT + col0);
 #pragma unroll
           for (int c0 = 0; c0 < C::kCols; c0 += 16) {
             uint32_t v[16];
@@ -744,7 +746,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   QSPEC_STAMP_FLUSH();
   if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::kTmemCols);
+    tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 

@@ -214,8 +214,9 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
   uint8_t* wsp = static_cast<uint8_t*>(workspace);
 
   CUtensorMap tw, tx;
+  // 64-byte swizzle: the converter threads read one 64-byte row each
   if (!make_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wq, n, k / 2, kTileN, kUnitK / 2,
-                 CU_TENSOR_MAP_SWIZZLE_NONE))
+                 CU_TENSOR_MAP_SWIZZLE_64B))
     return QSPEC_ERR_CUDA;
   GemmArgs a;
   a.M = static_cast<int>(m);

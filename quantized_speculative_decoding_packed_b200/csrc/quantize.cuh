@@ -130,13 +130,17 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
       for (int j = 0; j < 8; ++j) p |= (static_cast<uint32_t>(q[j]) & 0xFu) << (4 * j);
       *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(out) + row * (k / 2) + c / 2) = p;
     } else {
-      uint32_t lo = 0, hi = 0;
+      // int8 operand for the GEMM, each block of 8 channels stored in the
+      // order (0,2,4,6,1,3,5,7): the GEMM widens packed weight nibbles into
+      // the same order with masks alone, and a dot product does not depend
+      // on the order of its terms.
+      uint32_t ev = 0, od = 0;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        lo |= (static_cast<uint32_t>(q[j]) & 0xFFu) << (8 * j);
-        hi |= (static_cast<uint32_t>(q[j + 4]) & 0xFFu) << (8 * j);
+        ev |= (static_cast<uint32_t>(q[2 * j]) & 0xFFu) << (8 * j);
+        od |= (static_cast<uint32_t>(q[2 * j + 1]) & 0xFFu) << (8 * j);
       }
-      *reinterpret_cast<uint2*>(static_cast<int8_t*>(out) + row * k + c) = make_uint2(lo, hi);
+      *reinterpret_cast<uint2*>(static_cast<int8_t*>(out) + row * k + c) = make_uint2(ev, od);
     }
   }
 }
