@@ -61,7 +61,11 @@ constexpr int kConvWarps = 8;                    // two teams of four (one per l
 constexpr int kConvTeams = 2;                    // the teams take alternate units
 constexpr int kConvTeamWarps = kConvWarps / kConvTeams;
 constexpr int kCtlWarps = 4;
+#ifdef QSPEC_TRACE
+constexpr int kSmemLimit = 232448 - 4096;        // trace builds keep 4 KB of static stamps
+#else
 constexpr int kSmemLimit = 232448;               // sm_100 dynamic shared memory per CTA
+#endif
 constexpr int kMaxGrid = 1024;                   // ticket slots in the workspace
 constexpr int kMaxPk = 24, kMaxA = 8, kMaxAcc = 8, kMaxX = 8;
 constexpr int kTmemCols = 512;                   // all of tensor memory: one CTA per SM
@@ -86,9 +90,9 @@ struct GemmCfg {
   static constexpr int kMmaK = kInt8 ? 32 : 16;
   static constexpr int kMmas = kUnitK / kMmaK;                   // MMAs per unit
   static constexpr int kTeams = (MT <= 48) ? 1 : (MT <= 96 ? 2 : 4);   // column teams
-  // Group teams: with few tokens the epilogue's cost is per group, not per
-  // column, so two teams take alternate groups and add up at tile ends.
-  static constexpr int kTeamsG = (MT <= 32) ? 2 : 1;
+  // Group teams take alternate groups and add up at tile ends.  Measured: two
+  // teams are no faster than one at 16 tokens, so one is used.
+  static constexpr int kTeamsG = 1;
   static constexpr int kTeamWarps = 4 * kTeams;                  // warps of one group team
   static constexpr int kEpiWarps = kTeamWarps * kTeamsG;
   static constexpr int kCols = MT / kTeams;                      // token columns per epilogue thread
@@ -101,7 +105,7 @@ struct GemmCfg {
   static constexpr int kScaleAhead = 4;
   static constexpr int kScaleSlots = kScaleAhead + 1;
   static constexpr int kScaleBytes = kScaleSlots * kEpiThreads * 4;
-  static constexpr int kXchgBytes = (kTeamsG > 1) ? MT * kTileN * 4 : 0;   // team sums
+  static constexpr int kXchgBytes = (kTeamsG - 1) * MT * kTileN * 4;   // team sums
   // Ring depths from the shared-memory budget: packed weights first (they
   // cover HBM latency), activations (an L2 hit) with what is left.
   static constexpr int kAvail = kSmemLimit - 1024 - kBarBytes - kScaleBytes - kXchgBytes;
@@ -202,7 +206,9 @@ __device__ __forceinline__ bool take_tile_ticket(const GemmArgs& args, long long
   return old == static_cast<uint32_t>(c_hi - c_lo);
 }
 
-template <bool kInt8, int MT>
+// kDbg (int8 mode only): also write the per-group integer accumulators.  A
+// separate instantiation keeps those stores out of the hot loop's code.
+template <bool kInt8, int MT, bool kDbg>
 __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     qgemm_kernel(const __grid_constant__ CUtensorMap tmap_w,
                  const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ GemmArgs args) {
@@ -310,6 +316,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     for (long long u = u_begin; u < u_end; ++u, ++i, cur.next(ku, args.m_tiles)) {
       const int s = i % NPK;
       const uint32_t ph = (i / NPK) & 1;
+      QSPEC_STAMP(13, i);
       if (!warp_wait(smem_u32(&pk_empty[s]), ph ^ 1, abort_flag, args.status)) break;
       if (elect_one_lane()) {
         mbar_arrive_expect_tx(smem_u32(&pk_full[s]), kPkBytes);
@@ -381,6 +388,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       ok = warp_wait(smem_u32(&a_full[sa]), (i / NA) & 1, abort_flag, args.status);
       ok = ok && warp_wait(smem_u32(&x_full[sx]), (i / NX) & 1, abort_flag, args.status);
       if (!ok) break;
+      QSPEC_STAMP(3, i);
       tc_fence_after();
       const uint32_t a_col = tmem_base + static_cast<uint32_t>(sa * C::kACols);
       const uint32_t b_base = smem_u32(x_buf + sx * C::kXBytes);
@@ -411,6 +419,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
         mma_commit(smem_u32(&x_empty[sx]));
       }
       __syncwarp();
+      QSPEC_STAMP(4, i);
       if (i == 0 && lane == 0) QSPEC_PHASE(3);
     }
     // All MMAs this warp issued have finished once mma_done completes.
@@ -438,6 +447,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       ok = ok && warp_wait(smem_u32(&a_empty[sa]), ((i / NA) & 1) ^ 1, abort_flag, args.status);
       if (!ok) break;
       if (i == 0 && r == 0) QSPEC_PHASE(2);
+      if (quad == 0) QSPEC_STAMP(cteam == 0 ? 1 : 9, i);
       const uint8_t* rowp = pk_buf + sp * kPkBytes + r * (kUnitK / 2);
       uint4 v[4];
 #pragma unroll
@@ -494,6 +504,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       __syncwarp();
       if (elect_one_lane()) mbar_arrive(smem_u32(&a_full[sa]));
       __syncwarp();
+      if (quad == 0) QSPEC_STAMP(cteam == 0 ? 2 : 10, i);
     }
   } else if (warp >= kCtlWarps + kConvWarps) {
     // ------------------------------------------------ epilogue
@@ -530,7 +541,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       ++pf_idx;
       if (++pf_h == gpu) {
         pf_h = 0;
-        if (++pf.kc == ku) {   // next tile: scales restart at the row's group 0
+        if (__builtin_expect(++pf.kc == ku, 0)) {   // next tile: scales restart at group 0
           pf.kc = 0;
           if (++pf.m_tile == args.m_tiles) {
             pf.m_tile = 0;
@@ -635,16 +646,19 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
           const int b = j % NACC;
           const uint32_t pha = (j / NACC) & 1;
           const int g = kc * gpu + h;
+          if (ew == 0) QSPEC_STAMP(14, j);
           cp_async_wait<C::kScaleAhead - 1>();   // this thread's copy for group j has landed
           uint32_t sw;
           asm volatile("ld.shared.b32 %0, [%1];" : "=r"(sw) : "r"(slot0 + rd_slot * kSlotStride));
           if (++rd_slot == C::kScaleSlots) rd_slot = 0;
           const uint32_t hbits = ((row_par ^ static_cast<uint32_t>(g)) & 1u) ? (sw >> 16) : (sw & 0xFFFFu);
           const float sc = __half2float(__ushort_as_half(static_cast<unsigned short>(hbits)));
+          if (ew == 0) QSPEC_STAMP(15, j);
           issue_scale();   // refills the slot read one group ago
           ok = warp_wait(smem_u32(&acc_full[b]), pha, abort_flag, args.status);
           if (!ok) break;
           if (ew == 0) QSPEC_STAMP(5, j);
+          if (ew == C::kTeamWarps) QSPEC_STAMP(11, j);
           tc_fence_after();
           const uint32_t taddr = lane_addr + static_cast<uint32_t>(C::kAccCol0 + b * MT + col0);
 #pragma unroll
@@ -660,6 +674,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
               if (elect_one_lane()) mbar_arrive(smem_u32(&acc_empty[b]));
               __syncwarp();
               if (ew == 0) QSPEC_STAMP(6, j);
+              if (ew == C::kTeamWarps) QSPEC_STAMP(12, j);
               if (et == 0 && j == 0) QSPEC_PHASE(4);
             }
 #pragma unroll
@@ -669,8 +684,8 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
                 run[c0 + e] = fmaf(sc, a, run[c0 + e]);
               }
             }
-            if constexpr (kInt8) {
-              if (args.dbg_acc != nullptr && n < args.N) {
+            if constexpr (kInt8 && kDbg) {
+              if (n < args.N) {
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                   const int m = m0 + c0 + e;
@@ -681,22 +696,29 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
               }
             }
           }
+          if (ew == 0) QSPEC_STAMP(8, j);
         }
       }
       if (!ok) break;
       if (et == 0) QSPEC_PHASE(u >= u_end ? 5 : 7);
 
       if constexpr (C::kTeamsG > 1) {
-        // group team 1 hands its sums to team 0 through shared memory
-        float* xc = xchg + (col0 * kTileN + row);
+        // the other group teams hand their sums to team 0 through shared
+        // memory; team 0 adds them in team order
+        constexpr int kSlot = MT * kTileN;
         if (!writer) {
+          float* xc = xchg + (gteam - 1) * kSlot + (col0 * kTileN + row);
 #pragma unroll
           for (int c = 0; c < C::kCols; ++c) xc[c * kTileN] = run[c];
         }
         if (!epi_barrier()) break;
         if (writer) {
 #pragma unroll
-          for (int c = 0; c < C::kCols; ++c) run[c] += xc[c * kTileN];
+          for (int t2 = 0; t2 < C::kTeamsG - 1; ++t2) {
+            const float* xc = xchg + t2 * kSlot + (col0 * kTileN + row);
+#pragma unroll
+            for (int c = 0; c < C::kCols; ++c) run[c] += xc[c * kTileN];
+          }
         }
         if (!epi_barrier()) break;   // the exchange buffer is free again
       }

@@ -146,13 +146,13 @@ GemmPlan plan_gemm(bool int8_mode, int64_t m, int64_t n, int64_t k, int sm_count
   return p;
 }
 
-template <bool kInt8, int MT>
+template <bool kInt8, int MT, bool kDbg>
 qspec_status launch_qgemm_t(const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a,
                             int grid, int dev, cudaStream_t stream) {
   using C = GemmCfg<kInt8, MT>;
   static bool attr_set[kMaxDevices] = {};
   if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(qgemm_kernel<kInt8, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(qgemm_kernel<kInt8, MT, kDbg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess) {
       cudaGetLastError();
       return QSPEC_ERR_CUDA;
@@ -173,7 +173,7 @@ qspec_status launch_qgemm_t(const CUtensorMap& tw, const CUtensorMap& tx, const 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, qgemm_kernel<kInt8, MT>, tw, tx, a) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, qgemm_kernel<kInt8, MT, kDbg>, tw, tx, a) != cudaSuccess) {
     cudaGetLastError();
     return QSPEC_ERR_CUDA;
   }
@@ -183,14 +183,29 @@ qspec_status launch_qgemm_t(const CUtensorMap& tw, const CUtensorMap& tx, const 
 template <bool kInt8>
 qspec_status launch_qgemm(int mt, const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a,
                           int grid, int dev, cudaStream_t stream) {
+  const bool dbg = kInt8 && a.dbg_acc != nullptr;
   switch (mt) {
-    case 16: return launch_qgemm_t<kInt8, 16>(tw, tx, a, grid, dev, stream);
-    case 32: return launch_qgemm_t<kInt8, 32>(tw, tx, a, grid, dev, stream);
-    case 48: return launch_qgemm_t<kInt8, 48>(tw, tx, a, grid, dev, stream);
-    case 64: return launch_qgemm_t<kInt8, 64>(tw, tx, a, grid, dev, stream);
-    case 80: return launch_qgemm_t<kInt8, 80>(tw, tx, a, grid, dev, stream);
-    case 96: return launch_qgemm_t<kInt8, 96>(tw, tx, a, grid, dev, stream);
-    case 128: return launch_qgemm_t<kInt8, 128>(tw, tx, a, grid, dev, stream);
+    case 16:
+      return dbg ? launch_qgemm_t<kInt8, 16, kInt8>(tw, tx, a, grid, dev, stream)
+                 : launch_qgemm_t<kInt8, 16, false>(tw, tx, a, grid, dev, stream);
+    case 32:
+      return dbg ? launch_qgemm_t<kInt8, 32, kInt8>(tw, tx, a, grid, dev, stream)
+                 : launch_qgemm_t<kInt8, 32, false>(tw, tx, a, grid, dev, stream);
+    case 48:
+      return dbg ? launch_qgemm_t<kInt8, 48, kInt8>(tw, tx, a, grid, dev, stream)
+                 : launch_qgemm_t<kInt8, 48, false>(tw, tx, a, grid, dev, stream);
+    case 64:
+      return dbg ? launch_qgemm_t<kInt8, 64, kInt8>(tw, tx, a, grid, dev, stream)
+                 : launch_qgemm_t<kInt8, 64, false>(tw, tx, a, grid, dev, stream);
+    case 80:
+      return dbg ? launch_qgemm_t<kInt8, 80, kInt8>(tw, tx, a, grid, dev, stream)
+                 : launch_qgemm_t<kInt8, 80, false>(tw, tx, a, grid, dev, stream);
+    case 96:
+      return dbg ? launch_qgemm_t<kInt8, 96, kInt8>(tw, tx, a, grid, dev, stream)
+                 : launch_qgemm_t<kInt8, 96, false>(tw, tx, a, grid, dev, stream);
+    case 128:
+      return dbg ? launch_qgemm_t<kInt8, 128, kInt8>(tw, tx, a, grid, dev, stream)
+                 : launch_qgemm_t<kInt8, 128, false>(tw, tx, a, grid, dev, stream);
     default: return QSPEC_ERR_INVALID_ARG;
   }
 }
