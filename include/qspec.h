@@ -105,7 +105,9 @@ qspec_status qspec_quant_act(const uint16_t* x, int64_t m, int64_t k, uint8_t* x
  *           call that completes leaves it ready for the next one.
  *  dbg_acc  optional (may be NULL): [m][n][k/group] int32 out, the per-group
  *           integer accumulators.
- * Requires m, n >= 1, group in {64, 128}, k a multiple of 128.
+ * Requires m, n >= 1, group in {64, 128}, k a multiple of 128, and fewer than
+ * 2^22 work units ceil(m / T) * ceil(n / 128) * (k / 128), where the token
+ * tile T is m rounded up to a multiple of 16 for m <= 96, else 128.
  */
 qspec_status qspec_gemm_w4a4(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
                              const uint16_t* ws, int64_t n, int32_t group, float* y,

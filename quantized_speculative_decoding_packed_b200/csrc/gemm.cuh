@@ -90,11 +90,7 @@ struct GemmCfg {
   static constexpr int kMmaK = kInt8 ? 32 : 16;
   static constexpr int kMmas = kUnitK / kMmaK;                   // MMAs per unit
   static constexpr int kTeams = (MT <= 48) ? 1 : (MT <= 96 ? 2 : 4);   // column teams
-  // Group teams take alternate groups and add up at tile ends.  Measured: two
-  // teams are no faster than one at 16 tokens, so one is used.
-  static constexpr int kTeamsG = 1;
-  static constexpr int kTeamWarps = 4 * kTeams;                  // warps of one group team
-  static constexpr int kEpiWarps = kTeamWarps * kTeamsG;
+  static constexpr int kEpiWarps = 4 * kTeams;
   static constexpr int kCols = MT / kTeams;                      // token columns per epilogue thread
   static_assert(kCols % 8 == 0, "epilogue columns must be a multiple of 8");
   static constexpr int kEpiThreads = 32 * kEpiWarps;
@@ -105,15 +101,14 @@ struct GemmCfg {
   static constexpr int kScaleAhead = 4;
   static constexpr int kScaleSlots = kScaleAhead + 1;
   static constexpr int kScaleBytes = kScaleSlots * kEpiThreads * 4;
-  static constexpr int kXchgBytes = (kTeamsG - 1) * MT * kTileN * 4;   // team sums
   // Ring depths from the shared-memory budget: packed weights first (they
   // cover HBM latency), activations (an L2 hit) with what is left.
-  static constexpr int kAvail = kSmemLimit - 1024 - kBarBytes - kScaleBytes - kXchgBytes;
+  static constexpr int kAvail = kSmemLimit - 1024 - kBarBytes - kScaleBytes;
   static constexpr int kNumX = cmin(kMaxX, cmax(3, (kAvail - 16 * kPkBytes) / kXBytes));
   static constexpr int kNumPk = cmin(kMaxPk, (kAvail - kNumX * kXBytes) / kPkBytes);
   static_assert(kNumX >= 3 && kNumPk >= 8, "shared memory too small for the rings");
   static constexpr int kSmemBytes =
-      1024 + kNumPk * kPkBytes + kNumX * kXBytes + kScaleBytes + kXchgBytes + kBarBytes;
+      1024 + kNumPk * kPkBytes + kNumX * kXBytes + kScaleBytes + kBarBytes;
   static_assert(kSmemBytes <= kSmemLimit, "shared memory overflow");
 };
 
@@ -132,14 +127,19 @@ struct GemmArgs {
   float* partials;         // [2 * gridDim.x][MT][128]
 };
 
+// Unit arithmetic is 32-bit (the host keeps units below kMaxUnits and the
+// grid at most kMaxGrid, so no product reaches 2^32): a 64-bit division is a
+// long software sequence on the GPU.
+constexpr long long kMaxUnits = 1ll << 22;
+
 // First unit of CTA c when `units` are split over `grid` CTAs.
-__host__ __device__ __forceinline__ long long unit_begin(long long c, long long units,
-                                                         long long grid) {
+__host__ __device__ __forceinline__ uint32_t unit_begin(uint32_t c, uint32_t units,
+                                                        uint32_t grid) {
   return (c * units) / grid;
 }
 // The CTA that owns unit u.
-__host__ __device__ __forceinline__ long long unit_owner(long long u, long long units,
-                                                         long long grid) {
+__host__ __device__ __forceinline__ uint32_t unit_owner(uint32_t u, uint32_t units,
+                                                        uint32_t grid) {
   return ((u + 1) * grid - 1) / units;
 }
 
@@ -164,10 +164,10 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* v) {
 struct UnitCursor {
   int kc, m_tile, n_tile;
   __device__ __forceinline__ void init(long long u, int ku, int m_tiles) {
-    const long long t = u / ku;
-    kc = static_cast<int>(u - t * ku);
-    n_tile = static_cast<int>(t / m_tiles);
-    m_tile = static_cast<int>(t - static_cast<long long>(n_tile) * m_tiles);
+    const uint32_t t = static_cast<uint32_t>(u) / static_cast<uint32_t>(ku);
+    kc = static_cast<int>(static_cast<uint32_t>(u) - t * static_cast<uint32_t>(ku));
+    n_tile = static_cast<int>(t / static_cast<uint32_t>(m_tiles));
+    m_tile = static_cast<int>(t - static_cast<uint32_t>(n_tile) * static_cast<uint32_t>(m_tiles));
   }
   __device__ __forceinline__ void next(int ku, int m_tiles) {
     if (++kc == ku) {
@@ -176,6 +176,24 @@ struct UnitCursor {
         m_tile = 0;
         ++n_tile;
       }
+    }
+  }
+};
+
+// Position in a ring of n slots (slot, phase parity) for item index i,
+// advanced without divisions: step(by) for any by <= n.
+struct RingPos {
+  int slot;
+  uint32_t phase;
+  __device__ __forceinline__ void init(int i, int n) {
+    slot = i % n;
+    phase = static_cast<uint32_t>(i / n) & 1u;
+  }
+  __device__ __forceinline__ void step(int by, int n) {
+    slot += by;
+    if (slot >= n) {
+      slot -= n;
+      phase ^= 1u;
     }
   }
 };
@@ -221,8 +239,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   uint8_t* pk_buf = smem;
   uint8_t* x_buf = pk_buf + NPK * kPkBytes;
   uint32_t* scale_ring = reinterpret_cast<uint32_t*>(x_buf + NX * C::kXBytes);
-  float* xchg = reinterpret_cast<float*>(scale_ring + C::kScaleSlots * C::kEpiThreads);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(xchg) + C::kXchgBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(scale_ring + C::kScaleSlots * C::kEpiThreads);
   uint64_t* pk_full = bars;
   uint64_t* pk_empty = pk_full + kMaxPk;
   uint64_t* a_full = pk_empty + kMaxPk;    // widened unit in tensor memory
@@ -266,10 +283,10 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     }
     for (int b = 0; b < NACC; ++b) {
       mbar_init(smem_u32(&acc_full[b]), 1);
-      mbar_init(smem_u32(&acc_empty[b]), C::kTeamWarps);
+      mbar_init(smem_u32(&acc_empty[b]), C::kEpiWarps);
     }
     mbar_init(smem_u32(mma_done), 2);
-    mbar_init(smem_u32(flush_bar), C::kTeamWarps);
+    mbar_init(smem_u32(flush_bar), C::kEpiWarps);
     mbar_init(smem_u32(ticket_bar), 1);
     misc[3] = 0;
     mbar_init(smem_u32(epi_sync), C::kEpiWarps);
@@ -303,7 +320,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     // itself); it probes for the published share once per unit, having run
     // far enough ahead that the ticket's latency costs the pipeline nothing,
     // and leaves any reduction to the epilogue's many threads.
-    const long long t_head = u_begin / ku;
+    const long long t_head = static_cast<uint32_t>(u_begin) / static_cast<uint32_t>(ku);
     const long long head_end = (u_end < (t_head + 1) * ku) ? u_end : (t_head + 1) * ku;
     bool head_pending = (u_begin < u_end) && head_end < u_end && u_begin != t_head * ku;
     // W4A16: the weights may come from the preceding grid.  W4A4 always runs
@@ -381,21 +398,24 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     const int parity = warp - 2;
     int i = parity;
     bool ok = true;
-    for (long long u = u_begin + parity; u < u_end && ok; u += 2, i += 2) {
-      int j = i * gpu;
-      const int sa = i % NA;
-      const int sx = i % NX;
-      ok = warp_wait(smem_u32(&a_full[sa]), (i / NA) & 1, abort_flag, args.status);
-      ok = ok && warp_wait(smem_u32(&x_full[sx]), (i / NX) & 1, abort_flag, args.status);
+    RingPos ra, rx, racc;
+    ra.init(parity, NA);
+    rx.init(parity, NX);
+    for (long long u = u_begin + parity; u < u_end && ok;
+         u += 2, i += 2, ra.step(2, NA), rx.step(2, NX)) {
+      const int sa = ra.slot;
+      const int sx = rx.slot;
+      racc.init(i * gpu, NACC);
+      ok = warp_wait(smem_u32(&a_full[sa]), ra.phase, abort_flag, args.status);
+      ok = ok && warp_wait(smem_u32(&x_full[sx]), rx.phase, abort_flag, args.status);
       if (!ok) break;
       QSPEC_STAMP(3, i);
       tc_fence_after();
       const uint32_t a_col = tmem_base + static_cast<uint32_t>(sa * C::kACols);
       const uint32_t b_base = smem_u32(x_buf + sx * C::kXBytes);
-      for (int h = 0; h < gpu; ++h, ++j) {
-        const int b = j % NACC;
-        const uint32_t pha = (j / NACC) & 1;
-        ok = warp_wait(smem_u32(&acc_empty[b]), pha ^ 1, abort_flag, args.status);
+      for (int h = 0; h < gpu; ++h, racc.step(1, NACC)) {
+        const int b = racc.slot;
+        ok = warp_wait(smem_u32(&acc_empty[b]), racc.phase ^ 1u, abort_flag, args.status);
         if (!ok) break;
         tc_fence_after();
         // One elected lane issues the group's MMAs and its commit back to back.
@@ -440,11 +460,15 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     const uint32_t swz = static_cast<uint32_t>((r >> 1) & 3);
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     int i = cteam;
-    for (long long u = u_begin + cteam; u < u_end; u += kConvTeams, i += kConvTeams) {
-      const int sp = i % NPK;
-      const int sa = i % NA;
-      bool ok = warp_wait(smem_u32(&pk_full[sp]), (i / NPK) & 1, abort_flag, args.status);
-      ok = ok && warp_wait(smem_u32(&a_empty[sa]), ((i / NA) & 1) ^ 1, abort_flag, args.status);
+    RingPos rp, ra;
+    rp.init(cteam, NPK);
+    ra.init(cteam, NA);
+    for (long long u = u_begin + cteam; u < u_end;
+         u += kConvTeams, i += kConvTeams, rp.step(kConvTeams, NPK), ra.step(kConvTeams, NA)) {
+      const int sp = rp.slot;
+      const int sa = ra.slot;
+      bool ok = warp_wait(smem_u32(&pk_full[sp]), rp.phase, abort_flag, args.status);
+      ok = ok && warp_wait(smem_u32(&a_empty[sa]), ra.phase ^ 1u, abort_flag, args.status);
       if (!ok) break;
       if (i == 0 && r == 0) QSPEC_PHASE(2);
       if (quad == 0) QSPEC_STAMP(cteam == 0 ? 1 : 9, i);
@@ -510,12 +534,11 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     // ------------------------------------------------ epilogue
     const int ew = warp - (kCtlWarps + kConvWarps);
     const int quad = warp & 3;                 // tensor-memory lanes this warp may read
-    const int team = (ew >> 2) % C::kTeams;    // column team
-    const int gteam = (ew >> 2) / C::kTeams;   // group team: groups j with j % kTeamsG == gteam
-    const bool writer = (gteam == 0);          // group team 0 writes the tile results
+    const int team = ew >> 2;                  // column team
     const int col0 = team * C::kCols;
     const int row = quad * 32 + lane;
     const int et = ew * 32 + lane;             // 0 .. kEpiThreads-1
+    const int G = args.groups_per_row;
     grid_dependency_wait();   // no global write before the preceding grid is done
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
 
@@ -524,44 +547,44 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     // slot with cp.async (nothing waits on a register) and reads group j's
     // scale once that copy has landed: the load latency hides behind
     // kScaleAhead groups of work.  A word that would end past the last
-    // scale is copied as its first half only.
+    // scale is copied as its first half only.  The groups of a tile are
+    // consecutive in a row, so the cursor only steps an index and counts
+    // down the groups left in its tile.
     const int groups_total = static_cast<int>(u_end - u_begin) * gpu;
-    const long long ws_elems = static_cast<long long>(args.N) * args.groups_per_row;
+    const long long ws_elems = static_cast<long long>(args.N) * G;
     const uint32_t slot0 = smem_u32(scale_ring + et);
     constexpr uint32_t kSlotStride = C::kEpiThreads * 4;
-    UnitCursor pf;
-    pf.init(u_begin, ku, args.m_tiles);
-    int pf_h = 0, pf_j = 0, pf_slot = 0;
-    // scale index of the prefetch cursor's group; groups of a tile are consecutive
-    bool pf_row_ok = pf.n_tile * kTileN + row < args.N;
-    long long pf_idx = static_cast<long long>(pf.n_tile * kTileN + row) * args.groups_per_row +
-                       static_cast<long long>(pf.kc) * gpu;
-    auto pf_advance = [&]() {
-      ++pf_j;
-      ++pf_idx;
-      if (++pf_h == gpu) {
-        pf_h = 0;
-        if (__builtin_expect(++pf.kc == ku, 0)) {   // next tile: scales restart at group 0
-          pf.kc = 0;
-          if (++pf.m_tile == args.m_tiles) {
-            pf.m_tile = 0;
-            ++pf.n_tile;
-          }
-          const int nn = pf.n_tile * kTileN + row;
-          pf_row_ok = nn < args.N;
-          pf_idx = static_cast<long long>(nn) * args.groups_per_row;
-        }
-      }
-    };
-    // copy the scale of this team's next group
+    int pf_j = 0, pf_slot = 0, pf_m_tile, pf_n_tile, pf_left;
+    long long pf_idx;
+    bool pf_row_ok;
+    {
+      UnitCursor pc;
+      pc.init(u_begin, ku, args.m_tiles);
+      pf_m_tile = pc.m_tile;
+      pf_n_tile = pc.n_tile;
+      pf_left = (ku - pc.kc) * gpu;
+      const int nn = pf_n_tile * kTileN + row;
+      pf_row_ok = nn < args.N;
+      pf_idx = static_cast<long long>(nn) * G + static_cast<long long>(pc.kc) * gpu;
+    }
     auto issue_scale = [&]() {
-      while (pf_j < groups_total && (pf_j % C::kTeamsG) != gteam) pf_advance();
       if (pf_j < groups_total) {
         if (pf_row_ok) {
           const long long w0 = pf_idx & ~1ll;
           cp_async_4(slot0 + pf_slot * kSlotStride, args.ws + w0, (w0 + 1 < ws_elems) ? 4u : 2u);
         }
-        pf_advance();
+        ++pf_j;
+        ++pf_idx;
+        if (__builtin_expect(--pf_left == 0, 0)) {   // next tile: its row's group 0
+          if (++pf_m_tile == args.m_tiles) {
+            pf_m_tile = 0;
+            ++pf_n_tile;
+          }
+          const int nn = pf_n_tile * kTileN + row;
+          pf_row_ok = nn < args.N;
+          pf_idx = static_cast<long long>(nn) * G;
+          pf_left = ku * gpu;
+        }
       }
       if (++pf_slot == C::kScaleSlots) pf_slot = 0;
       cp_async_commit();   // one group per scale, possibly empty, keeps the count uniform
@@ -603,16 +626,18 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
         for (int c = 0; c < C::kCols; ++c) run[c] += __ldcg(src + (col0 + c) * kTileN + row);
       }
       if (et == 0) args.counters[c_lo] = 0u;   // ready for the next launch
-      const int n_tile = static_cast<int>(t / args.m_tiles);
-      const int m_tile = static_cast<int>(t - static_cast<long long>(n_tile) * args.m_tiles);
-      write_y(n_tile * kTileN + row, m_tile * MT + col0);
+      const uint32_t n_tile = static_cast<uint32_t>(t) / static_cast<uint32_t>(args.m_tiles);
+      const uint32_t m_tile = static_cast<uint32_t>(t) - n_tile * static_cast<uint32_t>(args.m_tiles);
+      write_y(static_cast<int>(n_tile) * kTileN + row, static_cast<int>(m_tile) * MT + col0);
     };
-    const long long t_head = u_begin / ku;
+    const long long t_head = static_cast<uint32_t>(u_begin) / static_cast<uint32_t>(ku);
     const long long head_end = (u_end < (t_head + 1) * ku) ? u_end : (t_head + 1) * ku;
     const bool head_handoff = (u_begin < u_end) && head_end < u_end && u_begin != t_head * ku;
     long long to_reduce[2];
     int n_reduce = 0;
-    int j = 0, rd_slot = 0;
+    int rd_slot = 0;
+    RingPos acc;              // accumulator ring position of the next group
+    acc.init(0, NACC);
     bool ok = true;
     volatile int* reducer_flag = reinterpret_cast<volatile int*>(&misc[2]);
     uint32_t epi_phase = 0;
@@ -626,120 +651,94 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       return fine;
     };
     long long u = u_begin;
-    UnitCursor cur;
-    cur.init(u_begin, ku, args.m_tiles);
+    UnitCursor tc;            // the tile of the next segment (no divisions per segment)
+    tc.init(u_begin, ku, args.m_tiles);
     while (u < u_end && ok) {
-      const long long t = static_cast<long long>(cur.n_tile) * args.m_tiles + cur.m_tile;
-      const long long seg_start = u;
+      // one tile segment: units [seg_start, seg_end) of tile t
+      const int n_tile = tc.n_tile, m_tile = tc.m_tile;
+      const long long t = static_cast<long long>(n_tile) * args.m_tiles + m_tile;
       const long long tile_u0 = t * ku;
+      const long long seg_start = u;
       const long long seg_end = (u_end < tile_u0 + ku) ? u_end : tile_u0 + ku;
-      const int n = cur.n_tile * kTileN + row;
-      const int m0 = cur.m_tile * MT + col0;
+      tc.kc = 0;
+      if (++tc.m_tile == args.m_tiles) {
+        tc.m_tile = 0;
+        ++tc.n_tile;
+      }
+      const int n = n_tile * kTileN + row;
+      const int m0 = m_tile * MT + col0;
       // scale (n, g) sits in the upper half of its word when n * G + g is odd
-      const uint32_t row_par = static_cast<uint32_t>(n & args.groups_per_row & 1);
+      const uint32_t row_par = static_cast<uint32_t>(n & G & 1);
 #pragma unroll
       for (int c = 0; c < C::kCols; ++c) run[c] = 0.f;
-      for (; u < seg_end && ok; ++u, cur.next(ku, args.m_tiles)) {
-        const int kc = cur.kc;
-        for (int h = 0; h < gpu; ++h, ++j) {
-          if ((j % C::kTeamsG) != gteam) continue;   // the other group team's group
-          const int b = j % NACC;
-          const uint32_t pha = (j / NACC) & 1;
-          const int g = kc * gpu + h;
-          if (ew == 0) QSPEC_STAMP(14, j);
-          cp_async_wait<C::kScaleAhead - 1>();   // this thread's copy for group j has landed
-          uint32_t sw;
-          asm volatile("ld.shared.b32 %0, [%1];" : "=r"(sw) : "r"(slot0 + rd_slot * kSlotStride));
-          if (++rd_slot == C::kScaleSlots) rd_slot = 0;
-          const uint32_t hbits = ((row_par ^ static_cast<uint32_t>(g)) & 1u) ? (sw >> 16) : (sw & 0xFFFFu);
-          const float sc = __half2float(__ushort_as_half(static_cast<unsigned short>(hbits)));
-          if (ew == 0) QSPEC_STAMP(15, j);
-          issue_scale();   // refills the slot read one group ago
-          ok = warp_wait(smem_u32(&acc_full[b]), pha, abort_flag, args.status);
-          if (!ok) break;
-          if (ew == 0) QSPEC_STAMP(5, j);
-          if (ew == C::kTeamWarps) QSPEC_STAMP(11, j);
-          tc_fence_after();
-          const uint32_t taddr = lane_addr + static_cast<uint32_t>(C::kAccCol0 + b * MT + col0);
+      const int seg_groups = static_cast<int>(seg_end - seg_start) * gpu;
+      int g = static_cast<int>(seg_start - tile_u0) * gpu;   // the row's scale group
+      for (int jj = 0; jj < seg_groups; ++jj, ++g) {
+        if (ew == 0) QSPEC_STAMP(14, (static_cast<int>(seg_start - u_begin) * gpu + jj) & 63);
+        cp_async_wait<C::kScaleAhead - 1>();   // this thread's copy for this group has landed
+        uint32_t sw;
+        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(sw) : "r"(slot0 + rd_slot * kSlotStride));
+        if (++rd_slot == C::kScaleSlots) rd_slot = 0;
+        const uint32_t hbits = ((row_par ^ static_cast<uint32_t>(g)) & 1u) ? (sw >> 16) : (sw & 0xFFFFu);
+        const float sc = __half2float(__ushort_as_half(static_cast<unsigned short>(hbits)));
+        issue_scale();   // refills the slot read one group ago
+        ok = warp_wait(smem_u32(&acc_full[acc.slot]), acc.phase, abort_flag, args.status);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t taddr =
+            lane_addr + static_cast<uint32_t>(C::kAccCol0 + acc.slot * MT + col0);
 #pragma unroll
-          for (int c0 = 0; c0 < C::kCols; c0 += 16) {
-            uint32_t v[16];
-            tmem_ld8(taddr + c0, v);
-            if (c0 + 8 < C::kCols) tmem_ld8(taddr + c0 + 8, v + 8);
-            tmem_ld_wait();
-            if (c0 + 16 >= C::kCols) {
-              // all columns of this group are in registers: hand the buffer back
-              tc_fence_before();
-              __syncwarp();
-              if (elect_one_lane()) mbar_arrive(smem_u32(&acc_empty[b]));
-              __syncwarp();
-              if (ew == 0) QSPEC_STAMP(6, j);
-              if (ew == C::kTeamWarps) QSPEC_STAMP(12, j);
-              if (et == 0 && j == 0) QSPEC_PHASE(4);
+        for (int c0 = 0; c0 < C::kCols; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld8(taddr + c0, v);
+          if (c0 + 8 < C::kCols) tmem_ld8(taddr + c0 + 8, v + 8);
+          tmem_ld_wait();
+          if (c0 + 16 >= C::kCols) {
+            // all columns of this group are in registers: hand the buffer back
+            tc_fence_before();
+            __syncwarp();
+            if (elect_one_lane()) mbar_arrive(smem_u32(&acc_empty[acc.slot]));
+            __syncwarp();
+          }
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            if (c0 + e < C::kCols) {
+              const float a = kInt8 ? static_cast<float>(static_cast<int>(v[e])) : __uint_as_float(v[e]);
+              run[c0 + e] = fmaf(sc, a, run[c0 + e]);
             }
+          }
+          if constexpr (kInt8 && kDbg) {
+            if (n < args.N) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              if (c0 + e < C::kCols) {
-                const float a = kInt8 ? static_cast<float>(static_cast<int>(v[e])) : __uint_as_float(v[e]);
-                run[c0 + e] = fmaf(sc, a, run[c0 + e]);
-              }
-            }
-            if constexpr (kInt8 && kDbg) {
-              if (n < args.N) {
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                  const int m = m0 + c0 + e;
-                  if (c0 + e < C::kCols && m < args.M)
-                    args.dbg_acc[(static_cast<long long>(m) * args.N + n) * args.groups_per_row + g] =
-                        static_cast<int>(v[e]) >> 4;   // exact: a multiple of 16
-                }
+              for (int e = 0; e < 16; ++e) {
+                const int m = m0 + c0 + e;
+                if (c0 + e < C::kCols && m < args.M)
+                  args.dbg_acc[(static_cast<long long>(m) * args.N + n) * G + g] =
+                      static_cast<int>(v[e]) >> 4;   // exact: a multiple of 16
               }
             }
           }
-          if (ew == 0) QSPEC_STAMP(8, j);
         }
+        acc.step(1, NACC);
       }
       if (!ok) break;
+      u = seg_end;
       if (et == 0) QSPEC_PHASE(u >= u_end ? 5 : 7);
 
-      if constexpr (C::kTeamsG > 1) {
-        // the other group teams hand their sums to team 0 through shared
-        // memory; team 0 adds them in team order
-        constexpr int kSlot = MT * kTileN;
-        if (!writer) {
-          float* xc = xchg + (gteam - 1) * kSlot + (col0 * kTileN + row);
-#pragma unroll
-          for (int c = 0; c < C::kCols; ++c) xc[c * kTileN] = run[c];
-        }
-        if (!epi_barrier()) break;
-        if (writer) {
-#pragma unroll
-          for (int t2 = 0; t2 < C::kTeamsG - 1; ++t2) {
-            const float* xc = xchg + t2 * kSlot + (col0 * kTileN + row);
-#pragma unroll
-            for (int c = 0; c < C::kCols; ++c) run[c] += xc[c * kTileN];
-          }
-        }
-        if (!epi_barrier()) break;   // the exchange buffer is free again
-      }
       const bool full = (seg_start == tile_u0) && (seg_end == tile_u0 + ku);
       if (full) {
-        if (writer) write_y(n, m0);
+        write_y(n, m0);
       } else {
         const int k = (seg_start == u_begin) ? 0 : 1;
         float* mine = args.partials + static_cast<long long>(2 * cta + k) * MT * kTileN;
-        if (writer) {
 #pragma unroll
-          for (int c = 0; c < C::kCols; ++c) mine[(col0 + c) * kTileN + row] = run[c];
-        }
+        for (int c = 0; c < C::kCols; ++c) mine[(col0 + c) * kTileN + row] = run[c];
         if (seg_end < u_end) {
           // The CTA's first tile with more to follow: publish the share and go
           // on; the weight producer takes the ticket.
-          if (writer) {
-            __syncwarp();
-            if (elect_one_lane()) mbar_arrive(smem_u32(flush_bar));
-            __syncwarp();
-          }
+          __syncwarp();
+          if (elect_one_lane()) mbar_arrive(smem_u32(flush_bar));
+          __syncwarp();
         } else {
           // The CTA's last tile: take the ticket here.
           if (!epi_barrier()) break;
@@ -755,7 +754,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       ok = warp_wait(smem_u32(ticket_bar), 0, abort_flag, args.status);
       if (ok && misc[3] != 0u) to_reduce[n_reduce++] = t_head;
     }
-    for (int r = 0; ok && writer && r < n_reduce; ++r) reduce_tile(to_reduce[r]);
+    for (int r = 0; ok && r < n_reduce; ++r) reduce_tile(to_reduce[r]);
     cp_async_wait<0>();
   }
 

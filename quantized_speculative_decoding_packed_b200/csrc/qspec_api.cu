@@ -116,7 +116,10 @@ bool gemm_shape_ok(int64_t m, int64_t n, int64_t k, int32_t group) {
   if (m < 1 || n < 1 || k < 128 || (k % 128) != 0) return false;
   if (group != 64 && group != 128) return false;
   if (m > (1ll << 30) || n > (1ll << 30) || k > (1ll << 30)) return false;
-  return true;
+  // the kernel's 32-bit unit arithmetic
+  const long long mt = pick_mt(m);
+  const long long units = ((m + mt - 1) / mt) * ((n + kTileN - 1) / kTileN) * (k / kUnitK);
+  return units < kMaxUnits;
 }
 
 GemmPlan plan_gemm(bool int8_mode, int64_t m, int64_t n, int64_t k, int sm_count) {
