@@ -161,9 +161,10 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 // Waits for the phase with the given parity to complete.  Returns false (and
 // raises the CTA-wide abort flag and the device status word) if the wait
 // runs past kWaitLimitNs or another thread of the CTA has already aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* status) {
-  if (mbar_try_wait(bar, parity)) return true;
+// The slow path lives out of line: the hot loops keep one try_wait and a
+// branch, and their code stays compact in the instruction caches.
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                            uint32_t* status) {
   const uint64_t start = global_timer_ns();
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;   // sleeps <= 0.2 ms
@@ -174,6 +175,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          uint32_t* status) {
+  if (__builtin_expect(mbar_try_wait(bar, parity), 1)) return true;
+  return mbar_wait_slow(bar, parity, abort_flag, status);
 }
 
 // Warp-level wait: every lane polls (one warp-wide instruction per poll, no

@@ -55,8 +55,9 @@
 namespace qspec {
 
 constexpr int kTileN = 128;                      // weight rows per tile (MMA M)
-constexpr int kUnitK = 128;                      // input channels per unit
-constexpr int kPkBytes = kTileN * kUnitK / 2;    // packed bytes per unit
+// Input channels per unit: 256 in int8 mode (16 KB of packed weights per
+// hand-off), 128 in bf16 mode (whose activation tiles are 4x larger).
+__host__ __device__ constexpr int unit_k(bool int8_mode) { return int8_mode ? 256 : 128; }
 constexpr int kConvWarps = 8;                    // two teams of four (one per lane quadrant)
 constexpr int kConvTeams = 2;                    // the teams take alternate units
 constexpr int kConvTeamWarps = kConvWarps / kConvTeams;
@@ -76,6 +77,8 @@ __host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
 template <bool kInt8, int MT>
 struct GemmCfg {
   static_assert(MT % 16 == 0 && MT >= 16 && MT <= 128, "token tile must be 16..128, step 16");
+  static constexpr int kUnitK = unit_k(kInt8);
+  static constexpr int kPkBytes = kTileN * kUnitK / 2;           // packed bytes per unit
   static constexpr int kElem = kInt8 ? 1 : 2;                    // bytes per widened element
   static constexpr int kAtoms = kUnitK * kElem / 128;            // 128-byte K atoms per row
   static constexpr int kXBytes = MT * 128 * kAtoms;              // activation tile
@@ -83,7 +86,7 @@ struct GemmCfg {
   // columns along K): 32 columns of int8 or 64 of bf16 per unit, then the
   // per-group accumulators (MT columns each) in what is left.
   static constexpr int kACols = kUnitK * kElem / 4;
-  static constexpr int kNumA = (kInt8 && MT <= 32) ? kMaxA : 4;
+  static constexpr int kNumA = kInt8 ? (MT <= 32 ? 6 : (MT <= 64 ? 4 : 2)) : 4;
   static constexpr int kAccCol0 = kNumA * kACols;
   static constexpr int kNumAcc = cmin(kMaxAcc, (kTmemCols - kAccCol0) / MT);
   static_assert(kNumAcc >= 2, "tensor memory too small for two accumulators");
@@ -104,9 +107,9 @@ struct GemmCfg {
   // Ring depths from the shared-memory budget: packed weights first (they
   // cover HBM latency), activations (an L2 hit) with what is left.
   static constexpr int kAvail = kSmemLimit - 1024 - kBarBytes - kScaleBytes;
-  static constexpr int kNumX = cmin(kMaxX, cmax(3, (kAvail - 16 * kPkBytes) / kXBytes));
+  static constexpr int kNumX = cmin(kMaxX, cmax(3, (kAvail - 128 * 1024) / kXBytes));
   static constexpr int kNumPk = cmin(kMaxPk, (kAvail - kNumX * kXBytes) / kPkBytes);
-  static_assert(kNumX >= 3 && kNumPk >= 8, "shared memory too small for the rings");
+  static_assert(kNumX >= 3 && kNumPk >= 6, "shared memory too small for the rings");
   static constexpr int kSmemBytes =
       1024 + kNumPk * kPkBytes + kNumX * kXBytes + kScaleBytes + kBarBytes;
   static_assert(kSmemBytes <= kSmemLimit, "shared memory overflow");
@@ -237,7 +240,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* pk_buf = smem;
-  uint8_t* x_buf = pk_buf + NPK * kPkBytes;
+  uint8_t* x_buf = pk_buf + NPK * C::kPkBytes;
   uint32_t* scale_ring = reinterpret_cast<uint32_t*>(x_buf + NX * C::kXBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(scale_ring + C::kScaleSlots * C::kEpiThreads);
   uint64_t* pk_full = bars;
@@ -336,9 +339,9 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       QSPEC_STAMP(13, i);
       if (!warp_wait(smem_u32(&pk_empty[s]), ph ^ 1, abort_flag, args.status)) break;
       if (elect_one_lane()) {
-        mbar_arrive_expect_tx(smem_u32(&pk_full[s]), kPkBytes);
-        tma_load_2d(smem_u32(pk_buf + s * kPkBytes), &tmap_w, smem_u32(&pk_full[s]),
-                    cur.kc * (kUnitK / 2), cur.n_tile * kTileN);
+        mbar_arrive_expect_tx(smem_u32(&pk_full[s]), C::kPkBytes);
+        tma_load_2d(smem_u32(pk_buf + s * C::kPkBytes), &tmap_w, smem_u32(&pk_full[s]),
+                    cur.kc * (C::kUnitK / 2), cur.n_tile * kTileN);
       }
       __syncwarp();
       QSPEC_STAMP(0, i);
@@ -377,7 +380,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
 #pragma unroll
         for (int a = 0; a < C::kAtoms; ++a) {
           tma_load_2d(smem_u32(x_buf + s * C::kXBytes + a * MT * 128), &tmap_x,
-                      smem_u32(&x_full[s]), cur.kc * kUnitK + a * (128 / C::kElem),
+                      smem_u32(&x_full[s]), cur.kc * C::kUnitK + a * (128 / C::kElem),
                       cur.m_tile * MT);
         }
       }
@@ -451,13 +454,16 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     // ------------------------------------------------ converters
     // Two teams of four warps (one per tensor-memory lane quadrant) take
     // alternate units.  Thread = weight row = tensor-memory lane: it reads the
-    // row's 64 packed bytes (the TMA's 64-byte swizzle puts 16-byte chunk c of
-    // row r at c ^ ((r >> 1) & 3), so a quarter warp hits eight distinct bank
-    // groups), widens them in registers and stores them to its own lane.
+    // row's packed bytes (int8 mode: 128 B, the TMA's 128-byte swizzle puts
+    // 16-byte chunk c of row r at c ^ (r & 7); bf16 mode: 64 B, the 64-byte
+    // swizzle puts it at c ^ ((r >> 1) & 3); either way a quarter warp hits
+    // eight distinct bank groups), widens them in registers and stores them
+    // to its own lane.
+    constexpr int kChunks = C::kUnitK / 32;    // 16-byte packed chunks per row
     const int cteam = (warp - kCtlWarps) / kConvTeamWarps;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
-    const uint32_t swz = static_cast<uint32_t>((r >> 1) & 3);
+    const uint32_t swz = static_cast<uint32_t>(kInt8 ? (r & 7) : ((r >> 1) & 3));
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     int i = cteam;
     RingPos rp, ra;
@@ -472,10 +478,10 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       if (!ok) break;
       if (i == 0 && r == 0) QSPEC_PHASE(2);
       if (quad == 0) QSPEC_STAMP(cteam == 0 ? 1 : 9, i);
-      const uint8_t* rowp = pk_buf + sp * kPkBytes + r * (kUnitK / 2);
-      uint4 v[4];
+      const uint8_t* rowp = pk_buf + sp * C::kPkBytes + r * (C::kUnitK / 2);
+      uint4 v[kChunks];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < kChunks; ++c)
         v[c] = *reinterpret_cast<const uint4*>(rowp + ((static_cast<uint32_t>(c) ^ swz) << 4));
       // The packed slot may be refilled (by the async proxy) once every
       // lane's reads are done.
@@ -491,18 +497,22 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
         // sums; the epilogue divides by 16 exactly.  Each 8 channels land in
         // the order (0,2,4,6,1,3,5,7), the order in which the activation
         // quantizer stores them for this GEMM.
-        uint32_t o[32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t wv[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+        for (int half = 0; half < kChunks / 4; ++half) {   // 128 channels = 32 columns
+          uint32_t o[32];
 #pragma unroll
-          for (int wi = 0; wi < 4; ++wi) {
-            o[8 * c + 2 * wi] = (wv[wi] << 4) & 0xF0F0F0F0u;   // 16 q of k0 k2 k4 k6
-            o[8 * c + 2 * wi + 1] = wv[wi] & 0xF0F0F0F0u;      // 16 q of k1 k3 k5 k7
+          for (int c = 0; c < 4; ++c) {
+            const uint4 vc = v[4 * half + c];
+            const uint32_t wv[4] = {vc.x, vc.y, vc.z, vc.w};
+#pragma unroll
+            for (int wi = 0; wi < 4; ++wi) {
+              o[8 * c + 2 * wi] = (wv[wi] << 4) & 0xF0F0F0F0u;   // 16 q of k0 k2 k4 k6
+              o[8 * c + 2 * wi + 1] = wv[wi] & 0xF0F0F0F0u;      // 16 q of k1 k3 k5 k7
+            }
           }
+          tmem_st16(a_col + 32 * half, o);
+          tmem_st16(a_col + 32 * half + 16, o + 16);
         }
-        tmem_st16(a_col, o);
-        tmem_st16(a_col + 16, o + 16);
       } else {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -554,7 +564,10 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     const long long ws_elems = static_cast<long long>(args.N) * G;
     const uint32_t slot0 = smem_u32(scale_ring + et);
     constexpr uint32_t kSlotStride = C::kEpiThreads * 4;
-    int pf_j = 0, pf_slot = 0, pf_m_tile, pf_n_tile, pf_left;
+    // When K is not a multiple of the unit, the last unit of each tile ends in
+    // groups g >= G that do not exist: their weights and activations arrive
+    // zero-filled, so their accumulators are zero; they get scale 0 and no copy.
+    int pf_j = 0, pf_slot = 0, pf_m_tile, pf_n_tile, pf_left, pf_g;
     long long pf_idx;
     bool pf_row_ok;
     {
@@ -563,18 +576,20 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       pf_m_tile = pc.m_tile;
       pf_n_tile = pc.n_tile;
       pf_left = (ku - pc.kc) * gpu;
+      pf_g = pc.kc * gpu;
       const int nn = pf_n_tile * kTileN + row;
       pf_row_ok = nn < args.N;
       pf_idx = static_cast<long long>(nn) * G + static_cast<long long>(pc.kc) * gpu;
     }
     auto issue_scale = [&]() {
       if (pf_j < groups_total) {
-        if (pf_row_ok) {
+        if (pf_row_ok && pf_g < G) {
           const long long w0 = pf_idx & ~1ll;
           cp_async_4(slot0 + pf_slot * kSlotStride, args.ws + w0, (w0 + 1 < ws_elems) ? 4u : 2u);
         }
         ++pf_j;
         ++pf_idx;
+        ++pf_g;
         if (__builtin_expect(--pf_left == 0, 0)) {   // next tile: its row's group 0
           if (++pf_m_tile == args.m_tiles) {
             pf_m_tile = 0;
@@ -584,6 +599,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
           pf_row_ok = nn < args.N;
           pf_idx = static_cast<long long>(nn) * G;
           pf_left = ku * gpu;
+          pf_g = 0;
         }
       }
       if (++pf_slot == C::kScaleSlots) pf_slot = 0;
@@ -680,7 +696,8 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
         asm volatile("ld.shared.b32 %0, [%1];" : "=r"(sw) : "r"(slot0 + rd_slot * kSlotStride));
         if (++rd_slot == C::kScaleSlots) rd_slot = 0;
         const uint32_t hbits = ((row_par ^ static_cast<uint32_t>(g)) & 1u) ? (sw >> 16) : (sw & 0xFFFFu);
-        const float sc = __half2float(__ushort_as_half(static_cast<unsigned short>(hbits)));
+        const float sc =
+            (g < G) ? __half2float(__ushort_as_half(static_cast<unsigned short>(hbits))) : 0.f;
         issue_scale();   // refills the slot read one group ago
         ok = warp_wait(smem_u32(&acc_full[acc.slot]), acc.phase, abort_flag, args.status);
         if (!ok) break;
@@ -708,7 +725,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
             }
           }
           if constexpr (kInt8 && kDbg) {
-            if (n < args.N) {
+            if (n < args.N && g < G) {
 #pragma unroll
               for (int e = 0; e < 16; ++e) {
                 const int m = m0 + c0 + e;

@@ -118,7 +118,7 @@ bool gemm_shape_ok(int64_t m, int64_t n, int64_t k, int32_t group) {
   if (m > (1ll << 30) || n > (1ll << 30) || k > (1ll << 30)) return false;
   // the kernel's 32-bit unit arithmetic
   const long long mt = pick_mt(m);
-  const long long units = ((m + mt - 1) / mt) * ((n + kTileN - 1) / kTileN) * (k / kUnitK);
+  const long long units = ((m + mt - 1) / mt) * ((n + kTileN - 1) / kTileN) * (k / unit_k(false));
   return units < kMaxUnits;
 }
 
@@ -127,7 +127,8 @@ GemmPlan plan_gemm(bool int8_mode, int64_t m, int64_t n, int64_t k, int sm_count
   p.mt = pick_mt(m);
   p.m_tiles = static_cast<int>((m + p.mt - 1) / p.mt);
   p.n_tiles = static_cast<int>((n + kTileN - 1) / kTileN);
-  p.ku = static_cast<int>(k / kUnitK);
+  const int uk = unit_k(int8_mode);
+  p.ku = static_cast<int>((k + uk - 1) / uk);   // a last half unit reads zeros past k
   p.units = static_cast<long long>(p.m_tiles) * p.n_tiles * p.ku;
   const int max_grid = sm_count < kMaxGrid ? sm_count : kMaxGrid;
   p.grid = static_cast<int>(p.units < max_grid ? p.units : max_grid);
@@ -232,16 +233,18 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
   uint8_t* wsp = static_cast<uint8_t*>(workspace);
 
   CUtensorMap tw, tx;
-  // 64-byte swizzle: the converter threads read one 64-byte row each
-  if (!make_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wq, n, k / 2, kTileN, kUnitK / 2,
-                 CU_TENSOR_MAP_SWIZZLE_64B))
+  // Each converter thread reads one row of the packed tile: 128 B in int8
+  // mode (128-byte swizzle), 64 B in bf16 mode (64-byte swizzle).
+  const int uk = unit_k(kInt8);
+  if (!make_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wq, n, k / 2, kTileN, uk / 2,
+                 kInt8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
     return QSPEC_ERR_CUDA;
   GemmArgs a;
   a.M = static_cast<int>(m);
   a.N = static_cast<int>(n);
   a.K = static_cast<int>(k);
   a.groups_per_row = static_cast<int>(k / group);
-  a.groups_per_unit = kUnitK / group;
+  a.groups_per_unit = uk / group;
   a.m_tiles = p.m_tiles;
   a.n_tiles = p.n_tiles;
   a.ku = p.ku;
