@@ -53,7 +53,30 @@ def parse():
                     help="decoder layers (32 = the full model; smaller only for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--profile-gemm", metavar="MODE:SHAPE", default=None,
+                    help="profiling driver: three calls of one GEMM (MODE w4a4|w4a16, SHAPE "
+                         "qkv|o_proj|gate_up|down of the workload) on seeded weights, then exit")
     return ap.parse_args()
+
+
+def profile_gemm(spec):
+    """Three calls of one GEMM of the workload, for a profiler to capture one of them."""
+    import torch
+    from quantized_speculative_decoding_packed_b200 import qspec
+    mode, shape = spec.split(":")
+    n, k = {name: (n, k) for name, n, k in LAYERS}[shape]
+    m = M_DRAFT if mode == "w4a4" else M_VERIFY
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(rank_seed(0))
+    w = torch.randn((n, k), generator=gen, device="cuda", dtype=torch.float32) * 0.02
+    wq, ws = qspec.quantize_weights(w, GROUP)
+    del w
+    x = torch.randn((m, k), generator=gen, device="cuda").to(torch.bfloat16)
+    fn = qspec.gemm_w4a4 if mode == "w4a4" else qspec.gemm_w4a16
+    for _ in range(3):
+        y = fn(x, wq, ws, GROUP)
+    torch.cuda.synchronize()
+    print(f"{mode} {shape}: y[{m}][{n}] sum |y| = {float(y.abs().sum()):.6g}")
 
 
 # ---------------------------------------------------------------- algorithmic bytes / ops
@@ -242,6 +265,9 @@ def workload_config(layers):
 # ---------------------------------------------------------------- GPU arm
 def main():
     args = parse()
+    if args.profile_gemm:
+        profile_gemm(args.profile_gemm)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
