@@ -91,16 +91,31 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
       !QSPEC_ALIGN_OK(reinterpret_cast<uintptr_t>(out), 8))
     return;
 
-  float a = 0.f;
-  for (int64_t c = static_cast<int64_t>(tid) * 8; c < k; c += 256 * 8) {
-    const uint4 u = *reinterpret_cast<const uint4*>(xr + c);
+  // Each thread's chunks of 8 elements stay in registers between the two
+  // passes (up to kCache chunks: rows of up to 16384 elements are read once);
+  // longer rows read the rest again.
+  constexpr int kCache = 8;
+  uint4 cache[kCache];
+  auto absmax8 = [](const uint4& u, float m) {
     const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      a = fmaxf(a, fabsf(bf16_bits_to_float(w4[j] & 0xFFFFu)));
-      a = fmaxf(a, fabsf(bf16_bits_to_float(w4[j] >> 16)));
+      m = fmaxf(m, fabsf(bf16_bits_to_float(w4[j] & 0xFFFFu)));
+      m = fmaxf(m, fabsf(bf16_bits_to_float(w4[j] >> 16)));
+    }
+    return m;
+  };
+  float a = 0.f;
+#pragma unroll
+  for (int j = 0; j < kCache; ++j) {
+    const int64_t c = (static_cast<int64_t>(tid) + 256 * j) * 8;
+    if (c < k) {
+      cache[j] = *reinterpret_cast<const uint4*>(xr + c);
+      a = absmax8(cache[j], a);
     }
   }
+  for (int64_t c = (static_cast<int64_t>(tid) + 256 * kCache) * 8; c < k; c += 256 * 8)
+    a = absmax8(*reinterpret_cast<const uint4*>(xr + c), a);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
   if ((tid & 31) == 0) red[tid >> 5] = a;
@@ -113,8 +128,7 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
   const float inv = __fdiv_rn(7.0f, a);
   if (tid == 0) scales[row] = s;
 
-  for (int64_t c = static_cast<int64_t>(tid) * 8; c < k; c += 256 * 8) {
-    const uint4 u = *reinterpret_cast<const uint4*>(xr + c);
+  auto emit = [&](int64_t c, const uint4& u) {
     const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
     int q[8];
 #pragma unroll
@@ -142,7 +156,14 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
       }
       *reinterpret_cast<uint2*>(static_cast<int8_t*>(out) + row * k + c) = make_uint2(ev, od);
     }
+  };
+#pragma unroll
+  for (int j = 0; j < kCache; ++j) {
+    const int64_t c = (static_cast<int64_t>(tid) + 256 * j) * 8;
+    if (c < k) emit(c, cache[j]);
   }
+  for (int64_t c = (static_cast<int64_t>(tid) + 256 * kCache) * 8; c < k; c += 256 * 8)
+    emit(c, *reinterpret_cast<const uint4*>(xr + c));
 }
 
 }  // namespace qspec
