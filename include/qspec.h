@@ -70,7 +70,10 @@ enum {
  *  w   [n][k] fp32, row-major.
  *  wq  [n][k/2] bytes out: byte j of a row holds k = 2j in its low nibble and
  *      k = 2j+1 in its high nibble, two's complement.
- *  ws  [n][k/group] fp16 bit patterns out.
+ *  ws  [n][ldg] fp16 bit patterns out, ldg = k/group rounded up to a multiple
+ *      of 8 (rows start on 16-byte boundaries, so the GEMMs fetch scale tiles
+ *      with TMA); entry [n][g] is s_h of group g for g < k/group, the padding
+ *      entries are written as zero.  16-byte aligned.
  * Requires n >= 1, group in {64, 128}, k a multiple of group.
  */
 qspec_status qspec_quantize_weights(const float* w, int64_t n, int64_t k, int32_t group,
@@ -96,8 +99,8 @@ qspec_status qspec_quant_act(const uint16_t* x, int64_t m, int64_t k, uint8_t* x
  * is computed exactly on the int8 tensor cores (int32), and
  *   y[m][n] = s_a[m] * sum_g s_h[n][g] * acc[m][n][g]   (fp32 arithmetic).
  *  x        [m][k] bf16.
- *  wq, ws   as produced by qspec_quantize_weights for [n][k] weights; wq
- *           16-byte aligned, ws 4-byte aligned (scales are fetched as words).
+ *  wq, ws   as produced by qspec_quantize_weights for [n][k] weights (ws with
+ *           its padded row stride); both 16-byte aligned.
  *  y        [m][n] fp32 out.
  *  workspace  device scratch of at least
  *           qspec_workspace_size(QSPEC_OP_GEMM_W4A4, m, n, k, group, 0, 0, 0)

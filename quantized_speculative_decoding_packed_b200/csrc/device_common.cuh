@@ -71,6 +71,14 @@ constexpr uint32_t kDevBadInput = 2u;
 // A wait that has not completed after this long is treated as a fault.
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;   // 1 s
 
+// Row stride (in fp16 scales) of the group-scale matrix ws: k/group rounded
+// up to a multiple of 8, so that each row starts on a 16-byte boundary and
+// the GEMM can fetch 8 groups x 128 rows of scales with one TMA copy.  The
+// padding entries hold zeros.
+__host__ __device__ constexpr int64_t scale_row_stride(int64_t groups_per_row) {
+  return (groups_per_row + 7) / 8 * 8;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

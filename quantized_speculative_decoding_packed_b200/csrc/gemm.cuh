@@ -69,6 +69,10 @@ constexpr int kSmemLimit = 232448;               // sm_100 dynamic shared memory
 #endif
 constexpr int kMaxGrid = 1024;                   // ticket slots in the workspace
 constexpr int kMaxPk = 24, kMaxA = 8, kMaxAcc = 8, kMaxX = 8;
+// Group scales arrive by TMA, 8 groups x 128 rows (2 KB) per tile, into a ring.
+constexpr int kScaleTileGroups = 8;
+constexpr int kScaleTileBytes = kTileN * kScaleTileGroups * 2;
+constexpr int kNumSc = 8;
 constexpr int kTmemCols = 512;                   // all of tensor memory: one CTA per SM
 
 __host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
@@ -100,10 +104,7 @@ struct GemmCfg {
   static constexpr int kWarps = kCtlWarps + kConvWarps + kEpiWarps;
   static constexpr int kThreads = 32 * kWarps;
   static constexpr int kBarBytes = 1024;
-  // group scales travel global -> shared by cp.async, kScaleAhead groups ahead
-  static constexpr int kScaleAhead = 4;
-  static constexpr int kScaleSlots = kScaleAhead + 1;
-  static constexpr int kScaleBytes = kScaleSlots * kEpiThreads * 4;
+  static constexpr int kScaleBytes = kNumSc * kScaleTileBytes;
   // Ring depths from the shared-memory budget: packed weights first (they
   // cover HBM latency), activations (an L2 hit) with what is left.
   static constexpr int kAvail = kSmemLimit - 1024 - kBarBytes - kScaleBytes;
@@ -232,7 +233,8 @@ __device__ __forceinline__ bool take_tile_ticket(const GemmArgs& args, long long
 template <bool kInt8, int MT, bool kDbg>
 __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     qgemm_kernel(const __grid_constant__ CUtensorMap tmap_w,
-                 const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ GemmArgs args) {
+                 const __grid_constant__ CUtensorMap tmap_x,
+                 const __grid_constant__ CUtensorMap tmap_s, const __grid_constant__ GemmArgs args) {
   using C = GemmCfg<kInt8, MT>;
   constexpr int NPK = C::kNumPk, NA = C::kNumA, NX = C::kNumX, NACC = C::kNumAcc;
   extern __shared__ uint8_t smem_raw[];
@@ -241,8 +243,8 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* pk_buf = smem;
   uint8_t* x_buf = pk_buf + NPK * C::kPkBytes;
-  uint32_t* scale_ring = reinterpret_cast<uint32_t*>(x_buf + NX * C::kXBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(scale_ring + C::kScaleSlots * C::kEpiThreads);
+  uint8_t* sc_buf = x_buf + NX * C::kXBytes;     // group-scale tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sc_buf + C::kScaleBytes);
   uint64_t* pk_full = bars;
   uint64_t* pk_empty = pk_full + kMaxPk;
   uint64_t* a_full = pk_empty + kMaxPk;    // widened unit in tensor memory
@@ -252,7 +254,9 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   uint64_t* acc_full = x_empty + kMaxX;
   uint64_t* acc_empty = acc_full + kMaxAcc;
   uint64_t* mma_done = acc_empty + kMaxAcc;
-  uint64_t* flush_bar = mma_done + 1;   // the head split tile's share is published
+  uint64_t* sc_full = mma_done + 1;     // [kNumSc]: a scale tile has landed
+  uint64_t* sc_empty = sc_full + kNumSc; // [kNumSc]: the epilogue is done with it
+  uint64_t* flush_bar = sc_empty + kNumSc;   // the head split tile's share is published
   uint64_t* ticket_bar = flush_bar + 1; // ... and its ticket taken (result in misc[3])
   uint64_t* epi_sync = ticket_bar + 1;
   uint32_t* misc = reinterpret_cast<uint32_t*>(epi_sync + 1);
@@ -289,6 +293,10 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       mbar_init(smem_u32(&acc_empty[b]), C::kEpiWarps);
     }
     mbar_init(smem_u32(mma_done), 2);
+    for (int s = 0; s < kNumSc; ++s) {
+      mbar_init(smem_u32(&sc_full[s]), 1);
+      mbar_init(smem_u32(&sc_empty[s]), C::kEpiWarps);
+    }
     mbar_init(smem_u32(flush_bar), C::kEpiWarps);
     mbar_init(smem_u32(ticket_bar), 1);
     misc[3] = 0;
@@ -300,6 +308,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmap_w);
     prefetch_tensormap(&tmap_x);
+    prefetch_tensormap(&tmap_s);
   }
   if (warp == 2) {
     tmem_alloc(smem_u32(&misc[0]), kTmemCols);
@@ -330,6 +339,12 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     // behind its own activation quantization, which launched this grid only
     // after the grid before it had completed.
     if constexpr (!kInt8) grid_dependency_wait();
+    // Group scales: one TMA tile (8 groups x 128 rows) whenever a unit starts a
+    // new run of 8 groups of its tile, or is this CTA's first unit; the
+    // epilogue walks the same sequence.
+    RingPos rs;
+    rs.init(0, kNumSc);
+    int n_sc = 0;
     int i = 0;
     UnitCursor cur;
     cur.init(u_begin, ku, args.m_tiles);
@@ -345,6 +360,18 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       }
       __syncwarp();
       QSPEC_STAMP(0, i);
+      const int g0 = cur.kc * gpu;
+      if (u == u_begin || (g0 & (kScaleTileGroups - 1)) == 0) {
+        if (!warp_wait(smem_u32(&sc_empty[rs.slot]), rs.phase ^ 1u, abort_flag, args.status)) break;
+        if (elect_one_lane()) {
+          mbar_arrive_expect_tx(smem_u32(&sc_full[rs.slot]), kScaleTileBytes);
+          tma_load_2d(smem_u32(sc_buf + rs.slot * kScaleTileBytes), &tmap_s, smem_u32(&sc_full[rs.slot]),
+                      g0 & ~(kScaleTileGroups - 1), cur.n_tile * kTileN);
+        }
+        __syncwarp();
+        rs.step(1, kNumSc);
+        ++n_sc;
+      }
       if (head_pending && __all_sync(0xffffffffu, mbar_test_wait(smem_u32(flush_bar), 0))) {
         if (lane == 0) {
           misc[3] = take_tile_ticket(args, t_head, units, grid) ? 1u : 0u;
@@ -364,6 +391,8 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     if (*abort_flag) {
       for (int j = (i > NPK ? i - NPK : 0); j < i; ++j)
         mbar_wait_drain(smem_u32(&pk_full[j % NPK]), (j / NPK) & 1);
+      for (int j = (n_sc > kNumSc ? n_sc - kNumSc : 0); j < n_sc; ++j)
+        mbar_wait_drain(smem_u32(&sc_full[j % kNumSc]), (j / kNumSc) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ activation producer
@@ -552,61 +581,14 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     grid_dependency_wait();   // no global write before the preceding grid is done
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
 
-    // Group scales.  Each thread copies the aligned 32-bit word holding its
-    // row's fp16 scale of group j + kScaleAhead into a private shared-memory
-    // slot with cp.async (nothing waits on a register) and reads group j's
-    // scale once that copy has landed: the load latency hides behind
-    // kScaleAhead groups of work.  A word that would end past the last
-    // scale is copied as its first half only.  The groups of a tile are
-    // consecutive in a row, so the cursor only steps an index and counts
-    // down the groups left in its tile.
-    const int groups_total = static_cast<int>(u_end - u_begin) * gpu;
-    const long long ws_elems = static_cast<long long>(args.N) * G;
-    const uint32_t slot0 = smem_u32(scale_ring + et);
-    constexpr uint32_t kSlotStride = C::kEpiThreads * 4;
-    // When K is not a multiple of the unit, the last unit of each tile ends in
-    // groups g >= G that do not exist: their weights and activations arrive
-    // zero-filled, so their accumulators are zero; they get scale 0 and no copy.
-    int pf_j = 0, pf_slot = 0, pf_m_tile, pf_n_tile, pf_left, pf_g;
-    long long pf_idx;
-    bool pf_row_ok;
-    {
-      UnitCursor pc;
-      pc.init(u_begin, ku, args.m_tiles);
-      pf_m_tile = pc.m_tile;
-      pf_n_tile = pc.n_tile;
-      pf_left = (ku - pc.kc) * gpu;
-      pf_g = pc.kc * gpu;
-      const int nn = pf_n_tile * kTileN + row;
-      pf_row_ok = nn < args.N;
-      pf_idx = static_cast<long long>(nn) * G + static_cast<long long>(pc.kc) * gpu;
-    }
-    auto issue_scale = [&]() {
-      if (pf_j < groups_total) {
-        if (pf_row_ok && pf_g < G) {
-          const long long w0 = pf_idx & ~1ll;
-          cp_async_4(slot0 + pf_slot * kSlotStride, args.ws + w0, (w0 + 1 < ws_elems) ? 4u : 2u);
-        }
-        ++pf_j;
-        ++pf_idx;
-        ++pf_g;
-        if (__builtin_expect(--pf_left == 0, 0)) {   // next tile: its row's group 0
-          if (++pf_m_tile == args.m_tiles) {
-            pf_m_tile = 0;
-            ++pf_n_tile;
-          }
-          const int nn = pf_n_tile * kTileN + row;
-          pf_row_ok = nn < args.N;
-          pf_idx = static_cast<long long>(nn) * G;
-          pf_left = ku * gpu;
-          pf_g = 0;
-        }
-      }
-      if (++pf_slot == C::kScaleSlots) pf_slot = 0;
-      cp_async_commit();   // one group per scale, possibly empty, keeps the count uniform
-    };
-#pragma unroll
-    for (int a = 0; a < C::kScaleAhead; ++a) issue_scale();
+    // Group scales come as TMA tiles of 8 groups x 128 rows from the weight
+    // producer, in the order it meets them: a new tile with this CTA's first
+    // group and whenever a group index g of a tile reaches a multiple of 8.
+    // Groups g >= k/group (a half unit at the end of k) read the stored zeros.
+    RingPos rsc;              // next scale tile
+    rsc.init(0, kNumSc);
+    int sc_cur = -1;          // scale tile being read
+    const uint32_t sc_row = smem_u32(sc_buf) + static_cast<uint32_t>(row * kScaleTileGroups * 2);
 
     float run[C::kCols];
     // y rows m0 .. m0+kCols-1 of output column n from run[]
@@ -651,7 +633,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     const bool head_handoff = (u_begin < u_end) && head_end < u_end && u_begin != t_head * ku;
     long long to_reduce[2];
     int n_reduce = 0;
-    int rd_slot = 0;
     RingPos acc;              // accumulator ring position of the next group
     acc.init(0, NACC);
     bool ok = true;
@@ -683,22 +664,29 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       }
       const int n = n_tile * kTileN + row;
       const int m0 = m_tile * MT + col0;
-      // scale (n, g) sits in the upper half of its word when n * G + g is odd
-      const uint32_t row_par = static_cast<uint32_t>(n & G & 1);
 #pragma unroll
       for (int c = 0; c < C::kCols; ++c) run[c] = 0.f;
       const int seg_groups = static_cast<int>(seg_end - seg_start) * gpu;
       int g = static_cast<int>(seg_start - tile_u0) * gpu;   // the row's scale group
       for (int jj = 0; jj < seg_groups; ++jj, ++g) {
         if (ew == 0) QSPEC_STAMP(14, (static_cast<int>(seg_start - u_begin) * gpu + jj) & 63);
-        cp_async_wait<C::kScaleAhead - 1>();   // this thread's copy for this group has landed
-        uint32_t sw;
-        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(sw) : "r"(slot0 + rd_slot * kSlotStride));
-        if (++rd_slot == C::kScaleSlots) rd_slot = 0;
-        const uint32_t hbits = ((row_par ^ static_cast<uint32_t>(g)) & 1u) ? (sw >> 16) : (sw & 0xFFFFu);
-        const float sc =
-            (g < G) ? __half2float(__ushort_as_half(static_cast<unsigned short>(hbits))) : 0.f;
-        issue_scale();   // refills the slot read one group ago
+        if (sc_cur < 0 || (g & (kScaleTileGroups - 1)) == 0) {
+          if (sc_cur >= 0) {   // done with the previous tile
+            __syncwarp();
+            if (elect_one_lane()) mbar_arrive(smem_u32(&sc_empty[sc_cur]));
+            __syncwarp();
+          }
+          ok = warp_wait(smem_u32(&sc_full[rsc.slot]), rsc.phase, abort_flag, args.status);
+          if (!ok) break;
+          sc_cur = rsc.slot;
+          rsc.step(1, kNumSc);
+        }
+        uint16_t hbits;
+        asm volatile("ld.shared.u16 %0, [%1];"
+                     : "=h"(hbits)
+                     : "r"(sc_row + static_cast<uint32_t>(sc_cur * kScaleTileBytes +
+                                                          (g & (kScaleTileGroups - 1)) * 2)));
+        const float sc = __half2float(__ushort_as_half(hbits));
         ok = warp_wait(smem_u32(&acc_full[acc.slot]), acc.phase, abort_flag, args.status);
         if (!ok) break;
         tc_fence_after();
@@ -772,7 +760,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       if (ok && misc[3] != 0u) to_reduce[n_reduce++] = t_head;
     }
     for (int r = 0; ok && r < n_reduce; ++r) reduce_tile(to_reduce[r]);
-    cp_async_wait<0>();
   }
 
   QSPEC_TRACE_AT(0xFFF0);

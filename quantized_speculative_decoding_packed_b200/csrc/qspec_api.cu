@@ -151,7 +151,8 @@ GemmPlan plan_gemm(bool int8_mode, int64_t m, int64_t n, int64_t k, int sm_count
 }
 
 template <bool kInt8, int MT, bool kDbg>
-qspec_status launch_qgemm_t(const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a,
+qspec_status launch_qgemm_t(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ts,
+                            const GemmArgs& a,
                             int grid, int dev, cudaStream_t stream) {
   using C = GemmCfg<kInt8, MT>;
   static bool attr_set[kMaxDevices] = {};
@@ -177,7 +178,7 @@ qspec_status launch_qgemm_t(const CUtensorMap& tw, const CUtensorMap& tx, const 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, qgemm_kernel<kInt8, MT, kDbg>, tw, tx, a) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, qgemm_kernel<kInt8, MT, kDbg>, tw, tx, ts, a) != cudaSuccess) {
     cudaGetLastError();
     return QSPEC_ERR_CUDA;
   }
@@ -185,31 +186,32 @@ qspec_status launch_qgemm_t(const CUtensorMap& tw, const CUtensorMap& tx, const 
 }
 
 template <bool kInt8>
-qspec_status launch_qgemm(int mt, const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a,
+qspec_status launch_qgemm(int mt, const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ts,
+                          const GemmArgs& a,
                           int grid, int dev, cudaStream_t stream) {
   const bool dbg = kInt8 && a.dbg_acc != nullptr;
   switch (mt) {
     case 16:
-      return dbg ? launch_qgemm_t<kInt8, 16, kInt8>(tw, tx, a, grid, dev, stream)
-                 : launch_qgemm_t<kInt8, 16, false>(tw, tx, a, grid, dev, stream);
+      return dbg ? launch_qgemm_t<kInt8, 16, kInt8>(tw, tx, ts, a, grid, dev, stream)
+                 : launch_qgemm_t<kInt8, 16, false>(tw, tx, ts, a, grid, dev, stream);
     case 32:
-      return dbg ? launch_qgemm_t<kInt8, 32, kInt8>(tw, tx, a, grid, dev, stream)
-                 : launch_qgemm_t<kInt8, 32, false>(tw, tx, a, grid, dev, stream);
+      return dbg ? launch_qgemm_t<kInt8, 32, kInt8>(tw, tx, ts, a, grid, dev, stream)
+                 : launch_qgemm_t<kInt8, 32, false>(tw, tx, ts, a, grid, dev, stream);
     case 48:
-      return dbg ? launch_qgemm_t<kInt8, 48, kInt8>(tw, tx, a, grid, dev, stream)
-                 : launch_qgemm_t<kInt8, 48, false>(tw, tx, a, grid, dev, stream);
+      return dbg ? launch_qgemm_t<kInt8, 48, kInt8>(tw, tx, ts, a, grid, dev, stream)
+                 : launch_qgemm_t<kInt8, 48, false>(tw, tx, ts, a, grid, dev, stream);
     case 64:
-      return dbg ? launch_qgemm_t<kInt8, 64, kInt8>(tw, tx, a, grid, dev, stream)
-                 : launch_qgemm_t<kInt8, 64, false>(tw, tx, a, grid, dev, stream);
+      return dbg ? launch_qgemm_t<kInt8, 64, kInt8>(tw, tx, ts, a, grid, dev, stream)
+                 : launch_qgemm_t<kInt8, 64, false>(tw, tx, ts, a, grid, dev, stream);
     case 80:
-      return dbg ? launch_qgemm_t<kInt8, 80, kInt8>(tw, tx, a, grid, dev, stream)
-                 : launch_qgemm_t<kInt8, 80, false>(tw, tx, a, grid, dev, stream);
+      return dbg ? launch_qgemm_t<kInt8, 80, kInt8>(tw, tx, ts, a, grid, dev, stream)
+                 : launch_qgemm_t<kInt8, 80, false>(tw, tx, ts, a, grid, dev, stream);
     case 96:
-      return dbg ? launch_qgemm_t<kInt8, 96, kInt8>(tw, tx, a, grid, dev, stream)
-                 : launch_qgemm_t<kInt8, 96, false>(tw, tx, a, grid, dev, stream);
+      return dbg ? launch_qgemm_t<kInt8, 96, kInt8>(tw, tx, ts, a, grid, dev, stream)
+                 : launch_qgemm_t<kInt8, 96, false>(tw, tx, ts, a, grid, dev, stream);
     case 128:
-      return dbg ? launch_qgemm_t<kInt8, 128, kInt8>(tw, tx, a, grid, dev, stream)
-                 : launch_qgemm_t<kInt8, 128, false>(tw, tx, a, grid, dev, stream);
+      return dbg ? launch_qgemm_t<kInt8, 128, kInt8>(tw, tx, ts, a, grid, dev, stream)
+                 : launch_qgemm_t<kInt8, 128, false>(tw, tx, ts, a, grid, dev, stream);
     default: return QSPEC_ERR_INVALID_ARG;
   }
 }
@@ -220,7 +222,7 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
                       size_t workspace_bytes, int32_t* dbg_acc, void* stream_v) {
   if (!x || !wq || !ws || !y || !workspace) return QSPEC_ERR_INVALID_ARG;
   if (!gemm_shape_ok(m, n, k, group)) return QSPEC_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(wq, 16) || !aligned(ws, 4) || !aligned(y, 4) ||
+  if (!aligned(x, 16) || !aligned(wq, 16) || !aligned(ws, 16) || !aligned(y, 4) ||
       !aligned(workspace, 16) || (dbg_acc && !aligned(dbg_acc, 4)))
     return QSPEC_ERR_INVALID_ARG;
   int dev = 0;
@@ -232,7 +234,7 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
   cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
   uint8_t* wsp = static_cast<uint8_t*>(workspace);
 
-  CUtensorMap tw, tx;
+  CUtensorMap tw, tx, ts;
   // Each converter thread reads one row of the packed tile: 128 B in int8
   // mode (128-byte swizzle), 64 B in bf16 mode (64-byte swizzle).
   const int uk = unit_k(kInt8);
@@ -284,7 +286,12 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
                    CU_TENSOR_MAP_SWIZZLE_128B))
       return QSPEC_ERR_CUDA;
   }
-  return launch_qgemm<kInt8>(p.mt, tw, tx, a, p.grid, dev, stream);
+  // group scales: [n][ldg] fp16, one box = 8 groups x 128 rows (zero-filled
+  // past row n-1; groups k/group .. ldg-1 are stored zeros)
+  if (!make_tmap(&ts, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, ws, n, scale_row_stride(k / group), kTileN, 8,
+                 CU_TENSOR_MAP_SWIZZLE_NONE))
+    return QSPEC_ERR_CUDA;
+  return launch_qgemm<kInt8>(p.mt, tw, tx, ts, a, p.grid, dev, stream);
 }
 
 }  // namespace
@@ -311,7 +318,7 @@ qspec_status qspec_quantize_weights(const float* w, int64_t n, int64_t k, int32_
   if (!w || !wq || !ws) return QSPEC_ERR_INVALID_ARG;
   if (n < 1 || (group != 64 && group != 128) || k < group || (k % group) != 0)
     return QSPEC_ERR_INVALID_ARG;
-  if (!aligned(w, 16) || !aligned(wq, 2) || !aligned(ws, 2)) return QSPEC_ERR_INVALID_ARG;
+  if (!aligned(w, 16) || !aligned(wq, 2) || !aligned(ws, 16)) return QSPEC_ERR_INVALID_ARG;
   const long long warps = n * (k / group);
   const long long blocks = (warps + 7) / 8;
   if (blocks > 0x7FFFFFFFll) return QSPEC_ERR_INVALID_ARG;

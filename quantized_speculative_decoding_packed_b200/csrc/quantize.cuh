@@ -18,6 +18,7 @@ namespace qspec {
 __device__ __forceinline__ int clamp_q(int v) { return v < -8 ? -8 : (v > 7 ? 7 : v); }
 
 // One warp per (row n, group g).  Lane l handles GROUP/32 consecutive values.
+// ws rows have scale_row_stride(k / GROUP) entries; the padding is zeroed.
 template <int GROUP>
 __global__ void __launch_bounds__(256) quantize_weights_kernel(const float* __restrict__ w,
                                                                int64_t n_rows, int64_t k,
@@ -61,7 +62,11 @@ __global__ void __launch_bounds__(256) quantize_weights_kernel(const float* __re
   } else {
     *dst = static_cast<uint8_t>(packed);
   }
-  if (lane == 0) ws[row * groups_per_row + g] = __half_as_ushort(sh);
+  const int64_t ldg = scale_row_stride(groups_per_row);
+  if (lane == 0) ws[row * ldg + g] = __half_as_ushort(sh);
+  // the row's padding entries (a row's last group writes them)
+  if (g == groups_per_row - 1 && lane < ldg - groups_per_row)
+    ws[row * ldg + groups_per_row + lane] = 0;
 }
 
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) {

@@ -106,15 +106,23 @@ def workspace_status(ws: torch.Tensor, stream=None) -> int:
     return int(LIB.qspec_workspace_status(_ptr(ws), _stream(stream)))
 
 
+def scale_row_stride(k: int, group: int) -> int:
+    """Entries per row of the scale matrix: k/group rounded up to a multiple of 8."""
+    return (k // group + 7) // 8 * 8
+
+
 def quantize_weights(w: torch.Tensor, group: int = 128, wq: torch.Tensor | None = None,
                      ws: torch.Tensor | None = None, stream=None):
-    """fp32 [N][K] -> (wq uint8 [N][K/2], ws fp16 [N][K/group])."""
+    """fp32 [N][K] -> (wq uint8 [N][K/2], ws fp16 [N][scale_row_stride(K, group)]).
+
+    ws[:, :K/group] holds the group scales; the padding columns are zero.
+    """
     _need(w, torch.float32, "w")
     n, k = w.shape
     if wq is None:
         wq = torch.empty((n, k // 2), dtype=torch.uint8, device=w.device)
     if ws is None:
-        ws = torch.empty((n, k // group), dtype=torch.float16, device=w.device)
+        ws = torch.empty((n, scale_row_stride(k, group)), dtype=torch.float16, device=w.device)
     _check(LIB.qspec_quantize_weights(_ptr(w), n, k, group, _ptr(wq), _ptr(ws), _stream(stream)),
            "qspec_quantize_weights")
     return wq, ws

@@ -21,7 +21,11 @@ def _check_weights(qs, w, group):
     wq, ws = qs.quantize_weights(cuda_f32(w), group)
     torch.cuda.synchronize()
     q, s_h = orc.quantize_weights(w, group)
-    assert np.array_equal(ws.cpu().numpy().view(np.uint16), s_h.view(np.uint16))
+    got = ws.cpu().numpy().view(np.uint16)
+    g_cnt = s_h.shape[1]
+    assert got.shape[1] == qs.scale_row_stride(w.shape[1], group)
+    assert np.array_equal(got[:, :g_cnt], s_h.view(np.uint16))
+    assert not got[:, g_cnt:].any()                    # row padding is stored as zeros
     assert np.array_equal(wq.cpu().numpy(), orc.pack_int4(q))
 
 

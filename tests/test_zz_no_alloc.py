@@ -77,7 +77,7 @@ def test_refuses_shapes_beyond_the_builtin_scratch(qs):
     m, n, k = 200, 4096, 4096          # token tile 128: split-K slots exceed 16 MiB on a 148-SM part
     x = torch.zeros((m, k), dtype=torch.bfloat16, device="cuda")
     wq = torch.zeros((n, k // 2), dtype=torch.uint8, device="cuda")
-    ws = torch.zeros((n, k // 128), dtype=torch.float16, device="cuda")
+    ws = torch.zeros((n, qs.scale_row_stride(k, 128)), dtype=torch.float16, device="cuda")
     y = torch.zeros((m, n), dtype=torch.float32, device="cuda")
     assert _call_noalloc(qs, x, wq, ws, n, 128, y) == 4    # QSPEC_ERR_WORKSPACE_TOO_SMALL
     torch.cuda.synchronize()
