@@ -74,6 +74,29 @@ constexpr int kScaleTileGroups = 8;
 constexpr int kScaleTileBytes = kTileN * kScaleTileGroups * 2;
 constexpr int kNumSc = 8;
 constexpr int kTmemCols = 512;                   // all of tensor memory: one CTA per SM
+// mbarriers (rings, MMA drain, scale tiles, split-tile hand-offs) and 8 words
+// of flags share a 1 KB block, in this order: pk_full, pk_empty, a_full,
+// a_empty, x_full, x_empty, acc_full, acc_empty, mma_done, sc_full, sc_empty,
+// flush[2], ticket[2], tail.
+namespace bar {
+constexpr int kPkFull = 0, kPkEmpty = kPkFull + kMaxPk, kAFull = kPkEmpty + kMaxPk;
+constexpr int kAEmpty = kAFull + kMaxA, kXFull = kAEmpty + kMaxA, kXEmpty = kXFull + kMaxX;
+constexpr int kAccFull = kXEmpty + kMaxX, kAccEmpty = kAccFull + kMaxAcc;
+constexpr int kMmaDone = kAccEmpty + kMaxAcc, kScFull = kMmaDone + 1, kScEmpty = kScFull + kNumSc;
+constexpr int kFlush = kScEmpty + kNumSc, kTicket = kFlush + 2, kTail = kTicket + 2;
+constexpr int kCount = kTail + 1;
+}  // namespace bar
+constexpr int kNumBars = bar::kCount;
+static_assert(kNumBars * 8 + 8 * 4 <= 1024, "barrier block overflow");
+
+// Arrival count of barrier b in that order.
+__device__ __forceinline__ uint32_t bar_count(int b, int epi_warps) {
+  if (b >= bar::kPkEmpty && b < bar::kAEmpty) return kConvTeamWarps;   // pk_empty, a_full
+  if (b >= bar::kAccEmpty && b < bar::kMmaDone) return epi_warps;      // acc_empty
+  if (b == bar::kMmaDone) return 2;                                    // both MMA warps
+  if (b >= bar::kScEmpty && b < bar::kTicket) return epi_warps;        // sc_empty, flush
+  return 1;
+}
 
 __host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 __host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
@@ -212,7 +235,9 @@ __device__ __forceinline__ void grid_launch_dependents() {
 }
 
 // Ticket of split tile t after this CTA published its share (one thread).
-// Returns true for the tile's last contributor, which then adds the shares.
+// Returns true for the tile's last contributor, which then adds the shares;
+// the last contributor also returns the ticket to zero for the next launch
+// (nobody else touches it once every contributor has arrived).
 __device__ __forceinline__ bool take_tile_ticket(const GemmArgs& args, long long t,
                                                  long long units, long long grid) {
   const long long tile_u0 = t * args.ku;
@@ -225,7 +250,20 @@ __device__ __forceinline__ bool take_tile_ticket(const GemmArgs& args, long long
                : "=r"(old)
                : "l"(args.counters + c_lo)
                : "memory");
-  return old == static_cast<uint32_t>(c_hi - c_lo);
+  const bool last = old == static_cast<uint32_t>(c_hi - c_lo);
+  if (last) args.counters[c_lo] = 0u;
+  return last;
+}
+
+// Number of contributors that have ticketed split tile t so far (relaxed;
+// pair with fence_acquire_gpu before reading their shares).
+__device__ __forceinline__ uint32_t peek_ticket(const uint32_t* counter) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+  return v;
+}
+__device__ __forceinline__ void fence_acquire_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
 }
 
 // kDbg (int8 mode only): also write the per-group integer accumulators.  A
@@ -245,23 +283,26 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   uint8_t* x_buf = pk_buf + NPK * C::kPkBytes;
   uint8_t* sc_buf = x_buf + NX * C::kXBytes;     // group-scale tiles
   uint64_t* bars = reinterpret_cast<uint64_t*>(sc_buf + C::kScaleBytes);
-  uint64_t* pk_full = bars;
-  uint64_t* pk_empty = pk_full + kMaxPk;
-  uint64_t* a_full = pk_empty + kMaxPk;    // widened unit in tensor memory
-  uint64_t* a_empty = a_full + kMaxA;
-  uint64_t* x_full = a_empty + kMaxA;
-  uint64_t* x_empty = x_full + kMaxX;
-  uint64_t* acc_full = x_empty + kMaxX;
-  uint64_t* acc_empty = acc_full + kMaxAcc;
-  uint64_t* mma_done = acc_empty + kMaxAcc;
-  uint64_t* sc_full = mma_done + 1;     // [kNumSc]: a scale tile has landed
-  uint64_t* sc_empty = sc_full + kNumSc; // [kNumSc]: the epilogue is done with it
-  uint64_t* flush_bar = sc_empty + kNumSc;   // the head split tile's share is published
-  uint64_t* ticket_bar = flush_bar + 1; // ... and its ticket taken (result in misc[3])
-  uint64_t* epi_sync = ticket_bar + 1;
-  uint32_t* misc = reinterpret_cast<uint32_t*>(epi_sync + 1);
-  // misc[0]: tensor-memory base; misc[1]: abort flag; misc[2]: reducer flag;
-  // misc[3]: this CTA is the last contributor of its head split tile
+  uint64_t* pk_full = bars + bar::kPkFull;
+  uint64_t* pk_empty = bars + bar::kPkEmpty;
+  uint64_t* a_full = bars + bar::kAFull;     // widened unit in tensor memory
+  uint64_t* a_empty = bars + bar::kAEmpty;
+  uint64_t* x_full = bars + bar::kXFull;
+  uint64_t* x_empty = bars + bar::kXEmpty;
+  uint64_t* acc_full = bars + bar::kAccFull;
+  uint64_t* acc_empty = bars + bar::kAccEmpty;
+  uint64_t* mma_done = bars + bar::kMmaDone;
+  uint64_t* sc_full = bars + bar::kScFull;   // [kNumSc]: a scale tile has landed
+  uint64_t* sc_empty = bars + bar::kScEmpty; // [kNumSc]: the epilogue is done with it
+  // [0]: the head split tile's share is published, [1]: the tail split tile's
+  uint64_t* flush_bar = bars + bar::kFlush;
+  uint64_t* ticket_bar = bars + bar::kTicket;  // ... and its ticket taken (misc[3], misc[6])
+  uint64_t* tail_bar = bars + bar::kTail;      // the other contributor's tail share is out
+  uint32_t* misc = reinterpret_cast<uint32_t*>(bars + bar::kCount);
+  // misc[0]: tensor-memory base; misc[1]: abort flag; misc[3]: this CTA is the
+  // last contributor of its head split tile; misc[5]: some epilogue warp left
+  // its tail-tile share in the workspace; misc[6]: ... and this CTA is the
+  // tail tile's last contributor
   volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[1]);
 
   const int warp = threadIdx.x >> 5;
@@ -273,36 +314,27 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   const long long u_end = unit_begin(cta + 1, units, grid);
   const int ku = args.ku;
   const int gpu = args.groups_per_unit;
+  // The CTA's last segment [max(u_begin, tail_u0), u_end) lies in tile t_tail;
+  // it is a split tile unless it covers the whole tile.  When this CTA holds
+  // the tile's first unit and exactly one other CTA (the next one, which
+  // meets the tile at the start of its range) holds the rest, that CTA's
+  // share is normally published long before this one gets there: the tail
+  // then takes a fast path that adds the share directly (tail_fast).
+  const long long t_tail =
+      (u_begin < u_end) ? static_cast<uint32_t>(u_end - 1) / static_cast<uint32_t>(ku) : 0;
+  const long long tail_u0 = t_tail * ku;
+  const bool tail_split = (u_begin < u_end) && !(u_begin <= tail_u0 && u_end == tail_u0 + ku);
+  const bool tail_fast = tail_split && u_begin <= tail_u0 &&
+                         unit_owner(tail_u0 + ku - 1, units, grid) == cta + 1;
 
   if (threadIdx.x == 0) QSPEC_PHASE(0);
+  if (threadIdx.x == 0) QSPEC_STAMP(8, 0);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NPK; ++s) {
-      mbar_init(smem_u32(&pk_full[s]), 1);
-      mbar_init(smem_u32(&pk_empty[s]), kConvTeamWarps);
-    }
-    for (int s = 0; s < NA; ++s) {
-      mbar_init(smem_u32(&a_full[s]), kConvTeamWarps);
-      mbar_init(smem_u32(&a_empty[s]), 1);
-    }
-    for (int s = 0; s < NX; ++s) {
-      mbar_init(smem_u32(&x_full[s]), 1);
-      mbar_init(smem_u32(&x_empty[s]), 1);
-    }
-    for (int b = 0; b < NACC; ++b) {
-      mbar_init(smem_u32(&acc_full[b]), 1);
-      mbar_init(smem_u32(&acc_empty[b]), C::kEpiWarps);
-    }
-    mbar_init(smem_u32(mma_done), 2);
-    for (int s = 0; s < kNumSc; ++s) {
-      mbar_init(smem_u32(&sc_full[s]), 1);
-      mbar_init(smem_u32(&sc_empty[s]), C::kEpiWarps);
-    }
-    mbar_init(smem_u32(flush_bar), C::kEpiWarps);
-    mbar_init(smem_u32(ticket_bar), 1);
-    misc[3] = 0;
-    mbar_init(smem_u32(epi_sync), C::kEpiWarps);
+    for (int b = 0; b < kNumBars; ++b) mbar_init(smem_u32(&bars[b]), bar_count(b, C::kEpiWarps));
     misc[1] = 0;
-    misc[2] = 0;
+    misc[3] = 0;
+    misc[5] = 0;
+    misc[6] = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -320,6 +352,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   const uint32_t tmem_base = misc[0];
   QSPEC_TRACE_AT(tmem_base & 0xFFFF);
   if (threadIdx.x == 0) QSPEC_PHASE(1);
+  if (threadIdx.x == 0) QSPEC_STAMP(8, 1);
   // The next grid may be scheduled as SMs free up; it waits for this one to
   // complete before it reads inputs or writes anything.
   if (threadIdx.x == 0) grid_launch_dependents();
@@ -345,6 +378,9 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     RingPos rs;
     rs.init(0, kNumSc);
     int n_sc = 0;
+    bool tail_seen = false;
+    bool poll_pending = false;
+    uint32_t poll_val = 0;
     int i = 0;
     UnitCursor cur;
     cur.init(u_begin, ku, args.m_tiles);
@@ -372,6 +408,17 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
         rs.step(1, kNumSc);
         ++n_sc;
       }
+      if (tail_fast && u >= tail_u0 && lane == 0 && !tail_seen) {
+        if (poll_pending && poll_val == 1u) {
+          fence_acquire_gpu();
+          mbar_arrive(smem_u32(tail_bar));
+          tail_seen = true;
+        } else {
+          poll_val = peek_ticket(args.counters + cta);
+          poll_pending = true;
+        }
+      }
+      __syncwarp();
       if (head_pending && __all_sync(0xffffffffu, mbar_test_wait(smem_u32(flush_bar), 0))) {
         if (lane == 0) {
           misc[3] = take_tile_ticket(args, t_head, units, grid) ? 1u : 0u;
@@ -385,6 +432,54 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       if (lane == 0) {
         misc[3] = take_tile_ticket(args, t_head, units, grid) ? 1u : 0u;
         mbar_arrive(smem_u32(ticket_bar));
+      }
+      __syncwarp();
+    }
+    // Tail split tile: once this warp has issued every unit, watch the other
+    // contributor's ticket (fast-path tiles) until it arrives or the epilogue
+    // has finished the tail segment; then take this CTA's ticket if any
+    // epilogue warp left its share in the workspace.  If every warp took the
+    // fast path, this CTA was the last contributor and only returns the
+    // ticket to zero.
+    if (tail_split && !*abort_flag) {
+      bool fine = true;
+      tail_seen = __shfl_sync(0xffffffffu, tail_seen ? 1 : 0, 0) != 0;
+      if (tail_fast && !tail_seen) {
+        const uint64_t start = global_timer_ns();
+        for (;;) {
+          if (__all_sync(0xffffffffu, mbar_test_wait(smem_u32(&flush_bar[1]), 0))) break;
+          uint32_t c = 0;
+          if (lane == 0) c = peek_ticket(args.counters + cta);
+          if (__shfl_sync(0xffffffffu, c, 0) == 1u) {
+            if (lane == 0) {
+              fence_acquire_gpu();
+              mbar_arrive(smem_u32(tail_bar));
+            }
+            __syncwarp();
+            break;
+          }
+          if (*abort_flag) {
+            fine = false;
+            break;
+          }
+          if (global_timer_ns() - start > kWaitLimitNs) {
+            if (lane == 0) {
+              *abort_flag = 1;
+              if (args.status) atomicOr(args.status, kDevTimeout);
+            }
+            fine = false;
+            break;
+          }
+        }
+      }
+      fine = fine && warp_wait(smem_u32(&flush_bar[1]), 0, abort_flag, args.status);
+      if (fine && lane == 0) {
+        if (misc[5] != 0u) {
+          misc[6] = take_tile_ticket(args, t_tail, units, grid) ? 1u : 0u;
+          mbar_arrive(smem_u32(&ticket_bar[1]));
+        } else {
+          args.counters[cta] = 0u;
+        }
       }
       __syncwarp();
     }
@@ -438,6 +533,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       const int sa = ra.slot;
       const int sx = rx.slot;
       racc.init(i * gpu, NACC);
+      QSPEC_STAMP(15, i);
       ok = warp_wait(smem_u32(&a_full[sa]), ra.phase, abort_flag, args.status);
       ok = ok && warp_wait(smem_u32(&x_full[sx]), rx.phase, abort_flag, args.status);
       if (!ok) break;
@@ -449,6 +545,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
         const int b = racc.slot;
         ok = warp_wait(smem_u32(&acc_empty[b]), racc.phase ^ 1u, abort_flag, args.status);
         if (!ok) break;
+        QSPEC_STAMP(11, i * gpu + h);
         tc_fence_after();
         // One elected lane issues the group's MMAs and its commit back to back.
         if (elect_one_lane()) {
@@ -464,6 +561,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
           mma_commit(smem_u32(&acc_full[b]));
         }
         __syncwarp();
+        QSPEC_STAMP(12, i * gpu + h);
       }
       if (!ok) break;
       if (elect_one_lane()) {
@@ -623,7 +721,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
 #pragma unroll
         for (int c = 0; c < C::kCols; ++c) run[c] += __ldcg(src + (col0 + c) * kTileN + row);
       }
-      if (et == 0) args.counters[c_lo] = 0u;   // ready for the next launch
       const uint32_t n_tile = static_cast<uint32_t>(t) / static_cast<uint32_t>(args.m_tiles);
       const uint32_t m_tile = static_cast<uint32_t>(t) - n_tile * static_cast<uint32_t>(args.m_tiles);
       write_y(static_cast<int>(n_tile) * kTileN + row, static_cast<int>(m_tile) * MT + col0);
@@ -631,22 +728,10 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     const long long t_head = static_cast<uint32_t>(u_begin) / static_cast<uint32_t>(ku);
     const long long head_end = (u_end < (t_head + 1) * ku) ? u_end : (t_head + 1) * ku;
     const bool head_handoff = (u_begin < u_end) && head_end < u_end && u_begin != t_head * ku;
-    long long to_reduce[2];
-    int n_reduce = 0;
     RingPos acc;              // accumulator ring position of the next group
     acc.init(0, NACC);
     bool ok = true;
-    volatile int* reducer_flag = reinterpret_cast<volatile int*>(&misc[2]);
-    uint32_t epi_phase = 0;
-    // All epilogue warps meet here; bounded, unlike a hardware named barrier.
-    auto epi_barrier = [&]() -> bool {
-      __syncwarp();
-      if (elect_one_lane()) mbar_arrive(smem_u32(epi_sync));
-      __syncwarp();
-      const bool fine = warp_wait(smem_u32(epi_sync), epi_phase, abort_flag, args.status);
-      epi_phase ^= 1u;
-      return fine;
-    };
+    bool tail_slow = false;   // this warp left its tail-tile share for the ticket
     long long u = u_begin;
     UnitCursor tc;            // the tile of the next segment (no divisions per segment)
     tc.init(u_begin, ku, args.m_tiles);
@@ -666,10 +751,14 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       const int m0 = m_tile * MT + col0;
 #pragma unroll
       for (int c = 0; c < C::kCols; ++c) run[c] = 0.f;
+      const bool full = (seg_start == tile_u0) && (seg_end == tile_u0 + ku);
+      const bool fast_tail = tail_fast && seg_end >= u_end;
       const int seg_groups = static_cast<int>(seg_end - seg_start) * gpu;
       int g = static_cast<int>(seg_start - tile_u0) * gpu;   // the row's scale group
       for (int jj = 0; jj < seg_groups; ++jj, ++g) {
-        if (ew == 0) QSPEC_STAMP(14, (static_cast<int>(seg_start - u_begin) * gpu + jj) & 63);
+        const int gi = static_cast<int>(seg_start - u_begin) * gpu + jj;   // trace index
+        (void)gi;
+        if (ew == 0) QSPEC_STAMP(14, gi);
         if (sc_cur < 0 || (g & (kScaleTileGroups - 1)) == 0) {
           if (sc_cur >= 0) {   // done with the previous tile
             __syncwarp();
@@ -689,6 +778,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
         const float sc = __half2float(__ushort_as_half(hbits));
         ok = warp_wait(smem_u32(&acc_full[acc.slot]), acc.phase, abort_flag, args.status);
         if (!ok) break;
+        if (ew == 0) QSPEC_STAMP(5, gi);
         tc_fence_after();
         const uint32_t taddr =
             lane_addr + static_cast<uint32_t>(C::kAccCol0 + acc.slot * MT + col0);
@@ -704,6 +794,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
             __syncwarp();
             if (elect_one_lane()) mbar_arrive(smem_u32(&acc_empty[acc.slot]));
             __syncwarp();
+            if (ew == 0) QSPEC_STAMP(6, gi);
           }
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -729,37 +820,55 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       if (!ok) break;
       u = seg_end;
       if (et == 0) QSPEC_PHASE(u >= u_end ? 5 : 7);
+      if (et == 0 && u >= u_end) QSPEC_STAMP(8, 4);
 
-      const bool full = (seg_start == tile_u0) && (seg_end == tile_u0 + ku);
       if (full) {
         write_y(n, m0);
       } else {
-        const int k = (seg_start == u_begin) ? 0 : 1;
-        float* mine = args.partials + static_cast<long long>(2 * cta + k) * MT * kTileN;
+        // A split tile.  Fast tail: the other contributor has published, so
+        // this warp adds its share (same order as the reduction: this CTA's
+        // share first) and writes y.  Otherwise the share goes to the
+        // workspace and the weight producer takes the ticket (the head tile
+        // right away, the tail tile once every warp is done with it).
+        const bool last_seg = seg_end >= u_end;
+        bool fast = false;
+        if (fast_tail) {
+          fast = __all_sync(0xffffffffu, mbar_test_wait(smem_u32(tail_bar), 0));
+          if (fast) {
+            // the next CTA's share sits in its head slot
+            const float* src = args.partials + static_cast<long long>(2 * (cta + 1)) * MT * kTileN;
 #pragma unroll
-        for (int c = 0; c < C::kCols; ++c) mine[(col0 + c) * kTileN + row] = run[c];
-        if (seg_end < u_end) {
-          // The CTA's first tile with more to follow: publish the share and go
-          // on; the weight producer takes the ticket.
-          __syncwarp();
-          if (elect_one_lane()) mbar_arrive(smem_u32(flush_bar));
-          __syncwarp();
-        } else {
-          // The CTA's last tile: take the ticket here.
-          if (!epi_barrier()) break;
-          if (et == 0) *reducer_flag = take_tile_ticket(args, t, units, grid) ? 1 : 0;
-          if (!epi_barrier()) break;
-          if (*reducer_flag != 0) to_reduce[n_reduce++] = t;
+            for (int c = 0; c < C::kCols; ++c) run[c] += __ldcg(src + (col0 + c) * kTileN + row);
+            write_y(n, m0);
+          }
         }
+        if (!fast) {
+          const int k = (seg_start == u_begin) ? 0 : 1;
+          float* mine = args.partials + static_cast<long long>(2 * cta + k) * MT * kTileN;
+#pragma unroll
+          for (int c = 0; c < C::kCols; ++c) mine[(col0 + c) * kTileN + row] = run[c];
+        }
+        __syncwarp();
+        if (elect_one_lane()) {
+          if (last_seg && !fast) misc[5] = 1u;
+          mbar_arrive(smem_u32(&flush_bar[last_seg ? 1 : 0]));
+        }
+        __syncwarp();
+        tail_slow = last_seg && !fast;
       }
     }
     // The split tiles whose last ticket came to this CTA are added up here,
-    // after the CTA's own tiles: the last one and possibly the head one.
+    // after the CTA's own tiles.
+    if (et == 0) QSPEC_STAMP(8, 7);
     if (ok && head_handoff) {
-      ok = warp_wait(smem_u32(ticket_bar), 0, abort_flag, args.status);
-      if (ok && misc[3] != 0u) to_reduce[n_reduce++] = t_head;
+      ok = warp_wait(smem_u32(&ticket_bar[0]), 0, abort_flag, args.status);
+      if (ok && misc[3] != 0u) reduce_tile(t_head);
     }
-    for (int r = 0; ok && r < n_reduce; ++r) reduce_tile(to_reduce[r]);
+    if (ok && tail_slow) {
+      ok = warp_wait(smem_u32(&ticket_bar[1]), 0, abort_flag, args.status);
+      if (ok && misc[6] != 0u) reduce_tile(t_tail);
+    }
+    if (et == 0) QSPEC_STAMP(8, 2);
   }
 
   QSPEC_TRACE_AT(0xFFF0);
@@ -768,6 +877,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) QSPEC_PHASE(8);
+  if (threadIdx.x == 0) QSPEC_STAMP(8, 3);
   QSPEC_STAMP_FLUSH();
   if (warp == 2) {
     tc_fence_after();
