@@ -346,7 +346,8 @@ def main():
                     t = with_events and li == 0
                     if t:
                         mark(("w4a4", pss, si, 0))
-                    qspec.gemm_w4a4(x16[si], wq[li][si], ws[li][si], GROUP, y=y16[si], work=work)
+                    qspec.gemm_w4a4(x16[si], wq[li][si], ws[li][si], GROUP, y=y16[si], work=work,
+                                    weights_ready=True)
                     if t:
                         mark(("w4a4", pss, si, 1))
         for li in range(L):
@@ -354,7 +355,8 @@ def main():
                 t = with_events and li == 0
                 if t:
                     mark(("w4a16", 0, si, 0))
-                qspec.gemm_w4a16(x80[si], wq[li][si], ws[li][si], GROUP, y=y80[si], work=work)
+                qspec.gemm_w4a16(x80[si], wq[li][si], ws[li][si], GROUP, y=y80[si], work=work,
+                                 weights_ready=True)
                 if t:
                     mark(("w4a16", 0, si, 1))
         if with_events:

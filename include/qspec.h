@@ -51,6 +51,21 @@ typedef enum qspec_status {
   QSPEC_ERR_BAD_INPUT = 6           /* a kernel saw invalid data, e.g. a draft token >= vocab */
 } qspec_status;
 
+/*
+ * GEMM flags.
+ *  QSPEC_GEMM_WEIGHTS_READY: `wq` and `ws` are not being written by any work
+ *    that may still be running when this call's kernels start (typically:
+ *    the weights were quantized or copied once, and that work has been waited
+ *    for).  The GEMM kernels are launched as programmatic dependents of the
+ *    preceding kernel on the stream; with this flag they stream the packed
+ *    weights and scales into shared and tensor memory while that kernel is
+ *    still finishing, and wait for it only where they read activations or
+ *    write anything.  Without the flag the weights are read only after the
+ *    preceding kernel has completed.  Results are identical either way.
+ * Other bits are reserved and must be zero.
+ */
+#define QSPEC_GEMM_WEIGHTS_READY 1u
+
 /* Operation ids for qspec_workspace_size(). */
 enum {
   QSPEC_OP_QUANTIZE_WEIGHTS = 0,
@@ -108,6 +123,7 @@ qspec_status qspec_quant_act(const uint16_t* x, int64_t m, int64_t k, uint8_t* x
  *           call that completes leaves it ready for the next one.
  *  dbg_acc  optional (may be NULL): [m][n][k/group] int32 out, the per-group
  *           integer accumulators.
+ *  flags    0 or QSPEC_GEMM_WEIGHTS_READY (see above).
  * Requires m, n >= 1, group in {64, 128}, k a multiple of 128, and fewer than
  * 2^22 work units ceil(m / T) * ceil(n / 128) * (k / 128), where the token
  * tile T is m rounded up to a multiple of 16 for m <= 96, else 128.
@@ -115,7 +131,7 @@ qspec_status qspec_quant_act(const uint16_t* x, int64_t m, int64_t k, uint8_t* x
 qspec_status qspec_gemm_w4a4(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
                              const uint16_t* ws, int64_t n, int32_t group, float* y,
                              void* workspace, size_t workspace_bytes, int32_t* dbg_acc,
-                             void* stream);
+                             uint32_t flags, void* stream);
 
 /*
  * W4A16 verifying GEMM: y = x . deq(wq, ws)^T with bf16 activations and the
@@ -127,7 +143,8 @@ qspec_status qspec_gemm_w4a4(const uint16_t* x, int64_t m, int64_t k, const uint
  */
 qspec_status qspec_gemm_w4a16(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
                               const uint16_t* ws, int64_t n, int32_t group, float* y,
-                              void* workspace, size_t workspace_bytes, void* stream);
+                              void* workspace, size_t workspace_bytes, uint32_t flags,
+                              void* stream);
 
 /*
  * Speculative accept / residual resample for a batch of sequences (SpecQuant
@@ -185,7 +202,7 @@ qspec_status qspec_spec_accept(const float* p, const float* q, const int32_t* dr
 #define QSPEC_STATIC_SCRATCH_BYTES (16u << 20)
 qspec_status qspec_gemm_w4a16_noalloc(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
                                       const uint16_t* ws, int64_t n, int32_t group, float* y,
-                                      void* stream);
+                                      uint32_t flags, void* stream);
 
 /* Bytes of workspace an operation needs on the current device (0 = none).
  * Unused size arguments are ignored.  Returns 0 for invalid arguments too. */
@@ -196,6 +213,10 @@ size_t qspec_workspace_size(int32_t op, int64_t m, int64_t n, int64_t k, int32_t
  * `workspace`, clears it, and returns QSPEC_OK, QSPEC_ERR_TIMEOUT or
  * QSPEC_ERR_BAD_INPUT (or QSPEC_ERR_CUDA if the read itself failed). */
 qspec_status qspec_workspace_status(void* workspace, void* stream);
+
+/* Version of this ABI (2: the GEMM entry points take `flags`). */
+#define QSPEC_ABI_VERSION 2
+int32_t qspec_abi_version(void);
 
 /* Static, human-readable name of a status code. */
 const char* qspec_status_string(qspec_status status);

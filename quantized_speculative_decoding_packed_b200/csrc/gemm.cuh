@@ -145,6 +145,7 @@ struct GemmArgs {
   int groups_per_unit;     // 128 / group (1 or 2)
   int m_tiles, n_tiles, ku;
   long long units;         // m_tiles * n_tiles * ku
+  int weights_ready;       // wq/ws may be read before the preceding grid completes
   const uint16_t* ws;      // fp16 scales [N][K/group]
   const float* s_a;        // W4A4: per-token scales [M]
   float* y;                // [M][N]
@@ -265,6 +266,14 @@ __device__ __forceinline__ uint32_t peek_ticket(const uint32_t* counter) {
 __device__ __forceinline__ void fence_acquire_gpu() {
   asm volatile("fence.acq_rel.gpu;" ::: "memory");
 }
+__device__ __forceinline__ uint32_t ld_acquire_cta(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_cta(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
 
 // kDbg (int8 mode only): also write the per-group integer accumulators.  A
 // separate instantiation keeps those stores out of the hot loop's code.
@@ -302,7 +311,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   // misc[0]: tensor-memory base; misc[1]: abort flag; misc[3]: this CTA is the
   // last contributor of its head split tile; misc[5]: some epilogue warp left
   // its tail-tile share in the workspace; misc[6]: ... and this CTA is the
-  // tail tile's last contributor
+  // tail tile's last contributor; misc[7]: the preceding grid has completed
   volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[1]);
 
   const int warp = threadIdx.x >> 5;
@@ -335,6 +344,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     misc[3] = 0;
     misc[5] = 0;
     misc[6] = 0;
+    misc[7] = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -368,10 +378,12 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     const long long t_head = static_cast<uint32_t>(u_begin) / static_cast<uint32_t>(ku);
     const long long head_end = (u_end < (t_head + 1) * ku) ? u_end : (t_head + 1) * ku;
     bool head_pending = (u_begin < u_end) && head_end < u_end && u_begin != t_head * ku;
-    // W4A16: the weights may come from the preceding grid.  W4A4 always runs
-    // behind its own activation quantization, which launched this grid only
-    // after the grid before it had completed.
-    if constexpr (!kInt8) grid_dependency_wait();
+    // The weights may come from the preceding grid unless the caller vouches
+    // otherwise.  W4A4 runs behind its own activation quantization, which
+    // then launches this grid only after the grid before it has completed.
+    if constexpr (!kInt8) {
+      if (!args.weights_ready) grid_dependency_wait();
+    }
     // Group scales: one TMA tile (8 groups x 128 rows) whenever a unit starts a
     // new run of 8 groups of its tile, or is this CTA's first unit; the
     // epilogue walks the same sequence.
@@ -408,7 +420,9 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
         rs.step(1, kNumSc);
         ++n_sc;
       }
-      if (tail_fast && u >= tail_u0 && lane == 0 && !tail_seen) {
+      // (only once the epilogue has seen the preceding grid complete: its
+      // tickets may still be in use before that)
+      if (tail_fast && u >= tail_u0 && lane == 0 && !tail_seen && ld_acquire_cta(&misc[7]) != 0u) {
         if (poll_pending && poll_val == 1u) {
           fence_acquire_gpu();
           mbar_arrive(smem_u32(tail_bar));
@@ -442,6 +456,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     // fast path, this CTA was the last contributor and only returns the
     // ticket to zero.
     if (tail_split && !*abort_flag) {
+      grid_dependency_wait();   // the preceding grid's tickets are settled
       bool fine = true;
       tail_seen = __shfl_sync(0xffffffffu, tail_seen ? 1 : 0, 0) != 0;
       if (tail_fast && !tail_seen) {
@@ -677,6 +692,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     const int et = ew * 32 + lane;             // 0 .. kEpiThreads-1
     const int G = args.groups_per_row;
     grid_dependency_wait();   // no global write before the preceding grid is done
+    if (et == 0) st_release_cta(&misc[7], 1u);   // ... and its tickets are settled
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
 
     // Group scales come as TMA tiles of 8 groups x 128 rows from the weight

@@ -219,8 +219,10 @@ qspec_status launch_qgemm(int mt, const CUtensorMap& tw, const CUtensorMap& tx, 
 template <bool kInt8>
 qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
                       const uint16_t* ws, int64_t n, int32_t group, float* y, void* workspace,
-                      size_t workspace_bytes, int32_t* dbg_acc, void* stream_v) {
+                      size_t workspace_bytes, int32_t* dbg_acc, uint32_t flags, void* stream_v) {
   if (!x || !wq || !ws || !y || !workspace) return QSPEC_ERR_INVALID_ARG;
+  if ((flags & ~QSPEC_GEMM_WEIGHTS_READY) != 0u) return QSPEC_ERR_INVALID_ARG;
+  const bool weights_ready = (flags & QSPEC_GEMM_WEIGHTS_READY) != 0u;
   if (!gemm_shape_ok(m, n, k, group)) return QSPEC_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(wq, 16) || !aligned(ws, 16) || !aligned(y, 4) ||
       !aligned(workspace, 16) || (dbg_acc && !aligned(dbg_acc, 4)))
@@ -251,6 +253,7 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
   a.n_tiles = p.n_tiles;
   a.ku = p.ku;
   a.units = p.units;
+  a.weights_ready = weights_ready ? 1 : 0;
   a.ws = ws;
   a.y = y;
   a.dbg_acc = dbg_acc;
@@ -261,7 +264,9 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
   if constexpr (kInt8) {
     int8_t* xq = reinterpret_cast<int8_t*>(wsp + p.off_xq);
     float* sa = reinterpret_cast<float*>(wsp + p.off_sa);
-    // Also a programmatic dependent: it waits for the preceding grid itself.
+    // Also a programmatic dependent: it waits for the preceding grid itself,
+    // and lets the GEMM launch once it has (or, when the weights are ready,
+    // at once: the GEMM then reads nothing else before its own waits).
     cudaLaunchConfig_t qc = {};
     qc.gridDim = dim3(static_cast<unsigned>(m));
     qc.blockDim = dim3(256);
@@ -272,8 +277,9 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
     qc.attrs = qa;
     qc.numAttrs = 1;
     void* qout = xq;
-    if (cudaLaunchKernelEx(&qc, quant_act_kernel<false>, x, static_cast<int64_t>(k), qout, sa) !=
-        cudaSuccess) {
+    const int early = weights_ready ? 1 : 0;
+    if (cudaLaunchKernelEx(&qc, quant_act_kernel<false>, x, static_cast<int64_t>(k), qout, sa,
+                           early) != cudaSuccess) {
       cudaGetLastError();
       return QSPEC_ERR_CUDA;
     }
@@ -340,23 +346,27 @@ qspec_status qspec_quant_act(const uint16_t* x, int64_t m, int64_t k, uint8_t* x
   qspec_status st = current_device(nullptr, nullptr);
   if (st != QSPEC_OK) return st;
   quant_act_kernel<true><<<static_cast<unsigned>(m), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      x, k, xq, xs);
+      x, k, xq, xs, 0);
   return cudaGetLastError() == cudaSuccess ? QSPEC_OK : QSPEC_ERR_CUDA;
 }
 
 qspec_status qspec_gemm_w4a4(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
                              const uint16_t* ws, int64_t n, int32_t group, float* y,
                              void* workspace, size_t workspace_bytes, int32_t* dbg_acc,
-                             void* stream) {
-  return run_gemm<true>(x, m, k, wq, ws, n, group, y, workspace, workspace_bytes, dbg_acc, stream);
+                             uint32_t flags, void* stream) {
+  return run_gemm<true>(x, m, k, wq, ws, n, group, y, workspace, workspace_bytes, dbg_acc, flags,
+                        stream);
 }
 
 qspec_status qspec_gemm_w4a16(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
                               const uint16_t* ws, int64_t n, int32_t group, float* y,
-                              void* workspace, size_t workspace_bytes, void* stream) {
-  return run_gemm<false>(x, m, k, wq, ws, n, group, y, workspace, workspace_bytes, nullptr,
+                              void* workspace, size_t workspace_bytes, uint32_t flags,
+                              void* stream) {
+  return run_gemm<false>(x, m, k, wq, ws, n, group, y, workspace, workspace_bytes, nullptr, flags,
                          stream);
 }
+
+int32_t qspec_abi_version(void) { return QSPEC_ABI_VERSION; }
 
 qspec_status qspec_spec_accept(const float* p, const float* q, const int32_t* draft,
                                const float* u_acc, const float* u_res, int32_t batch,
@@ -450,8 +460,9 @@ std::mutex g_static_scratch_mutex;
 
 qspec_status qspec_gemm_w4a16_noalloc(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
                                       const uint16_t* ws, int64_t n, int32_t group, float* y,
-                                      void* stream) {
+                                      uint32_t flags, void* stream) {
   if (!x || !wq || !ws || !y) return QSPEC_ERR_INVALID_ARG;
+  if ((flags & ~QSPEC_GEMM_WEIGHTS_READY) != 0u) return QSPEC_ERR_INVALID_ARG;
   if (!gemm_shape_ok(m, n, k, group)) return QSPEC_ERR_INVALID_ARG;
   int dev = 0;
   DeviceInfo info;
@@ -484,7 +495,7 @@ qspec_status qspec_gemm_w4a16_noalloc(const uint16_t* x, int64_t m, int64_t k, c
     return QSPEC_ERR_CUDA;
   }
   return run_gemm<false>(x, m, k, wq, ws, n, group, y, scratch, QSPEC_STATIC_SCRATCH_BYTES, nullptr,
-                         stream);
+                         flags, stream);
 }
 
 const char* qspec_status_string(qspec_status status) {

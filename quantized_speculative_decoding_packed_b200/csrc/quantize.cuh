@@ -79,19 +79,27 @@ __device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) {
 template <bool kPacked>
 __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restrict__ x,
                                                         int64_t k, void* __restrict__ out,
-                                                        float* __restrict__ scales) {
+                                                        float* __restrict__ scales,
+                                                        int early_trigger) {
   __shared__ float red[8];
   const int64_t row = blockIdx.x;
   const uint16_t* xr = x + row * k;
   const int tid = threadIdx.x;
   QSPEC_TRACE_AT(1);
   // This kernel may be launched as a programmatic dependent of the previous
-  // grid: wait for it (complete, memory flushed; a no-op otherwise), then let
-  // the GEMM that consumes our output launch.  That GEMM can then stream its
-  // weights at once, since whatever wrote them has finished, and waits for
-  // this kernel (griddepcontrol.wait) only where it reads x and s_a.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // grid: wait for it (complete, memory flushed; a no-op otherwise) and let
+  // the GEMM that consumes our output launch.  By default the GEMM launches
+  // only after the wait, so whatever wrote its weights has finished when it
+  // streams them; with early_trigger (the caller vouches that the weights
+  // are ready) it launches at once.  Either way the GEMM waits for this
+  // kernel (griddepcontrol.wait) where it reads x and s_a.
+  if (early_trigger) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+  } else {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  }
   if (!QSPEC_ALIGN_OK(reinterpret_cast<uintptr_t>(xr), 16) ||
       !QSPEC_ALIGN_OK(reinterpret_cast<uintptr_t>(out), 8))
     return;

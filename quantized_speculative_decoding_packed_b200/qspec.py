@@ -23,7 +23,9 @@ OP_QUANTIZE_WEIGHTS, OP_QUANT_ACT, OP_GEMM_W4A4, OP_GEMM_W4A16, OP_SPEC_ACCEPT =
 
 EXPORTED = ("qspec_quantize_weights", "qspec_quant_act", "qspec_gemm_w4a4", "qspec_gemm_w4a16",
             "qspec_spec_accept", "qspec_workspace_size", "qspec_workspace_status",
-            "qspec_status_string", "qspec_gemm_w4a16_noalloc")
+            "qspec_status_string", "qspec_gemm_w4a16_noalloc", "qspec_abi_version")
+ABI_VERSION = 2
+GEMM_WEIGHTS_READY = 1   # flag: wq/ws are not written by work still in flight
 
 
 class QSpecError(RuntimeError):
@@ -38,12 +40,15 @@ def _load() -> ctypes.CDLL:
             f"libqspec.so not found at {_LIB_PATH}; build it with "
             "`python -m quantized_speculative_decoding_packed_b200.build`")
     lib = ctypes.CDLL(_LIB_PATH)
-    P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+    P, I64, I32, U32, SZ = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_uint32,
+                            ctypes.c_size_t)
     lib.qspec_quantize_weights.argtypes = [P, I64, I64, I32, P, P, P]
     lib.qspec_quant_act.argtypes = [P, I64, I64, P, P, P]
-    lib.qspec_gemm_w4a4.argtypes = [P, I64, I64, P, P, I64, I32, P, P, SZ, P, P]
-    lib.qspec_gemm_w4a16.argtypes = [P, I64, I64, P, P, I64, I32, P, P, SZ, P]
-    lib.qspec_gemm_w4a16_noalloc.argtypes = [P, I64, I64, P, P, I64, I32, P, P]
+    lib.qspec_gemm_w4a4.argtypes = [P, I64, I64, P, P, I64, I32, P, P, SZ, P, U32, P]
+    lib.qspec_gemm_w4a16.argtypes = [P, I64, I64, P, P, I64, I32, P, P, SZ, U32, P]
+    lib.qspec_gemm_w4a16_noalloc.argtypes = [P, I64, I64, P, P, I64, I32, P, U32, P]
+    lib.qspec_abi_version.argtypes = []
+    lib.qspec_abi_version.restype = I32
     lib.qspec_spec_accept.argtypes = [P, P, P, P, P, I32, I32, I32, P, P, P, SZ, P]
     lib.qspec_workspace_size.argtypes = [I32, I64, I64, I64, I32, I32, I32, I32]
     lib.qspec_workspace_size.restype = SZ
@@ -54,6 +59,9 @@ def _load() -> ctypes.CDLL:
                  "qspec_gemm_w4a16", "qspec_spec_accept", "qspec_workspace_status",
                  "qspec_gemm_w4a16_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
+    if lib.qspec_abi_version() != ABI_VERSION:
+        raise ImportError(f"{_LIB_PATH} has ABI version {lib.qspec_abi_version()}, "
+                          f"this binding needs {ABI_VERSION}; rebuild the library")
     return lib
 
 
@@ -144,8 +152,14 @@ def quant_act(x: torch.Tensor, xq: torch.Tensor | None = None, xs: torch.Tensor 
 
 def gemm_w4a4(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor, group: int = 128,
               y: torch.Tensor | None = None, work: torch.Tensor | None = None,
-              dbg_acc: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """W4A4 drafting GEMM: y[M][N] fp32 = quant(x) . deq(wq, ws)^T."""
+              dbg_acc: torch.Tensor | None = None, stream=None,
+              weights_ready: bool = False) -> torch.Tensor:
+    """W4A4 drafting GEMM: y[M][N] fp32 = quant(x) . deq(wq, ws)^T.
+
+    weights_ready: wq/ws are not being written by work that may still be
+    running (sets QSPEC_GEMM_WEIGHTS_READY; the weights then stream while the
+    preceding kernel finishes).
+    """
     _need(x, torch.bfloat16, "x")
     m, k = x.shape
     n = wq.shape[0]
@@ -155,14 +169,15 @@ def gemm_w4a4(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor, group: int = 
     if work is None:
         work = workspace(need, x.device)
     _check(LIB.qspec_gemm_w4a4(_ptr(x), m, k, _ptr(wq), _ptr(ws), n, group, _ptr(y), _ptr(work),
-                               work.numel(), _ptr(dbg_acc), _stream(stream)), "qspec_gemm_w4a4")
+                               work.numel(), _ptr(dbg_acc), GEMM_WEIGHTS_READY if weights_ready else 0,
+                               _stream(stream)), "qspec_gemm_w4a4")
     return y
 
 
 def gemm_w4a16(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor, group: int = 128,
                y: torch.Tensor | None = None, work: torch.Tensor | None = None,
-               stream=None) -> torch.Tensor:
-    """W4A16 verifying GEMM: y[M][N] fp32 = x . deq(wq, ws)^T."""
+               stream=None, weights_ready: bool = False) -> torch.Tensor:
+    """W4A16 verifying GEMM: y[M][N] fp32 = x . deq(wq, ws)^T (weights_ready: as gemm_w4a4)."""
     _need(x, torch.bfloat16, "x")
     m, k = x.shape
     n = wq.shape[0]
@@ -172,12 +187,14 @@ def gemm_w4a16(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor, group: int =
     if work is None:
         work = workspace(need, x.device)
     _check(LIB.qspec_gemm_w4a16(_ptr(x), m, k, _ptr(wq), _ptr(ws), n, group, _ptr(y), _ptr(work),
-                                work.numel(), _stream(stream)), "qspec_gemm_w4a16")
+                                work.numel(), GEMM_WEIGHTS_READY if weights_ready else 0,
+                                _stream(stream)), "qspec_gemm_w4a16")
     return y
 
 
 def gemm_w4a16_noalloc(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor, group: int = 128,
-                       y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+                       y: torch.Tensor | None = None, stream=None,
+                       weights_ready: bool = False) -> torch.Tensor:
     """W4A16 verifying GEMM using the library's built-in scratch (no workspace).
 
     For callers that cannot allocate device memory where they call; the
@@ -189,6 +206,7 @@ def gemm_w4a16_noalloc(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor, grou
     if y is None:
         y = torch.empty((m, n), dtype=torch.float32, device=x.device)
     _check(LIB.qspec_gemm_w4a16_noalloc(_ptr(x), m, k, _ptr(wq), _ptr(ws), n, group, _ptr(y),
+                                        GEMM_WEIGHTS_READY if weights_ready else 0,
                                         _stream(stream)), "qspec_gemm_w4a16_noalloc")
     return y
 

@@ -179,13 +179,15 @@ def test_one_workspace_shared_across_shapes(qs):
         assert qs.workspace_status(work) == 0
 
 
-def test_back_to_back_calls_overlap_safely(qs):
+@pytest.mark.parametrize("weights_ready", [False, True])
+def test_back_to_back_calls_overlap_safely(qs, weights_ready):
     """Calls are launched so that each may start while the previous finishes.
 
     A chain of W4A4 and W4A16 calls on one stream, with no synchronisation,
     shares one workspace (split-tile shares and tickets, quantized
     activations) and rewrites the same outputs; run eagerly and as a CUDA
-    graph, every output must be bit-identical to a standalone call.
+    graph, every output must be bit-identical to a standalone call.  With
+    weights_ready the weights stream before the preceding call completes.
     """
     shapes = [(16, 12288, 4096), (80, 4096, 11008), (16, 4096, 11008), (80, 12288, 4096)]
     ops, want = [], []
@@ -208,7 +210,7 @@ def test_back_to_back_calls_overlap_safely(qs):
     def chain():
         for _ in range(3):
             for (fn, x, wq, ws, m, n) in ops:
-                fn(x, wq, ws, 128, y=outs[(m, n)], work=work)
+                fn(x, wq, ws, 128, y=outs[(m, n)], work=work, weights_ready=weights_ready)
 
     for y in outs.values():
         y.fill_(float("nan"))
@@ -230,4 +232,33 @@ def test_back_to_back_calls_overlap_safely(qs):
     torch.cuda.synchronize()
     for (fn, x, wq, ws, m, n), ref in zip(ops, want):
         assert torch.equal(outs[(m, n)], ref)
+    assert qs.workspace_status(work) == 0
+
+
+@pytest.mark.parametrize("mode", ["w4a4", "w4a16"])
+def test_weights_rewritten_just_before_the_call(qs, mode):
+    """Without QSPEC_GEMM_WEIGHTS_READY the GEMM reads the weights only after
+    the kernel before it has finished: quantizing new weights into the same
+    buffers right before the call (no synchronisation) gives the new result."""
+    m = 16 if mode == "w4a4" else 80
+    n, k = 4096, 4096
+    fn = qs.gemm_w4a4 if mode == "w4a4" else qs.gemm_w4a16
+    g_old = synth.gemm_inputs("llama2_7b", m, n, k, 128, stream=70)
+    g_new = synth.gemm_inputs("llama2_7b", m, n, k, 128, stream=71)
+    x = cuda_bf16(g_new.x_bits)
+    wq_new, ws_new = qs.quantize_weights(cuda_f32(g_new.w), 128)
+    want = fn(x, wq_new, ws_new, 128).clone()
+    w_new = cuda_f32(g_new.w)
+    wq, ws = qs.quantize_weights(cuda_f32(g_old.w), 128)
+    work = torch.zeros(qs.workspace_size(qs.OP_GEMM_W4A4, m, n, k, 128), dtype=torch.uint8,
+                       device="cuda")
+    y = torch.empty((m, n), dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    for _ in range(3):
+        fn(x, wq, ws, 128, y=y, work=work)                  # old weights, keeps the GPU busy
+        qs.quantize_weights(w_new, 128, wq=wq, ws=ws)       # overwrite in place
+        fn(x, wq, ws, 128, y=y, work=work)                  # must see the new weights
+        torch.cuda.synchronize()
+        assert torch.equal(y, want)
+        qs.quantize_weights(cuda_f32(g_old.w), 128, wq=wq, ws=ws)
     assert qs.workspace_status(work) == 0

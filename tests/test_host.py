@@ -20,7 +20,7 @@ def lib():
 
 def declared_symbols():
     text = open(HEADER).read()
-    return sorted(set(re.findall(r"^\s*(?:qspec_status|size_t|const char\*)\s+(qspec_\w+)\s*\(",
+    return sorted(set(re.findall(r"^\s*(?:qspec_status|size_t|int32_t|const char\*)\s+(qspec_\w+)\s*\(",
                                  text, flags=re.M)))
 
 
@@ -28,8 +28,12 @@ def test_header_declares_the_boundary():
     syms = declared_symbols()
     for name in ("qspec_quantize_weights", "qspec_quant_act", "qspec_gemm_w4a4",
                  "qspec_gemm_w4a16", "qspec_spec_accept", "qspec_workspace_size",
-                 "qspec_workspace_status", "qspec_status_string"):
+                 "qspec_workspace_status", "qspec_status_string", "qspec_abi_version"):
         assert name in syms
+
+
+def test_abi_version(lib):
+    assert lib.LIB.qspec_abi_version() == lib.ABI_VERSION == 2
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -61,16 +65,24 @@ def test_quantize_weights_rejects(lib, args):
                                          (4, 256, 256, 96), (4, 64, 256, 64)])
 def test_gemm_rejects_bad_shapes(lib, m, k, n, group):
     assert lib.LIB.qspec_gemm_w4a4(FAKE, m, k, FAKE, FAKE, n, group, FAKE, FAKE, 1 << 30, None,
-                                   None) == 1
+                                   0, None) == 1
     assert lib.LIB.qspec_gemm_w4a16(FAKE, m, k, FAKE, FAKE, n, group, FAKE, FAKE, 1 << 30,
-                                    None) == 1
+                                    0, None) == 1
 
 
 def test_gemm_rejects_misaligned_pointers(lib):
     odd = ctypes.c_void_p(0x10008)
-    assert lib.LIB.qspec_gemm_w4a16(odd, 4, 256, FAKE, FAKE, 256, 64, FAKE, FAKE, 1 << 30, None) == 1
-    assert lib.LIB.qspec_gemm_w4a16(FAKE, 4, 256, odd, FAKE, 256, 64, FAKE, FAKE, 1 << 30, None) == 1
-    assert lib.LIB.qspec_gemm_w4a16(FAKE, 4, 256, FAKE, FAKE, 256, 64, FAKE, None, 1 << 30, None) == 1
+    assert lib.LIB.qspec_gemm_w4a16(odd, 4, 256, FAKE, FAKE, 256, 64, FAKE, FAKE, 1 << 30, 0, None) == 1
+    assert lib.LIB.qspec_gemm_w4a16(FAKE, 4, 256, odd, FAKE, 256, 64, FAKE, FAKE, 1 << 30, 0, None) == 1
+    assert lib.LIB.qspec_gemm_w4a16(FAKE, 4, 256, FAKE, FAKE, 256, 64, FAKE, None, 1 << 30, 0, None) == 1
+
+
+def test_gemm_rejects_reserved_flags(lib):
+    # a valid-looking call (aligned fake pointers, a supported shape) with a reserved bit set
+    assert lib.LIB.qspec_gemm_w4a16(FAKE, 4, 256, FAKE, FAKE, 256, 64, FAKE, FAKE, 1 << 30, 2, None) == 1
+    assert lib.LIB.qspec_gemm_w4a4(FAKE, 4, 256, FAKE, FAKE, 256, 64, FAKE, FAKE, 1 << 30, None,
+                                   0x80000000, None) == 1
+    assert lib.LIB.qspec_gemm_w4a16_noalloc(FAKE, 4, 256, FAKE, FAKE, 256, 64, FAKE, 4, None) == 1
 
 
 @pytest.mark.parametrize("b,g,v", [(0, 4, 32), (2, 0, 32), (2, 17, 32), (2, 4, 30), (2, 4, 0),

@@ -28,7 +28,7 @@ def qs():
 def _call_noalloc(qs, x, wq, ws, n, group, y):
     P = ctypes.c_void_p
     return qs.LIB.qspec_gemm_w4a16_noalloc(P(x.data_ptr()), x.shape[0], x.shape[1], P(wq.data_ptr()),
-                                           P(ws.data_ptr()), n, group, P(y.data_ptr()),
+                                           P(ws.data_ptr()), n, group, P(y.data_ptr()), 0,
                                            P(torch.cuda.current_stream().cuda_stream))
 
 
