@@ -21,29 +21,33 @@
 // n), the tokens are the MMA's N operand (MT columns, 16..128), so decode
 // batches of 1..128 tokens fill the instruction without padding to 128.
 //
-// Work decomposition: a unit is one 128-row weight tile x 128 input channels.
-// Units are ordered (n-tile, m-tile, k-chunk) and split evenly over a
-// persistent grid of CTAs (stream-K): every CTA gets the same number of
-// units +-1, whatever the shape.  A CTA that covers a whole tile writes y
-// directly; partial tiles go to workspace slots and the last CTA to finish a
-// tile (an atomic ticket, no waiting) adds the slots in K order, so results
-// are deterministic.  The ticket of a CTA's first split tile is taken by the
-// weight producer, so the epilogue goes straight on to the next tile.  A split tile starts inside exactly one CTA's range and
-// at most one split tile starts in any CTA's range, so the ticket of a tile
-// is indexed by its first contributor; tickets return to zero after use.
+// Work decomposition: a unit is one 128-row weight tile x 256 input channels
+// (int8 mode) or x 128 (bf16 mode).  Units are ordered (n-tile, m-tile,
+// k-chunk) and split evenly over a persistent grid of CTAs (stream-K): every
+// CTA gets the same number of units +-1, whatever the shape.  A CTA that
+// covers a whole tile writes y directly; partial tiles go to workspace slots
+// and the last CTA to finish a tile (an atomic ticket, no waiting) adds the
+// slots in K order, so results are deterministic.  The weight producer takes
+// the tickets, so the epilogue goes straight on to the next tile; when the
+// other contributor of the CTA's last tile has already published, the
+// epilogue adds its share directly.  A split tile starts inside exactly one
+// CTA's range and at most one split tile starts in any CTA's range, so the
+// ticket of a tile is indexed by its first contributor; tickets return to
+// zero after use.
 //
 // Warp roles (one CTA per SM):
-//   warp 0      TMA producer for packed weight tiles (ring of up to 16 x 8 KB)
+//   warp 0      TMA producer for packed weight tiles and group-scale tiles;
+//               split-tile tickets
 //   warp 1      TMA producer for activation tiles (128-byte swizzled ring)
 //   warps 2, 3  MMA issuers for even / odd units (warp 2 also owns the
-//               tensor-memory allocation); two issuers halve the exposed
-//               per-instruction issue latency of the small decode MMAs
-//   8 warps     converters: packed nibbles -> int8 / bf16 operand tiles
+//               tensor-memory allocation)
+//   4 or 8      converters (one team in int8 mode, two in bf16 mode): packed
+//   warps       nibbles -> int8 / bf16 operand tiles in tensor memory
 //   4..16 warps epilogue: tensor memory -> registers, group scales, output
 //
-// Three independent rings decouple the latencies: packed weights (HBM
-// latency), widened weights (converter -> tensor core) and activations (L2
-// latency); a 4-deep tensor-memory ring decouples the MMAs from the epilogue.
+// Rings decouple the latencies: packed weights (HBM latency), widened weights
+// (converter -> tensor core), activations (L2 latency), group scales, and the
+// per-group accumulators in tensor memory (MMA -> epilogue).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -58,9 +62,7 @@ constexpr int kTileN = 128;                      // weight rows per tile (MMA M)
 // Input channels per unit: 256 in int8 mode (16 KB of packed weights per
 // hand-off), 128 in bf16 mode (whose activation tiles are 4x larger).
 __host__ __device__ constexpr int unit_k(bool int8_mode) { return int8_mode ? 256 : 128; }
-constexpr int kConvWarps = 8;                    // two teams of four (one per lane quadrant)
-constexpr int kConvTeams = 2;                    // the teams take alternate units
-constexpr int kConvTeamWarps = kConvWarps / kConvTeams;
+constexpr int kConvTeamWarps = 4;                // a converter team: one warp per lane quadrant
 constexpr int kCtlWarps = 4;
 #ifdef QSPEC_TRACE
 constexpr int kSmemLimit = 232448 - 4096;        // trace builds keep 4 KB of static stamps
@@ -124,6 +126,11 @@ struct GemmCfg {
   static constexpr int kCols = MT / kTeams;                      // token columns per epilogue thread
   static_assert(kCols % 8 == 0, "epilogue columns must be a multiple of 8");
   static constexpr int kEpiThreads = 32 * kEpiWarps;
+  // Converter teams take alternate units: two in bf16 mode (13 integer/bf16
+  // ops per 8 weights), one in int8 mode (3), where a second team's warps
+  // cost the other roles more issue slots than they save.
+  static constexpr int kConvTeams = kInt8 ? 1 : 2;
+  static constexpr int kConvWarps = kConvTeamWarps * kConvTeams;
   static constexpr int kWarps = kCtlWarps + kConvWarps + kEpiWarps;
   static constexpr int kThreads = 32 * kWarps;
   static constexpr int kBarBytes = 1024;
@@ -592,9 +599,9 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     __syncwarp();
     mbar_wait_drain(smem_u32(mma_done), 0);
     __syncwarp();
-  } else if (warp >= kCtlWarps && warp < kCtlWarps + kConvWarps) {
+  } else if (warp >= kCtlWarps && warp < kCtlWarps + C::kConvWarps) {
     // ------------------------------------------------ converters
-    // Two teams of four warps (one per tensor-memory lane quadrant) take
+    // Teams of four warps (one per tensor-memory lane quadrant) take
     // alternate units.  Thread = weight row = tensor-memory lane: it reads the
     // row's packed bytes (int8 mode: 128 B, the TMA's 128-byte swizzle puts
     // 16-byte chunk c of row r at c ^ (r & 7); bf16 mode: 64 B, the 64-byte
@@ -612,7 +619,8 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     rp.init(cteam, NPK);
     ra.init(cteam, NA);
     for (long long u = u_begin + cteam; u < u_end;
-         u += kConvTeams, i += kConvTeams, rp.step(kConvTeams, NPK), ra.step(kConvTeams, NA)) {
+         u += C::kConvTeams, i += C::kConvTeams, rp.step(C::kConvTeams, NPK),
+         ra.step(C::kConvTeams, NA)) {
       const int sp = rp.slot;
       const int sa = ra.slot;
       bool ok = warp_wait(smem_u32(&pk_full[sp]), rp.phase, abort_flag, args.status);
@@ -682,9 +690,9 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       __syncwarp();
       if (quad == 0) QSPEC_STAMP(cteam == 0 ? 2 : 10, i);
     }
-  } else if (warp >= kCtlWarps + kConvWarps) {
+  } else if (warp >= kCtlWarps + C::kConvWarps) {
     // ------------------------------------------------ epilogue
-    const int ew = warp - (kCtlWarps + kConvWarps);
+    const int ew = warp - (kCtlWarps + C::kConvWarps);
     const int quad = warp & 3;                 // tensor-memory lanes this warp may read
     const int team = ew >> 2;                  // column team
     const int col0 = team * C::kCols;
@@ -888,7 +896,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   }
 
   QSPEC_TRACE_AT(0xFFF0);
-  if (warp >= kCtlWarps + kConvWarps && (threadIdx.x & 31) == 0 && warp == kCtlWarps + kConvWarps)
+  if ((threadIdx.x & 31) == 0 && warp == kCtlWarps + C::kConvWarps)
     QSPEC_PHASE(6);
   tc_fence_before();
   __syncthreads();
