@@ -65,20 +65,17 @@ __host__ __device__ constexpr int unit_k(bool int8_mode) { return int8_mode ? 25
 constexpr int kConvTeamWarps = 4;                // a converter team: one warp per lane quadrant
 constexpr int kCtlWarps = 4;
 #ifdef QSPEC_TRACE
-constexpr int kTraceSmem = 4096;                 // trace builds keep 4 KB of static stamps
+constexpr int kSmemLimit = 232448 - 4096;        // trace builds keep 4 KB of static stamps
 #else
-constexpr int kTraceSmem = 0;
+constexpr int kSmemLimit = 232448;               // sm_100 dynamic shared memory per CTA
 #endif
-constexpr int kSmemLimit = 232448 - kTraceSmem;  // sm_100 dynamic shared memory per CTA
-// ... with two CTAs per SM: half of the SM's 228 KB, less 1 KB reserved per CTA
-constexpr int kSmemLimitPair = 233472 / 2 - 1024 - kTraceSmem;
 constexpr int kMaxGrid = 1024;                   // ticket slots in the workspace
 constexpr int kMaxPk = 24, kMaxA = 8, kMaxAcc = 8, kMaxX = 8;
 // Group scales arrive by TMA, 8 groups x 128 rows (2 KB) per tile, into a ring.
 constexpr int kScaleTileGroups = 8;
 constexpr int kScaleTileBytes = kTileN * kScaleTileGroups * 2;
 constexpr int kNumSc = 8;
-constexpr int kTmemCols = 512;                   // all of tensor memory (shared by kPerSm CTAs)
+constexpr int kTmemCols = 512;                   // all of tensor memory: one CTA per SM
 // mbarriers (rings, MMA drain, scale tiles, split-tile hand-offs) and 8 words
 // of flags share a 1 KB block, in this order: pk_full, pk_empty, a_full,
 // a_empty, x_full, x_empty, acc_full, acc_empty, mma_done, sc_full, sc_empty,
@@ -106,15 +103,9 @@ __device__ __forceinline__ uint32_t bar_count(int b, int epi_warps) {
 __host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 __host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
 
-// kPerSm: CTAs sharing an SM (1, or 2 for the int8 16-token tile on shapes
-// with many units per CTA: each pipeline then waits on its hand-offs while
-// the other one works).  Two CTAs per SM get half of shared and tensor memory.
-template <bool kInt8, int MT, int kPerSm = 1>
+template <bool kInt8, int MT>
 struct GemmCfg {
   static_assert(MT % 16 == 0 && MT >= 16 && MT <= 128, "token tile must be 16..128, step 16");
-  static_assert(kPerSm == 1 || (kPerSm == 2 && kInt8 && MT == 16), "two CTAs per SM: int8, MT 16");
-  static constexpr int kCtaSmem = kPerSm == 2 ? kSmemLimitPair : kSmemLimit;
-  static constexpr int kTmem = kTmemCols / kPerSm;
   static constexpr int kUnitK = unit_k(kInt8);
   static constexpr int kPkBytes = kTileN * kUnitK / 2;           // packed bytes per unit
   static constexpr int kElem = kInt8 ? 1 : 2;                    // bytes per widened element
@@ -124,10 +115,9 @@ struct GemmCfg {
   // columns along K): 32 columns of int8 or 64 of bf16 per unit, then the
   // per-group accumulators (MT columns each) in what is left.
   static constexpr int kACols = kUnitK * kElem / 4;
-  static constexpr int kNumA =
-      kPerSm == 2 ? 3 : (kInt8 ? (MT <= 32 ? 6 : (MT <= 64 ? 4 : 2)) : 4);
+  static constexpr int kNumA = kInt8 ? (MT <= 32 ? 6 : (MT <= 64 ? 4 : 2)) : 4;
   static constexpr int kAccCol0 = kNumA * kACols;
-  static constexpr int kNumAcc = cmin(kMaxAcc, (kTmem - kAccCol0) / MT);
+  static constexpr int kNumAcc = cmin(kMaxAcc, (kTmemCols - kAccCol0) / MT);
   static_assert(kNumAcc >= 2, "tensor memory too small for two accumulators");
   static constexpr int kMmaK = kInt8 ? 32 : 16;
   static constexpr int kMmas = kUnitK / kMmaK;                   // MMAs per unit
@@ -147,13 +137,13 @@ struct GemmCfg {
   static constexpr int kScaleBytes = kNumSc * kScaleTileBytes;
   // Ring depths from the shared-memory budget: packed weights first (they
   // cover HBM latency), activations (an L2 hit) with what is left.
-  static constexpr int kAvail = kCtaSmem - 1024 - kBarBytes - kScaleBytes;
+  static constexpr int kAvail = kSmemLimit - 1024 - kBarBytes - kScaleBytes;
   static constexpr int kNumX = cmin(kMaxX, cmax(3, (kAvail - 128 * 1024) / kXBytes));
   static constexpr int kNumPk = cmin(kMaxPk, (kAvail - kNumX * kXBytes) / kPkBytes);
-  static_assert(kNumX >= 3 && kNumPk >= (kPerSm == 2 ? 4 : 6), "shared memory too small for the rings");
+  static_assert(kNumX >= 3 && kNumPk >= 6, "shared memory too small for the rings");
   static constexpr int kSmemBytes =
       1024 + kNumPk * kPkBytes + kNumX * kXBytes + kScaleBytes + kBarBytes;
-  static_assert(kSmemBytes <= kCtaSmem, "shared memory overflow");
+  static_assert(kSmemBytes <= kSmemLimit, "shared memory overflow");
 };
 
 struct GemmArgs {
@@ -294,12 +284,12 @@ __device__ __forceinline__ void st_release_cta(uint32_t* p, uint32_t v) {
 
 // kDbg (int8 mode only): also write the per-group integer accumulators.  A
 // separate instantiation keeps those stores out of the hot loop's code.
-template <bool kInt8, int MT, bool kDbg, int kPerSm>
-__global__ void __launch_bounds__(GemmCfg<kInt8, MT, kPerSm>::kThreads, kPerSm)
+template <bool kInt8, int MT, bool kDbg>
+__global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     qgemm_kernel(const __grid_constant__ CUtensorMap tmap_w,
                  const __grid_constant__ CUtensorMap tmap_x,
                  const __grid_constant__ CUtensorMap tmap_s, const __grid_constant__ GemmArgs args) {
-  using C = GemmCfg<kInt8, MT, kPerSm>;
+  using C = GemmCfg<kInt8, MT>;
   constexpr int NPK = C::kNumPk, NA = C::kNumA, NX = C::kNumX, NACC = C::kNumAcc;
   extern __shared__ uint8_t smem_raw[];
   QSPEC_STAMP_DECL
@@ -370,7 +360,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kPerSm>::kThreads, kPerSm)
     prefetch_tensormap(&tmap_s);
   }
   if (warp == 2) {
-    tmem_alloc(smem_u32(&misc[0]), C::kTmem);
+    tmem_alloc(smem_u32(&misc[0]), kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -915,7 +905,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kPerSm>::kThreads, kPerSm)
   QSPEC_STAMP_FLUSH();
   if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::kTmem);
+    tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 

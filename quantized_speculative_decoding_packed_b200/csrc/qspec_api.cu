@@ -103,7 +103,6 @@ struct GemmPlan {
   int m_tiles = 1, n_tiles = 1, ku = 1;
   long long units = 0;
   int grid = 1;
-  int per_sm = 1;            // CTAs sharing an SM (GemmCfg)
   size_t off_counters = 0, off_partials = 0, off_xq = 0, off_sa = 0, total = 0;
 };
 
@@ -131,15 +130,7 @@ GemmPlan plan_gemm(bool int8_mode, int64_t m, int64_t n, int64_t k, int sm_count
   const int uk = unit_k(int8_mode);
   p.ku = static_cast<int>((k + uk - 1) / uk);   // a last half unit reads zeros past k
   p.units = static_cast<long long>(p.m_tiles) * p.n_tiles * p.ku;
-  // Two CTAs per SM for the int8 16-token tile when every CTA still gets
-  // enough units that a weight tile has at most about four contributors
-  // (measured: faster on Llama-2-7B QKV and gate+up, slower where tiles
-  // would be split over ten CTAs).
-  const long long quarter_tile = (p.ku + 3) / 4;
-  const long long min_units = 2ll * sm_count * (quarter_tile > 4 ? quarter_tile : 4);
-  p.per_sm = (int8_mode && p.mt == 16 && p.units >= min_units) ? 2 : 1;
-  const int want = sm_count * p.per_sm;
-  const int max_grid = want < kMaxGrid ? want : kMaxGrid;
+  const int max_grid = sm_count < kMaxGrid ? sm_count : kMaxGrid;
   p.grid = static_cast<int>(p.units < max_grid ? p.units : max_grid);
   // Fixed-position regions first, so that calls of any shape sharing one
   // workspace never see each other's scratch data in their status word or
@@ -159,15 +150,14 @@ GemmPlan plan_gemm(bool int8_mode, int64_t m, int64_t n, int64_t k, int sm_count
   return p;
 }
 
-template <bool kInt8, int MT, bool kDbg, int kPerSm = 1>
+template <bool kInt8, int MT, bool kDbg>
 qspec_status launch_qgemm_t(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ts,
                             const GemmArgs& a,
                             int grid, int dev, cudaStream_t stream) {
-  using C = GemmCfg<kInt8, MT, kPerSm>;
+  using C = GemmCfg<kInt8, MT>;
   static bool attr_set[kMaxDevices] = {};
   if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(qgemm_kernel<kInt8, MT, kDbg, kPerSm>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(qgemm_kernel<kInt8, MT, kDbg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess) {
       cudaGetLastError();
       return QSPEC_ERR_CUDA;
@@ -188,7 +178,7 @@ qspec_status launch_qgemm_t(const CUtensorMap& tw, const CUtensorMap& tx, const 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, qgemm_kernel<kInt8, MT, kDbg, kPerSm>, tw, tx, ts, a) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, qgemm_kernel<kInt8, MT, kDbg>, tw, tx, ts, a) != cudaSuccess) {
     cudaGetLastError();
     return QSPEC_ERR_CUDA;
   }
@@ -196,17 +186,12 @@ qspec_status launch_qgemm_t(const CUtensorMap& tw, const CUtensorMap& tx, const 
 }
 
 template <bool kInt8>
-qspec_status launch_qgemm(int mt, int per_sm, const CUtensorMap& tw, const CUtensorMap& tx,
-                          const CUtensorMap& ts, const GemmArgs& a,
+qspec_status launch_qgemm(int mt, const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ts,
+                          const GemmArgs& a,
                           int grid, int dev, cudaStream_t stream) {
   const bool dbg = kInt8 && a.dbg_acc != nullptr;
   switch (mt) {
     case 16:
-      if constexpr (kInt8) {
-        if (per_sm == 2)
-          return dbg ? launch_qgemm_t<true, 16, true, 2>(tw, tx, ts, a, grid, dev, stream)
-                     : launch_qgemm_t<true, 16, false, 2>(tw, tx, ts, a, grid, dev, stream);
-      }
       return dbg ? launch_qgemm_t<kInt8, 16, kInt8>(tw, tx, ts, a, grid, dev, stream)
                  : launch_qgemm_t<kInt8, 16, false>(tw, tx, ts, a, grid, dev, stream);
     case 32:
@@ -312,7 +297,7 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
   if (!make_tmap(&ts, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, ws, n, scale_row_stride(k / group), kTileN, 8,
                  CU_TENSOR_MAP_SWIZZLE_NONE))
     return QSPEC_ERR_CUDA;
-  return launch_qgemm<kInt8>(p.mt, p.per_sm, tw, tx, ts, a, p.grid, dev, stream);
+  return launch_qgemm<kInt8>(p.mt, tw, tx, ts, a, p.grid, dev, stream);
 }
 
 }  // namespace
