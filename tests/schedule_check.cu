@@ -7,6 +7,11 @@
 //     CTA index can key the tile's ticket.
 //  3. The partial-slot rule agrees between writer and reducer: a CTA's
 //     segment in tile t is its first segment iff unit_begin(c) >= t * ku.
+//  4. The tail fast path (restating the kernel's prologue): a CTA whose last
+//     segment is a split tile that it opens, with the next CTA as the only
+//     other contributor, finds that CTA's share in its first-segment slot;
+//     the head hand-off and the tail are different tiles; and the weight
+//     producer's and the epilogue's notions of a split last segment agree.
 #include <cstdio>
 #include <cstdlib>
 #include <set>
@@ -60,6 +65,31 @@ int main() {
             const bool reducer_first = (b >= t0);
             if (writer_first != reducer_first) return fail("slot rule", units, grid, c);
           }
+        }
+        // 4. tail fast path and head hand-off, as the kernel computes them
+        for (long long c = 0; c < grid; ++c) {
+          const long long ub = unit_begin(c, units, grid), ue = unit_begin(c + 1, units, grid);
+          const long long t_tail = (ue - 1) / ku, tail_u0 = t_tail * ku;
+          const bool tail_split = !(ub <= tail_u0 && ue == tail_u0 + ku);
+          const bool tail_fast =
+              tail_split && ub <= tail_u0 && unit_owner(tail_u0 + ku - 1, units, grid) == c + 1;
+          // the epilogue's last segment [max(ub, tail_u0), ue) and its "full" test
+          const long long last_start = ub > tail_u0 ? ub : tail_u0;
+          const bool last_full = (last_start == tail_u0) && (ue == tail_u0 + ku);
+          if (last_full == tail_split) return fail("tail split rule", units, grid, c);
+          if (tail_fast) {
+            if (c + 1 >= grid) return fail("fast tail: no next CTA", units, grid, c);
+            const long long nb = ue, ne = unit_begin(c + 2, units, grid);
+            if (!(nb > tail_u0 && nb < tail_u0 + ku)) return fail("fast tail: next start", units, grid, c);
+            if (ne < tail_u0 + ku) return fail("fast tail: next ends early", units, grid, c);
+            // the next CTA's segment in the tile is its first one (slot 2 (c+1) + 0)
+            if (!(nb >= tail_u0)) return fail("fast tail: slot", units, grid, c);
+            if (unit_owner(tail_u0, units, grid) != c) return fail("fast tail: first contributor", units, grid, c);
+          }
+          const long long t_head = ub / ku, head_end = (ue < (t_head + 1) * ku) ? ue : (t_head + 1) * ku;
+          const bool head_handoff = head_end < ue && ub != t_head * ku;
+          if (head_handoff && tail_split && t_head == t_tail) return fail("head is tail", units, grid, c);
+          if (head_handoff && (ue - ub) < 2) return fail("head hand-off in one unit", units, grid, c);
         }
         ++checked;
       }
