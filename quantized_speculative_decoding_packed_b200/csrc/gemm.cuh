@@ -377,11 +377,11 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------ packed-weight producer
     // (the whole warp walks the loop; an elected lane issues the copies)
-    // This warp also takes the ticket of the CTA's first tile when that tile
-    // is split and more tiles follow (the epilogue handles a split last tile
-    // itself); it probes for the published share once per unit, having run
-    // far enough ahead that the ticket's latency costs the pipeline nothing,
-    // and leaves any reduction to the epilogue's many threads.
+    // This warp also takes the split tiles' tickets: the CTA's first tile's
+    // when its share is published (probed once per unit, far enough ahead
+    // that the ticket's latency costs the pipeline nothing), the last tile's
+    // after its loop (see below); any reduction is left to the epilogue's
+    // many threads.
     const long long t_head = static_cast<uint32_t>(u_begin) / static_cast<uint32_t>(ku);
     const long long head_end = (u_end < (t_head + 1) * ku) ? u_end : (t_head + 1) * ku;
     bool head_pending = (u_begin < u_end) && head_end < u_end && u_begin != t_head * ku;
