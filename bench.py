@@ -53,6 +53,8 @@ def parse():
                     help="decoder layers (32 = the full model; smaller only for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-large-m", action="store_true",
+                    help="skip the M = 2048 (Llama-2-70B-shaped) GEMM report")
     ap.add_argument("--profile-gemm", metavar="MODE:SHAPE", default=None,
                     help="profiling driver: three calls of one GEMM (MODE w4a4|w4a16, SHAPE "
                          "qkv|o_proj|gate_up|down of the workload) on seeded weights, then exit")
@@ -458,6 +460,10 @@ def main():
         cpu = {"value": bytes_step / t_cpu / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
                "sample": desc}
 
+    large = None
+    if rank == 0 and world == 1 and not args.no_large_m:
+        large = large_m_report(torch, qspec, peaks)
+
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -467,11 +473,55 @@ def main():
                 "tops": world * ops_step / (ms_step * 1e-3) / 1e12,
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps,
-                "clocks": clk.summary(), "kernels": kern}
+                "clocks": clk.summary(), "kernels": kern, "large_m": large}
         print(json.dumps(line))
     if world > 1:
         del graph
         dist.destroy_process_group()
+
+
+LARGE_M = 2048
+LARGE_SHAPES = (("qkv", 10240, 8192), ("gate_up", 57344, 8192), ("down", 8192, 28672))
+
+
+def large_m_report(torch, qspec, peaks):
+    """Llama-2-70B-shaped GEMMs at M = 2048 in both modes, each timed alone (one warm-up
+    call, then 3 calls between CUDA events on the launching stream), against the dense
+    tensor peaks: bf16 = the measured burst figure, int8 = twice it (nominal ratio)."""
+    bf16 = float(peaks.get("bf16_tflops", 1590.0))
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(rank_seed(0) + 7)
+    shapes = {}
+    for name, n, k in LARGE_SHAPES:
+        w = torch.randn((n, k), generator=gen, device="cuda", dtype=torch.float32) * 0.02
+        wq, ws = qspec.quantize_weights(w, GROUP)
+        del w
+        x = torch.randn((LARGE_M, k), generator=gen, device="cuda").to(torch.bfloat16)
+        y = torch.empty((LARGE_M, n), dtype=torch.float32, device="cuda")
+        for mode in ("w4a4", "w4a16"):
+            fn = qspec.gemm_w4a4 if mode == "w4a4" else qspec.gemm_w4a16
+            op = qspec.OP_GEMM_W4A4 if mode == "w4a4" else qspec.OP_GEMM_W4A16
+            work = qspec.workspace(qspec.workspace_size(op, LARGE_M, n, k, GROUP))
+            fn(x, wq, ws, GROUP, y=y, work=work, weights_ready=True)
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(3):
+                fn(x, wq, ws, GROUP, y=y, work=work, weights_ready=True)
+            e1.record()
+            e1.synchronize()
+            t = e0.elapsed_time(e1) / 3 * 1e-3
+            tops = 2.0 * LARGE_M * n * k / t / 1e12
+            peak = bf16 * (2.0 if mode == "w4a4" else 1.0)
+            shapes[f"{name}_{mode}"] = {"n": n, "k": k, "us": t * 1e6, "tops": tops,
+                                        "frac": tops / peak}
+        del wq, ws, x, y
+    torch.cuda.empty_cache()
+    return {"m": LARGE_M, "bound": "tensor", "peak_bf16_tflops": bf16, "peak_int8_tops": 2 * bf16,
+            "peak_source": "MEASURED_PEAKS.json bf16_tflops (burst, measured); int8 = 2x"
+            if "bf16_tflops" in peaks else "fallback 1590 TFLOP/s; int8 = 2x",
+            "shapes": shapes}
 
 
 def measure_e2e(torch, stream, graph, acts, accept_in, outs, steps, bytes_step):
