@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -155,14 +156,15 @@ qspec_status launch_qgemm_t(const CUtensorMap& tw, const CUtensorMap& tx, const 
                             const GemmArgs& a,
                             int grid, int dev, cudaStream_t stream) {
   using C = GemmCfg<kInt8, MT>;
-  static bool attr_set[kMaxDevices] = {};
-  if (!attr_set[dev]) {
+  // Set once per device; concurrent first calls may both set it (idempotent).
+  static std::atomic<bool> attr_set[kMaxDevices];
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(qgemm_kernel<kInt8, MT, kDbg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess) {
       cudaGetLastError();
       return QSPEC_ERR_CUDA;
     }
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
@@ -388,14 +390,14 @@ qspec_status qspec_spec_accept(const float* p, const float* q, const int32_t* dr
   if (st != QSPEC_OK) return st;
   const int chunk = ((vocab + 4 * kAcceptCluster - 1) / (4 * kAcceptCluster)) * 4;
   const size_t smem = static_cast<size_t>(chunk) * 4;
-  static bool attr_set[kMaxDevices] = {};
-  if (!attr_set[dev]) {
+  static std::atomic<bool> attr_set[kMaxDevices];   // as for the GEMM kernels
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(spec_accept_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              204800) != cudaSuccess) {
       cudaGetLastError();
       return QSPEC_ERR_CUDA;
     }
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   spec_accept_kernel<<<batch * kAcceptCluster, kAcceptThreads, smem,
                        static_cast<cudaStream_t>(stream)>>>(
