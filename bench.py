@@ -55,6 +55,10 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-large-m", action="store_true",
                     help="skip the M = 2048 (Llama-2-70B-shaped) GEMM report")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the Llama-3-8B-shaped M sweep report")
+    ap.add_argument("--no-accept-report", action="store_true",
+                    help="skip the vocab-128256 accept/resample report")
     ap.add_argument("--profile-gemm", metavar="MODE:SHAPE", default=None,
                     help="profiling driver: three calls of one GEMM (MODE w4a4|w4a16, SHAPE "
                          "qkv|o_proj|gate_up|down of the workload) on seeded weights, then exit")
@@ -193,6 +197,63 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- CPU oracle sample
+def _oracle_shape_job(job):
+    """Oracle time of one layer shape on `c` sampled columns, both modes (one thread)."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import qspec_oracle as orc
+    from quantized_speculative_decoding_packed_b200 import synth
+    si, n, k, c, seed = job
+    with threadpool_limits(limits=1):
+        rng = synth.rng_for("llama2_7b", 50 + seed, si, c)
+        w = synth.weights(rng, c, k)
+        outl = synth.outlier_channels(synth.rng_for("llama2_7b", 2, k), k)
+        x16 = synth.bf16_bits_to_f32(synth.activations(rng, M_DRAFT, k, outl))
+        x80 = synth.bf16_bits_to_f32(synth.activations(rng, M_VERIFY, k, outl))
+        q, s_h = orc.quantize_weights(w, GROUP)
+        t0 = time.perf_counter()
+        orc.gemm_w4a4(x16, q, s_h, GROUP)
+        t1 = time.perf_counter()
+        orc.gemm_w4a16(x80, q, s_h, GROUP)
+        t2 = time.perf_counter()
+    return si, t1 - t0, t2 - t1
+
+
+def oracle_sample_all_cores(columns=2048, seed=0):
+    """The same sample as oracle_sample, split into column blocks run by a spawn
+    pool of single-threaded processes, one per host core.  The blocks' own
+    times add up to the single-thread step time (scaled exactly as in
+    oracle_sample); the pool's wall time against that sum is the measured
+    speed-up, and the step time on all cores is the single-thread time over it."""
+    import multiprocessing as mp
+    cores = os.cpu_count() or 1
+    jobs = []
+    for si, (name, n, k) in enumerate(LAYERS):
+        c = min(columns, n)
+        per = max(1, -(-c // cores))
+        for j in range(0, c, per):
+            jobs.append((si, n, k, min(per, c - j), seed + 7 * j))
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(cores) as pool:
+        pool.map(_oracle_shape_job, [(0, 256, 256, 1, 0)] * cores)   # start and warm the workers
+        t0 = time.perf_counter()
+        res = pool.map(_oracle_shape_job, jobs)
+        wall = time.perf_counter() - t0
+    busy = sum(t4 + t16 for (_, t4, t16) in res)
+    t_single = 0.0
+    for si, (name, n, k) in enumerate(LAYERS):
+        t4 = sum(r[1] for r in res if r[0] == si)
+        t16 = sum(r[2] for r in res if r[0] == si)
+        t_single += N_LAYERS * (n / min(columns, n)) * (GAMMA * t4 + t16)
+    speedup = busy / wall
+    desc = (f"oracle on {columns} output columns of each of the 4 layer shapes (W4A4 at M=16, "
+            f"W4A16 at M=80), split into {len(jobs)} column blocks over a spawn pool of {cores} "
+            f"single-threaded processes; single-thread step time (blocks' own times scaled by "
+            f"N/{columns} x 32 layers x ({GAMMA} draft + 1 verify passes)) divided by the "
+            f"measured pool speed-up {speedup:.2f}; accept step excluded")
+    return t_single / speedup, desc, cores
+
+
 def oracle_sample(columns=2048, seed=0):
     """Time the oracle on `columns` output columns of every layer shape (both
     modes) plus the full accept step; return (seconds per full step scaled
@@ -222,11 +283,12 @@ def oracle_sample(columns=2048, seed=0):
         ai = synth.accept_inputs(synth.rng_for("llama2_7b", 60 + seed), BATCH, GAMMA, VOCAB, 2.0, 0.5)
         t0 = time.perf_counter()
         n_acc, _ = orc.spec_accept(ai.p, ai.q, ai.draft, ai.u_acc, ai.u_res)
-        t_step += time.perf_counter() - t0
+        t_accept = time.perf_counter() - t0
+        t_step += t_accept
     desc = (f"oracle on {columns} output columns of each of the 4 layer shapes (W4A4 at M=16, "
-            f"W4A16 at M=80) plus the full accept step, scaled by N/{columns} x 32 layers x "
-            f"({GAMMA}+1) passes; single thread")
-    return t_step, desc, n_acc
+            f"W4A16 at M=80) plus the full accept step, extrapolated to the step by N/{columns} x "
+            f"32 layers x ({GAMMA} draft + 1 verify) passes; single thread")
+    return t_step, desc, n_acc, t_accept
 
 
 # ---------------------------------------------------------------- reference arm
@@ -237,7 +299,7 @@ def run_reference(args, rank, world):
     times = []
     n_acc = None
     for i in range(args.warmup + args.steps):
-        t, desc, n_acc = oracle_sample(columns=256, seed=i)
+        t, desc, n_acc, _ = oracle_sample(columns=256, seed=i)
         if i >= args.warmup:
             times.append(t)
     acc_b = accept_bytes(n_acc, GAMMA, VOCAB)
@@ -245,6 +307,8 @@ def run_reference(args, rank, world):
     value = (bytes_step + acc_b) / t / 1e9
     line = {"metric": METRIC, "value": value, "unit": "GB/s", "impl": "reference", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+            "ms_per_step_note": "extrapolated from each step's 256-column sample of every layer "
+                                "shape (x N/256 x 32 layers x 5 passes); the run itself is short",
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64/f64",
             "data": "synthetic", "config": workload_config(N_LAYERS),
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
@@ -456,13 +520,23 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t_cpu, desc, _ = oracle_sample()
-        cpu = {"value": bytes_step / t_cpu / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": desc}
+        t_cpu, desc, _, t_acc_cpu = oracle_sample()
+        t_all, desc_all, cores = oracle_sample_all_cores()
+        t_all += t_acc_cpu
+        cpu = {"value": bytes_step / t_all / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": desc_all + "; plus the accept step on one thread",
+               "single_thread": {"value": bytes_step / t_cpu / 1e9, "unit": "GB/s", "cores": 1,
+                                 "sample": desc}}
 
     large = None
     if rank == 0 and world == 1 and not args.no_large_m:
         large = large_m_report(torch, qspec, peaks)
+    sweep = None
+    if rank == 0 and world == 1 and not args.no_sweep:
+        sweep = m_sweep_report(torch, qspec, peaks)
+    acc_rep = None
+    if rank == 0 and world == 1 and not args.no_accept_report:
+        acc_rep = accept_report(torch, qspec, peaks)
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
@@ -473,7 +547,8 @@ def main():
                 "tops": world * ops_step / (ms_step * 1e-3) / 1e12,
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps,
-                "clocks": clk.summary(), "kernels": kern, "large_m": large}
+                "clocks": clk.summary(), "kernels": kern, "large_m": large,
+                "m_sweep": sweep, "accept_large_vocab": acc_rep}
         print(json.dumps(line))
     if world > 1:
         del graph
@@ -522,6 +597,157 @@ def large_m_report(torch, qspec, peaks):
             "peak_source": "MEASURED_PEAKS.json bf16_tflops (burst, measured); int8 = 2x"
             if "bf16_tflops" in peaks else "fallback 1590 TFLOP/s; int8 = 2x",
             "shapes": shapes}
+
+
+SWEEP_SHAPES = (("qkv", 6144, 4096), ("o_proj", 4096, 4096), ("gate_up", 28672, 4096),
+                ("down", 4096, 14336))
+SWEEP_M = (1, 8, 32, 128, 256)
+
+
+def _graph_time_per_call(torch, calls, reps=5):
+    """Device time per call of a CUDA graph of `calls` (a list of thunks), median of reps."""
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        for c in calls:
+            c()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for c in calls:
+                c()
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1) / len(calls) * 1e-3)
+    del graph
+    return statistics.median(ts)
+
+
+def m_sweep_report(torch, qspec, peaks):
+    """Llama-3-8B-shaped GEMMs (GQA: fused QKV 6144) at M in {1, 8, 32, 128, 256}, both
+    modes: device time per call in a CUDA graph of back-to-back calls whose weights
+    rotate over copies that together exceed the L2 three times (weights streamed from
+    HBM), with QSPEC_GEMM_WEIGHTS_READY.  Reported against both bounds: packed bytes
+    over the measured HBM bandwidth, and 2MNK over the dense tensor peak (bf16 = the
+    measured burst figure; int8 = twice it); `bound` names the larger time."""
+    hbm = float(peaks.get("hbm_gbs", 6650.0))
+    bf16 = float(peaks.get("bf16_tflops", 1590.0))
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(rank_seed(0) + 11)
+    out = {}
+    for name, n, k in SWEEP_SHAPES:
+        pb = packed_bytes(n, k)
+        copies = max(2, -(-3 * 126 * 2 ** 20 // pb))
+        wqs = []
+        for _ in range(copies):
+            w = torch.randn((n, k), generator=gen, device="cuda", dtype=torch.float32) * 0.02
+            wqs.append(qspec.quantize_weights(w, GROUP))
+            del w
+        for m in SWEEP_M:
+            x = torch.randn((m, k), generator=gen, device="cuda").to(torch.bfloat16)
+            y = torch.empty((m, n), dtype=torch.float32, device="cuda")
+            for mode in ("w4a4", "w4a16"):
+                fn = qspec.gemm_w4a4 if mode == "w4a4" else qspec.gemm_w4a16
+                op = qspec.OP_GEMM_W4A4 if mode == "w4a4" else qspec.OP_GEMM_W4A16
+                work = torch.zeros(qspec.workspace_size(op, m, n, k, GROUP), dtype=torch.uint8,
+                                   device="cuda")
+                calls = [(lambda c=c: fn(x, wqs[c][0], wqs[c][1], GROUP, y=y, work=work,
+                                         weights_ready=True)) for c in range(copies)] * 2
+                t = _graph_time_per_call(torch, calls)
+                peak = bf16 * (2.0 if mode == "w4a4" else 1.0)
+                t_hbm = gemm_bytes(m, n, k, mode) / (hbm * 1e9)
+                t_tc = 2.0 * m * n * k / (peak * 1e12)
+                out[f"{name}_m{m}_{mode}"] = {
+                    "n": n, "k": k, "m": m, "us": t * 1e6, "packed_gbs": pb / t / 1e9,
+                    "tops": 2.0 * m * n * k / t / 1e12,
+                    "frac_hbm": t_hbm / t, "frac_tensor": t_tc / t,
+                    "bound": "hbm" if t_hbm >= t_tc else "tensor"}
+            del x, y
+        del wqs
+        torch.cuda.empty_cache()
+    return {"workload": "Llama-3-8B-shaped GEMMs (GQA 32/8 heads), group 128",
+            "timing": "CUDA graph of back-to-back calls, weights rotating past L2 (3x L2)",
+            "peak_hbm_gbs": hbm, "peak_bf16_tflops": bf16, "peak_int8_tops": 2 * bf16,
+            "frac": "roofline time / measured time for each bound (frac_hbm uses all compulsory "
+                    "bytes: packed weights, scales, activations, output)",
+            "shapes": out}
+
+
+def accept_report(torch, qspec, peaks, sigmas=(0.1, 0.5, 1.0), batch=64, gamma=5, vocab=128256):
+    """The accept / residual-resample step at vocab 128256, batch 64, gamma 5, once per
+    draft-noise sigma: target logits N(0, 2^2), draft logits = target + N(0, sigma^2),
+    seeded; each call timed alone between CUDA events with the L2 flushed before it.
+    Algorithmic bytes come from the measured accepted lengths.  near_ties counts tested
+    positions whose uniform lies within 1e-6 of p/q (where a rounding difference could
+    flip the decision)."""
+    hbm = float(peaks.get("hbm_gbs", 6650.0))
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(rank_seed(0) + 13)
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device="cuda")
+    work = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    out = {}
+    for sigma in sigmas:
+        lp = torch.randn((batch, gamma + 1, vocab), generator=gen, device="cuda",
+                         dtype=torch.float64) * 2.0
+        lq = lp[:, :gamma] + torch.randn((batch, gamma, vocab), generator=gen, device="cuda",
+                                         dtype=torch.float64) * sigma
+        p = torch.softmax(lp, -1).float().contiguous()
+        q = torch.softmax(lq, -1).float().contiguous()
+        del lp, lq
+        draft = torch.multinomial(q.reshape(-1, vocab).double(), 1, generator=gen).reshape(
+            batch, gamma).to(torch.int32)
+        u_acc = (torch.randint(0, 1 << 24, (batch, gamma), generator=gen, device="cuda").double()
+                 / (1 << 24)).float()
+        u_res = (torch.randint(0, 1 << 24, (batch,), generator=gen, device="cuda").double()
+                 / (1 << 24)).float()
+        n_acc = torch.empty((batch,), dtype=torch.int32, device="cuda")
+        tokens = torch.empty((batch, gamma + 1), dtype=torch.int32, device="cuda")
+        ts = []
+        for rep in range(8):
+            flush.fill_(rep & 0xFF)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            qspec.spec_accept(p, q, draft, u_acc, u_res, n_accepted=n_acc, tokens=tokens, work=work)
+            e1.record()
+            e1.synchronize()
+            if rep >= 2:
+                ts.append(e0.elapsed_time(e1) * 1e-3)
+        if qspec.workspace_status(work) != 0:
+            raise RuntimeError("accept kernel reported bad input")
+        t = statistics.median(ts)
+        na = n_acc.cpu().numpy()
+        byts = accept_bytes(na, gamma, vocab)
+        # near-tie count over the positions the rule tested
+        idx = draft.long().unsqueeze(-1)
+        pv = p[:, :gamma].gather(2, idx).squeeze(-1).double()
+        qv = q.gather(2, idx).squeeze(-1).double()
+        tested = torch.arange(gamma, device="cuda")[None, :] <= n_acc[:, None].long().clamp(max=gamma - 1)
+        near = ((u_acc.double() - pv / qv).abs() < 1e-6) & tested
+        out[f"sigma_{sigma}"] = {"us": t * 1e6, "bytes": byts, "gbs": byts / t / 1e9,
+                                 "frac_hbm": byts / t / 1e9 / hbm,
+                                 "mean_accepted": float(na.mean()),
+                                 "acceptance_per_position": float(
+                                     (na.sum()) / (na.sum() + (na < gamma).sum())),
+                                 "near_ties": int(near.sum())}
+        del p, q
+    del flush
+    torch.cuda.empty_cache()
+    return {"workload": f"accept/resample, vocab {vocab}, batch {batch}, gamma {gamma}, "
+                        "target logits N(0, 2^2), draft = target + N(0, sigma^2)",
+            "timing": "each call alone between CUDA events, L2 flushed (256 MB write) before it",
+            "bytes": "per sequence: 2 gathered elements per tested position + one vocab row of p "
+                     "and q (rejection) or of p (all accepted) + outputs",
+            "peak_hbm_gbs": hbm, "sigmas": out}
 
 
 def measure_e2e(torch, stream, graph, acts, accept_in, outs, steps, bytes_step):

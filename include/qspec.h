@@ -65,6 +65,17 @@ typedef enum qspec_status {
  * Other bits are reserved and must be zero.
  */
 #define QSPEC_GEMM_WEIGHTS_READY 1u
+/*
+ *  QSPEC_GEMM_TEST_STALL: a test hook for the failure path, not for normal
+ *    use.  The GEMM's weight producer first waits, for 10 ms at most, on a
+ *    barrier that nothing signals; the wait runs out and every CTA gives up
+ *    exactly as on a real stall: it raises its abort flag, sets the device
+ *    status word, stops every role at its next wait, lets the copies it has
+ *    issued land, frees its tensor memory and returns.  `y` is left
+ *    incomplete; qspec_workspace_status() then returns QSPEC_ERR_TIMEOUT and
+ *    readies the workspace for the next call.
+ */
+#define QSPEC_GEMM_TEST_STALL 0x100u
 
 /* Operation ids for qspec_workspace_size(). */
 enum {
@@ -179,21 +190,27 @@ qspec_status qspec_spec_accept(const float* p, const float* q, const int32_t* dr
 /*
  * W4A16 verifying GEMM that allocates nothing and takes no workspace.
  * The pages have no counterpart to this entry point; it exists for callers
- * that cannot allocate device memory at the point of the call -- e.g. code
- * running where the CUDA runtime may not be entered to allocate, such as a
- * host function enqueued with cudaLaunchHostFunc, or a plugin hosted by an
- * application that owns all device memory and permits no allocation outside
- * its own pools.
+ * that cannot allocate device memory at the point of the call: a plugin
+ * hosted by an application that owns all device memory and permits no
+ * allocation outside its own pools, or a latency-critical path that must not
+ * enter the allocator (cudaMalloc/cudaFree may synchronise the device).
+ * Call it from ordinary host code: CUDA forbids CUDA calls inside a host
+ * function enqueued on a stream, and this entry point makes several.
  * Computes exactly what qspec_gemm_w4a16 computes, with its scratch held in a
  * file-scope device array of QSPEC_STATIC_SCRATCH_BYTES (16 MiB) that every
  * GPU loading this library keeps until the process exits.
  *  - The first call on a device looks up the array's device address (with
- *    that device current) and caches it; make that first call before any
- *    stream capture.
+ *    that device current) and keeps it for the life of the process; make
+ *    that first call before any stream capture, and do not use this entry
+ *    point on a device after cudaDeviceReset() on it.
  *  - Every call shares the one array: calls that overlap on the GPU (on
  *    different streams, or from different threads) race and must not be
- *    issued.  Each call clears the status word and split-tile tickets with an
- *    asynchronous memset on `stream`; nothing else needs to start at zero.
+ *    issued.  Each call clears the split-tile tickets with an asynchronous
+ *    memset on `stream` (so the GEMM cannot start streaming weights before
+ *    the preceding kernel ends, as it can on the workspace path); nothing
+ *    else needs to start at zero.
+ *  - Device faults (a wait that ran out) are recorded in the array's status
+ *    word, which stays set until qspec_gemm_w4a16_noalloc_status() reads it.
  *  - Shapes whose scratch would exceed the array (for example m > 96 on a
  *    148-SM B200) return QSPEC_ERR_WORKSPACE_TOO_SMALL and launch nothing.
  *  - Calls no cudaMalloc, cudaFree or other allocating routine.
@@ -204,6 +221,15 @@ qspec_status qspec_gemm_w4a16_noalloc(const uint16_t* x, int64_t m, int64_t k, c
                                       const uint16_t* ws, int64_t n, int32_t group, float* y,
                                       uint32_t flags, void* stream);
 
+/*
+ * Device status of qspec_gemm_w4a16_noalloc on the current device, without
+ * allocating: synchronizes `stream`, reads the built-in array's status word,
+ * clears it (and, after a timeout, the split-tile tickets) and returns
+ * QSPEC_OK, QSPEC_ERR_TIMEOUT or QSPEC_ERR_BAD_INPUT (QSPEC_ERR_CUDA if the
+ * read failed).  QSPEC_OK if no such call has run on the device.
+ */
+qspec_status qspec_gemm_w4a16_noalloc_status(void* stream);
+
 /* Bytes of workspace an operation needs on the current device (0 = none).
  * Unused size arguments are ignored.  Returns 0 for invalid arguments too. */
 size_t qspec_workspace_size(int32_t op, int64_t m, int64_t n, int64_t k, int32_t group,
@@ -211,11 +237,15 @@ size_t qspec_workspace_size(int32_t op, int64_t m, int64_t n, int64_t k, int32_t
 
 /* Synchronizes `stream`, reads the device status word at the start of
  * `workspace`, clears it, and returns QSPEC_OK, QSPEC_ERR_TIMEOUT or
- * QSPEC_ERR_BAD_INPUT (or QSPEC_ERR_CUDA if the read itself failed). */
+ * QSPEC_ERR_BAD_INPUT (or QSPEC_ERR_CUDA if the read itself failed).  After
+ * a timeout (which only a GEMM reports) it also clears the split-tile
+ * tickets the stopped call may have left taken, so the workspace is ready
+ * for the next call. */
 qspec_status qspec_workspace_status(void* workspace, void* stream);
 
-/* Version of this ABI (2: the GEMM entry points take `flags`). */
-#define QSPEC_ABI_VERSION 2
+/* Version of this ABI (3: adds QSPEC_GEMM_TEST_STALL and
+ * qspec_gemm_w4a16_noalloc_status). */
+#define QSPEC_ABI_VERSION 3
 int32_t qspec_abi_version(void);
 
 /* Static, human-readable name of a status code. */

@@ -172,12 +172,12 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 // The slow path lives out of line: the hot loops keep one try_wait and a
 // branch, and their code stays compact in the instruction caches.
 __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                            uint32_t* status) {
+                                            uint32_t* status, uint64_t limit_ns = kWaitLimitNs) {
   const uint64_t start = global_timer_ns();
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;   // sleeps <= 0.2 ms
     if (*abort_flag) return false;
-    if (global_timer_ns() - start > kWaitLimitNs) {
+    if (global_timer_ns() - start > limit_ns) {
       *abort_flag = 1;
       if (status) atomicOr(status, kDevTimeout);
       return false;
@@ -282,24 +282,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int n) {
   return (1u << 4)                  // D: f32
          | (1u << 7) | (1u << 10)   // A, B: bf16
          | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
-}
-
-template <bool kInt8>
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-  if constexpr (kInt8) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-  } else {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-  }
 }
 
 // Arrives on `bar` once all previously issued tcgen05.mma of this thread complete.

@@ -79,14 +79,15 @@ constexpr int kTmemCols = 512;                   // all of tensor memory: one CT
 // mbarriers (rings, MMA drain, scale tiles, split-tile hand-offs) and 8 words
 // of flags share a 1 KB block, in this order: pk_full, pk_empty, a_full,
 // a_empty, x_full, x_empty, acc_full, acc_empty, mma_done, sc_full, sc_empty,
-// flush[2], ticket[2], tail.
+// flush[2], ticket[2], tail, stall.
 namespace bar {
 constexpr int kPkFull = 0, kPkEmpty = kPkFull + kMaxPk, kAFull = kPkEmpty + kMaxPk;
 constexpr int kAEmpty = kAFull + kMaxA, kXFull = kAEmpty + kMaxA, kXEmpty = kXFull + kMaxX;
 constexpr int kAccFull = kXEmpty + kMaxX, kAccEmpty = kAccFull + kMaxAcc;
 constexpr int kMmaDone = kAccEmpty + kMaxAcc, kScFull = kMmaDone + 1, kScEmpty = kScFull + kNumSc;
 constexpr int kFlush = kScEmpty + kNumSc, kTicket = kFlush + 2, kTail = kTicket + 2;
-constexpr int kCount = kTail + 1;
+constexpr int kStall = kTail + 1;   // never signalled: the test hook's wait
+constexpr int kCount = kStall + 1;
 }  // namespace bar
 constexpr int kNumBars = bar::kCount;
 static_assert(kNumBars * 8 + 8 * 4 <= 1024, "barrier block overflow");
@@ -153,6 +154,8 @@ struct GemmArgs {
   int m_tiles, n_tiles, ku;
   long long units;         // m_tiles * n_tiles * ku
   int weights_ready;       // wq/ws may be read before the preceding grid completes
+  uint32_t test_stall_ns;  // test hook (0 = off): the weight producer first waits this
+                           // long on a barrier that nothing signals, then gives up
   const uint16_t* ws;      // fp16 scales [N][K/group]
   const float* s_a;        // W4A4: per-token scales [M]
   float* y;                // [M][N]
@@ -391,6 +394,13 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     if constexpr (!kInt8) {
       if (!args.weights_ready) grid_dependency_wait();
     }
+    // Test hook: a wait that nothing completes runs out, and the CTA gives up
+    // as it would on a real stall (abort flag, device status, every role
+    // stops at its next wait, copies in flight are drained).
+    bool run = true;
+    if (args.test_stall_ns != 0u)
+      run = __all_sync(0xffffffffu, mbar_wait_slow(smem_u32(bars + bar::kStall), 0, abort_flag,
+                                                   args.status, args.test_stall_ns));
     // Group scales: one TMA tile (8 groups x 128 rows) whenever a unit starts a
     // new run of 8 groups of its tile, or is this CTA's first unit; the
     // epilogue walks the same sequence.
@@ -403,7 +413,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     int i = 0;
     UnitCursor cur;
     cur.init(u_begin, ku, args.m_tiles);
-    for (long long u = u_begin; u < u_end; ++u, ++i, cur.next(ku, args.m_tiles)) {
+    for (long long u = u_begin; run && u < u_end; ++u, ++i, cur.next(ku, args.m_tiles)) {
       const int s = i % NPK;
       const uint32_t ph = (i / NPK) & 1;
       QSPEC_STAMP(13, i);

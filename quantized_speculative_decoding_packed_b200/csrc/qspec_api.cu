@@ -99,6 +99,10 @@ bool make_tmap(CUtensorMap* map, CUtensorMapDataType dtype, size_t elem, const v
 }
 
 // ---------------------------------------------------------------- GEMM planning
+// Every GEMM workspace starts with a 256-byte status block and the split-tile
+// tickets, at fixed offsets.
+constexpr size_t kStatusAndTicketBytes = 256 + static_cast<size_t>(kMaxGrid) * 4;
+
 struct GemmPlan {
   int mt = 16;               // token tile (MMA N)
   int m_tiles = 1, n_tiles = 1, ku = 1;
@@ -223,7 +227,7 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
                       const uint16_t* ws, int64_t n, int32_t group, float* y, void* workspace,
                       size_t workspace_bytes, int32_t* dbg_acc, uint32_t flags, void* stream_v) {
   if (!x || !wq || !ws || !y || !workspace) return QSPEC_ERR_INVALID_ARG;
-  if ((flags & ~QSPEC_GEMM_WEIGHTS_READY) != 0u) return QSPEC_ERR_INVALID_ARG;
+  if ((flags & ~(QSPEC_GEMM_WEIGHTS_READY | QSPEC_GEMM_TEST_STALL)) != 0u) return QSPEC_ERR_INVALID_ARG;
   const bool weights_ready = (flags & QSPEC_GEMM_WEIGHTS_READY) != 0u;
   if (!gemm_shape_ok(m, n, k, group)) return QSPEC_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(wq, 16) || !aligned(ws, 16) || !aligned(y, 4) ||
@@ -256,6 +260,7 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
   a.ku = p.ku;
   a.units = p.units;
   a.weights_ready = weights_ready ? 1 : 0;
+  a.test_stall_ns = (flags & QSPEC_GEMM_TEST_STALL) ? 10u * 1000u * 1000u : 0u;   // 10 ms
   a.ws = ws;
   a.y = y;
   a.dbg_acc = dbg_acc;
@@ -439,7 +444,13 @@ qspec_status qspec_workspace_status(void* workspace, void* stream) {
     return QSPEC_ERR_CUDA;
   }
   if (word == 0) return QSPEC_OK;
-  if (cudaMemsetAsync(workspace, 0, 4, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess) {
+  // A GEMM that gave up (the only kernels that time out) may have left
+  // split-tile tickets taken: clear them with the status word, so that the
+  // workspace is ready for the next call.  An accept workspace (256 bytes)
+  // only ever receives BAD_INPUT.
+  const size_t clear = (word & kDevTimeout) ? kStatusAndTicketBytes : 4;
+  if (cudaMemsetAsync(workspace, 0, clear, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
     cudaGetLastError();
     return QSPEC_ERR_CUDA;
   }
@@ -447,17 +458,34 @@ qspec_status qspec_workspace_status(void* workspace, void* stream) {
 }
 
 // ---------------------------------------------------------------- no-allocation variant
-// Built-in scratch for callers that cannot allocate device memory: code that
-// runs where the CUDA runtime may not be entered to allocate (for example a
-// host function enqueued with cudaLaunchHostFunc), or a plugin inside a host
-// application that owns all device memory and allows no allocation beyond
-// its own pools.  Every GPU that loads this library holds the array until
-// the process exits.
+// Built-in scratch for callers that cannot allocate device memory: a plugin
+// inside a host application that owns all device memory and allows no
+// allocation outside its own pools, or code that must not enter the
+// allocator at the point of the call (real-time paths that forbid the
+// implicit synchronisation cudaMalloc/cudaFree may cause).  Every GPU that
+// loads this library holds the array until the process exits; it starts
+// zero-filled.
 static __device__ __align__(256) unsigned char g_qspec_static_scratch[QSPEC_STATIC_SCRATCH_BYTES];
 
 namespace {
 void* g_static_scratch_ptr[kMaxDevices] = {};
 std::mutex g_static_scratch_mutex;
+
+// Device address of the built-in array on the current device (looked up once
+// per device, with that device current: in host code the array's name only
+// stands in for it), or nullptr on failure.
+void* static_scratch(int dev) {
+  std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
+  if (!g_static_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_qspec_static_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_static_scratch_ptr[dev] = p;
+  }
+  return g_static_scratch_ptr[dev];
+}
 }  // namespace
 
 qspec_status qspec_gemm_w4a16_noalloc(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
@@ -473,31 +501,33 @@ qspec_status qspec_gemm_w4a16_noalloc(const uint16_t* x, int64_t m, int64_t k, c
   // The scratch needed by this shape must fit in the built-in array.
   if (plan_gemm(false, m, n, k, info.sm_count).total > QSPEC_STATIC_SCRATCH_BYTES)
     return QSPEC_ERR_WORKSPACE_TOO_SMALL;
-  void* scratch = nullptr;
-  {
-    // One-time set-up per device, with that device current: host code must
-    // ask the runtime for the array's device address (the symbol's name is
-    // only a host-side stand-in).
-    std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
-    if (!g_static_scratch_ptr[dev]) {
-      void* p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_qspec_static_scratch) != cudaSuccess || p == nullptr) {
-        cudaGetLastError();
-        return QSPEC_ERR_CUDA;
-      }
-      g_static_scratch_ptr[dev] = p;
-    }
-    scratch = g_static_scratch_ptr[dev];
-  }
-  // The array keeps whatever the previous call left: reset the status word and
-  // the split-tile tickets, the only parts that must start at zero.
+  void* scratch = static_scratch(dev);
+  if (!scratch) return QSPEC_ERR_CUDA;
+  // The array keeps whatever the previous call left.  The split-tile tickets
+  // must start at zero (a call that gave up may have left some taken); the
+  // status word is left alone, so that a fault stays visible until
+  // qspec_gemm_w4a16_noalloc_status() reads it.
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(scratch, 0, 256 + static_cast<size_t>(kMaxGrid) * 4, s) != cudaSuccess) {
+  if (cudaMemsetAsync(static_cast<uint8_t*>(scratch) + 256, 0, kStatusAndTicketBytes - 256, s) !=
+      cudaSuccess) {
     cudaGetLastError();
     return QSPEC_ERR_CUDA;
   }
   return run_gemm<false>(x, m, k, wq, ws, n, group, y, scratch, QSPEC_STATIC_SCRATCH_BYTES, nullptr,
                          flags, stream);
+}
+
+qspec_status qspec_gemm_w4a16_noalloc_status(void* stream) {
+  int dev = 0;
+  qspec_status st = current_device(&dev, nullptr);
+  if (st != QSPEC_OK) return st;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
+    scratch = g_static_scratch_ptr[dev];
+  }
+  if (!scratch) return QSPEC_OK;   // no call has run on this device
+  return qspec_workspace_status(scratch, stream);
 }
 
 const char* qspec_status_string(qspec_status status) {

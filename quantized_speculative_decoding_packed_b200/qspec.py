@@ -23,9 +23,11 @@ OP_QUANTIZE_WEIGHTS, OP_QUANT_ACT, OP_GEMM_W4A4, OP_GEMM_W4A16, OP_SPEC_ACCEPT =
 
 EXPORTED = ("qspec_quantize_weights", "qspec_quant_act", "qspec_gemm_w4a4", "qspec_gemm_w4a16",
             "qspec_spec_accept", "qspec_workspace_size", "qspec_workspace_status",
-            "qspec_status_string", "qspec_gemm_w4a16_noalloc", "qspec_abi_version")
-ABI_VERSION = 2
+            "qspec_status_string", "qspec_gemm_w4a16_noalloc", "qspec_gemm_w4a16_noalloc_status",
+            "qspec_abi_version")
+ABI_VERSION = 3
 GEMM_WEIGHTS_READY = 1   # flag: wq/ws are not written by work still in flight
+GEMM_TEST_STALL = 0x100  # test hook: the GEMM's first wait runs out (QSPEC_GEMM_TEST_STALL)
 
 
 class QSpecError(RuntimeError):
@@ -47,6 +49,7 @@ def _load() -> ctypes.CDLL:
     lib.qspec_gemm_w4a4.argtypes = [P, I64, I64, P, P, I64, I32, P, P, SZ, P, U32, P]
     lib.qspec_gemm_w4a16.argtypes = [P, I64, I64, P, P, I64, I32, P, P, SZ, U32, P]
     lib.qspec_gemm_w4a16_noalloc.argtypes = [P, I64, I64, P, P, I64, I32, P, U32, P]
+    lib.qspec_gemm_w4a16_noalloc_status.argtypes = [P]
     lib.qspec_abi_version.argtypes = []
     lib.qspec_abi_version.restype = I32
     lib.qspec_spec_accept.argtypes = [P, P, P, P, P, I32, I32, I32, P, P, P, SZ, P]
@@ -57,7 +60,7 @@ def _load() -> ctypes.CDLL:
     lib.qspec_status_string.restype = ctypes.c_char_p
     for name in ("qspec_quantize_weights", "qspec_quant_act", "qspec_gemm_w4a4",
                  "qspec_gemm_w4a16", "qspec_spec_accept", "qspec_workspace_status",
-                 "qspec_gemm_w4a16_noalloc"):
+                 "qspec_gemm_w4a16_noalloc", "qspec_gemm_w4a16_noalloc_status"):
         getattr(lib, name).restype = ctypes.c_int
     if lib.qspec_abi_version() != ABI_VERSION:
         raise ImportError(f"{_LIB_PATH} has ABI version {lib.qspec_abi_version()}, "
@@ -150,15 +153,19 @@ def quant_act(x: torch.Tensor, xq: torch.Tensor | None = None, xs: torch.Tensor 
     return xq, xs
 
 
+def _flags(weights_ready: bool, flags: int) -> int:
+    return (GEMM_WEIGHTS_READY if weights_ready else 0) | flags
+
+
 def gemm_w4a4(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor, group: int = 128,
               y: torch.Tensor | None = None, work: torch.Tensor | None = None,
               dbg_acc: torch.Tensor | None = None, stream=None,
-              weights_ready: bool = False) -> torch.Tensor:
+              weights_ready: bool = False, flags: int = 0) -> torch.Tensor:
     """W4A4 drafting GEMM: y[M][N] fp32 = quant(x) . deq(wq, ws)^T.
 
     weights_ready: wq/ws are not being written by work that may still be
     running (sets QSPEC_GEMM_WEIGHTS_READY; the weights then stream while the
-    preceding kernel finishes).
+    preceding kernel finishes).  flags: further QSPEC_GEMM_* bits.
     """
     _need(x, torch.bfloat16, "x")
     m, k = x.shape
@@ -169,15 +176,15 @@ def gemm_w4a4(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor, group: int = 
     if work is None:
         work = workspace(need, x.device)
     _check(LIB.qspec_gemm_w4a4(_ptr(x), m, k, _ptr(wq), _ptr(ws), n, group, _ptr(y), _ptr(work),
-                               work.numel(), _ptr(dbg_acc), GEMM_WEIGHTS_READY if weights_ready else 0,
+                               work.numel(), _ptr(dbg_acc), _flags(weights_ready, flags),
                                _stream(stream)), "qspec_gemm_w4a4")
     return y
 
 
 def gemm_w4a16(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor, group: int = 128,
                y: torch.Tensor | None = None, work: torch.Tensor | None = None,
-               stream=None, weights_ready: bool = False) -> torch.Tensor:
-    """W4A16 verifying GEMM: y[M][N] fp32 = x . deq(wq, ws)^T (weights_ready: as gemm_w4a4)."""
+               stream=None, weights_ready: bool = False, flags: int = 0) -> torch.Tensor:
+    """W4A16 verifying GEMM: y[M][N] fp32 = x . deq(wq, ws)^T (weights_ready, flags: as gemm_w4a4)."""
     _need(x, torch.bfloat16, "x")
     m, k = x.shape
     n = wq.shape[0]
@@ -187,7 +194,7 @@ def gemm_w4a16(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor, group: int =
     if work is None:
         work = workspace(need, x.device)
     _check(LIB.qspec_gemm_w4a16(_ptr(x), m, k, _ptr(wq), _ptr(ws), n, group, _ptr(y), _ptr(work),
-                                work.numel(), GEMM_WEIGHTS_READY if weights_ready else 0,
+                                work.numel(), _flags(weights_ready, flags),
                                 _stream(stream)), "qspec_gemm_w4a16")
     return y
 
@@ -209,6 +216,11 @@ def gemm_w4a16_noalloc(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor, grou
                                         GEMM_WEIGHTS_READY if weights_ready else 0,
                                         _stream(stream)), "qspec_gemm_w4a16_noalloc")
     return y
+
+
+def noalloc_status(stream=None) -> int:
+    """Device status of gemm_w4a16_noalloc on the current device (read and cleared)."""
+    return int(LIB.qspec_gemm_w4a16_noalloc_status(_stream(stream)))
 
 
 def spec_accept(p: torch.Tensor, q: torch.Tensor, draft: torch.Tensor, u_acc: torch.Tensor,

@@ -165,3 +165,25 @@ def big_accept_inputs(sigma: float, batch: int = 64, gamma: int = 5,
     idx = ACCEPT_SIGMAS.index(sigma) if sigma in ACCEPT_SIGMAS else 99
     return accept_inputs(rng_for("accept", 3, idx, batch, vocab), batch=batch, gamma=gamma,
                          vocab=vocab, logit_std=2.0, noise_std=sigma)
+
+
+def layer_weights(config: str, n: int, k: int, stream: int = 0) -> np.ndarray:
+    """fp32 [n][k] weights of one linear layer of a workload, N(0, 0.02^2)."""
+    return weights(rng_for(config, 4, stream, n, k), n, k)
+
+
+def layer_activations(config: str, m: int, k: int, stream: int = 0) -> np.ndarray:
+    """bf16 bit patterns [m][k] of a layer's input: N(0, 1), round(0.01 k) outlier channels x20."""
+    outl = outlier_channels(rng_for(config, 2, k), k)
+    return activations(rng_for(config, 5, stream, m, k), m, k, outl)
+
+
+def layer_weights_cuda(config: str, n: int, k: int, stream: int = 0, device="cuda") -> torch.Tensor:
+    """fp32 [n][k] N(0, 0.02^2) weights drawn on the device by a seeded torch
+    generator (for the large shapes, where drawing on the host is slow).  The
+    host-side checks read back the rows they sample."""
+    seed = int(np.random.SeedSequence([SEED_BASE + CONFIG_IDS[config], 6, stream, n, k])
+               .generate_state(1, dtype=np.uint64)[0] >> 1)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    return torch.randn((n, k), generator=gen, device=device, dtype=torch.float32) * 0.02

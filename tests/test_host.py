@@ -33,7 +33,7 @@ def test_header_declares_the_boundary():
 
 
 def test_abi_version(lib):
-    assert lib.LIB.qspec_abi_version() == lib.ABI_VERSION == 2
+    assert lib.LIB.qspec_abi_version() == lib.ABI_VERSION == 3
 
 
 def test_library_exports_every_declared_symbol(lib):

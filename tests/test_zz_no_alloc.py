@@ -6,7 +6,9 @@ plugin whose host application owns all device memory), so its scratch lives
 in a fixed device array inside the library.  These tests call it through the
 C ABI and check it against qspec_gemm_w4a16 on the same inputs, twice in a
 row (the array keeps the previous call's contents), and that sizes beyond the
-array are refused.  The file is named so that pytest collects it last.
+array are refused, against the oracle on one shape, and that its status
+query (which allocates nothing either) reports no fault after normal calls.
+The file is named so that pytest collects it last.
 """
 import ctypes
 
@@ -14,7 +16,10 @@ import numpy as np
 import pytest
 import torch
 
+from oracle import qspec_oracle as orc
 from quantized_speculative_decoding_packed_b200 import synth
+
+from gpu_util import assert_close_1e3
 
 pytestmark = pytest.mark.gpu
 
@@ -82,3 +87,16 @@ def test_refuses_shapes_beyond_the_builtin_scratch(qs):
     assert _call_noalloc(qs, x, wq, ws, n, 128, y) == 4    # QSPEC_ERR_WORKSPACE_TOO_SMALL
     torch.cuda.synchronize()
     assert not y.any()                                       # nothing was launched
+
+
+def test_matches_oracle_and_reports_clean_status(qs):
+    m, n, k, group = 80, 4096, 4096, 128
+    gi = synth.gemm_inputs("llama2_7b", m, n, k, group, stream=79)
+    wq, ws = qs.quantize_weights(torch.from_numpy(gi.w).cuda(), group)
+    x = torch.from_numpy(gi.x_bits.view(np.int16)).view(torch.bfloat16).cuda()
+    y = torch.empty((m, n), dtype=torch.float32, device="cuda")
+    assert _call_noalloc(qs, x, wq, ws, n, group, y) == 0
+    assert qs.LIB.qspec_gemm_w4a16_noalloc_status(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)) == 0
+    cols = np.arange(0, n, 16)
+    q, s_h = orc.quantize_weights(gi.w[cols], group)
+    assert_close_1e3(y.cpu().numpy()[:, cols], orc.gemm_w4a16(gi.x, q, s_h, group))
