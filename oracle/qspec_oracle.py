@@ -232,3 +232,29 @@ def spec_accept(p: np.ndarray, q: np.ndarray, draft: np.ndarray, u_acc: np.ndarr
         tokens[b, :n] = draft[b, :n]
         tokens[b, n] = tok
     return n_acc, tokens
+
+
+# --------------------------------------------------------------------------
+# Greedy verification (SpecQuant review, paragraph 5: a draft that matches in
+# full is kept, and at the first mismatch the target model's own choice
+# replaces the draft token).  Reading: the target's choice at position i is
+# its most probable token t_i = argmax_j p[b, i, j], ties going to the lowest
+# index; draft position i is accepted while draft[b, i] == t_i; n = first
+# mismatch (gamma if none); the new token is t_n (the correction at the
+# mismatch, or the bonus token from row gamma when every draft matched).
+# --------------------------------------------------------------------------
+def greedy_accept(p: np.ndarray, draft: np.ndarray):
+    """-> (n_accepted int32 [B], tokens int32 [B][gamma+1]; -1 pads after the new token)."""
+    bsz, gamma = draft.shape
+    n_acc = np.empty(bsz, dtype=np.int32)
+    tokens = np.full((bsz, gamma + 1), -1, dtype=np.int32)
+    for b in range(bsz):
+        n = gamma
+        for i in range(gamma):
+            if int(draft[b, i]) != int(np.argmax(p[b, i])):   # first maximum: lowest index
+                n = i
+                break
+        n_acc[b] = n
+        tokens[b, :n] = draft[b, :n]
+        tokens[b, n] = int(np.argmax(p[b, n]))
+    return n_acc, tokens

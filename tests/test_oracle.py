@@ -329,3 +329,81 @@ def test_accept_outputs_shape_and_prefix():
         assert tok[b, :first].tolist() == ai.draft[b, :first].tolist()
         assert 0 <= tok[b, first] < 32
         assert np.all(tok[b, first + 1:] == -1)
+
+
+# ---------------------------------------------------------------- greedy verification
+def _first_max(row) -> int:
+    """Index of the largest entry, the lowest one among equals (plain scan)."""
+    best = 0
+    for j in range(1, len(row)):
+        if row[j] > row[best]:
+            best = j
+    return best
+
+
+def _greedy_brute(p, draft):
+    bsz, gamma = draft.shape
+    out_n, out_t = [], []
+    for b in range(bsz):
+        t = [_first_max(list(map(float, p[b, i]))) for i in range(gamma + 1)]
+        n = 0
+        while n < gamma and int(draft[b, n]) == t[n]:
+            n += 1
+        out_n.append(n)
+        out_t.append([int(d) for d in draft[b, :n]] + [t[n]] + [-1] * (gamma - n))
+    return np.array(out_n), np.array(out_t)
+
+
+def test_greedy_matches_brute_force_scan():
+    rng = np.random.default_rng(31)
+    for trial in range(40):
+        bsz, gamma, vocab = 3, int(rng.integers(1, 6)), int(rng.integers(2, 9))
+        p = rng.integers(0, 4, size=(bsz, gamma + 1, vocab)).astype(np.float32)   # many ties
+        t = np.array([[_first_max(list(p[b, i])) for i in range(gamma)] for b in range(bsz)])
+        # drafts that follow the target for a random prefix, then may deviate
+        draft = t.copy()
+        for b in range(bsz):
+            cut = int(rng.integers(0, gamma + 1))
+            if cut < gamma:
+                draft[b, cut] = int(rng.integers(0, vocab))
+        n, tok = orc.greedy_accept(p, draft.astype(np.int32))
+        n_ref, tok_ref = _greedy_brute(p, draft)
+        assert np.array_equal(n, n_ref) and np.array_equal(tok, tok_ref), trial
+
+
+def test_greedy_ties_go_to_the_lowest_index():
+    p = np.zeros((1, 2, 6), dtype=np.float32)
+    p[0, 0, [1, 4]] = 0.5          # tie between tokens 1 and 4
+    p[0, 1, [2, 5]] = 0.5
+    n, tok = orc.greedy_accept(p, np.array([[4]], dtype=np.int32))
+    assert n.tolist() == [0] and tok.tolist() == [[1, -1]]
+    n, tok = orc.greedy_accept(p, np.array([[1]], dtype=np.int32))
+    assert n.tolist() == [1] and tok.tolist() == [[1, 2]]
+
+
+def test_greedy_equals_sampling_rule_for_deterministic_models():
+    """With one-hot target rows and one-hot draft rows at the draft tokens, the
+    speculative sampling rule (a separately pinned function) accepts exactly
+    where the draft equals the target's token and resamples that token."""
+    rng = np.random.default_rng(32)
+    bsz, gamma, vocab = 6, 4, 7
+    t = rng.integers(0, vocab, size=(bsz, gamma + 1))
+    p = np.zeros((bsz, gamma + 1, vocab), dtype=np.float32)
+    for b in range(bsz):
+        for i in range(gamma + 1):
+            p[b, i, t[b, i]] = 1.0
+    draft = t[:, :gamma].copy()
+    for b in range(bsz):
+        cut = b % (gamma + 1)
+        if cut < gamma:
+            draft[b, cut] = (t[b, cut] + 1 + b) % vocab
+    q = np.zeros((bsz, gamma, vocab), dtype=np.float32)
+    for b in range(bsz):
+        for i in range(gamma):
+            q[b, i, draft[b, i]] = 1.0
+    u_acc = synth.uniforms24(rng, (bsz, gamma))
+    u_res = synth.uniforms24(rng, (bsz,))
+    n_s, tok_s = orc.spec_accept(p, q, draft.astype(np.int32), u_acc, u_res)
+    n_g, tok_g = orc.greedy_accept(p, draft.astype(np.int32))
+    assert np.array_equal(n_s, n_g) and np.array_equal(tok_s, tok_g)
+    assert n_g.tolist() == [0, 1, 2, 3, 4, 0]
