@@ -144,6 +144,42 @@ def gemm_w4a4(x: np.ndarray, qw: np.ndarray, s_h: np.ndarray, group: int,
 
 
 # --------------------------------------------------------------------------
+# W4A8 drafting variant: a higher-precision draft activation (the SpecQuant
+# abstract's family of INT4 / FP8 / FP16 model copies; the QSpec page names
+# outlier-aware activation handling as the lever on draft quality).  Reading:
+# the per-token recipe of quant_act with 8-bit levels: s_a = a / 127 and
+# inv = 127 / a in fp32, q = clamp(rint(x * inv), -128, 127), the product x * inv
+# rounded to fp32; a zero row gives 0.  The GEMM is the W4A4 one with these codes:
+#     y[m, n] = s_a[m] * sum_g s_h[n, g] * sum_{k in g} qa[m, k] * qw[n, k].
+# --------------------------------------------------------------------------
+S127 = F32(127.0)
+
+
+def quant_act8(x: np.ndarray):
+    """bf16-valued fp32 [M][K] -> (q int16 [M][K] in [-128, 127], s_a fp32 [M])."""
+    x = np.asarray(x, dtype=np.float32)
+    a = np.abs(x).max(axis=1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        s_a = (a / S127).astype(np.float32)
+        inv = (S127 / a).astype(np.float32)
+        t = (x * inv[:, None]).astype(np.float32)
+    q = np.clip(np.rint(t), -128, 127)
+    q = np.where((a == 0)[:, None], 0, q)
+    return q.astype(np.int16), s_a
+
+
+def gemm_w4a8(x: np.ndarray, qw: np.ndarray, s_h: np.ndarray, group: int,
+              return_acc: bool = False):
+    qa, s_a = quant_act8(x)
+    acc = gemm_w4a4_acc(qa, qw, group)
+    y = np.einsum("mng,ng->mn", acc.astype(np.float64), s_h.astype(np.float64))
+    y = y * s_a.astype(np.float64)[:, None]
+    if return_acc:
+        return y, acc
+    return y
+
+
+# --------------------------------------------------------------------------
 # W4A16 verifying GEMM (QSpec abstract: "high-precision weight-only
 # quantization for accurate verification").  y = x . (q * s_h)^T with the
 # bf16 activations and the exactly dequantized weights, in float64.

@@ -187,3 +187,22 @@ def layer_weights_cuda(config: str, n: int, k: int, stream: int = 0, device="cud
     gen = torch.Generator(device=device)
     gen.manual_seed(seed)
     return torch.randn((n, k), generator=gen, device=device, dtype=torch.float32) * 0.02
+
+
+def greedy_inputs(rng: np.random.Generator, p: np.ndarray, follow: float = 0.8,
+                  plant_prob: float = 1.0, top: float = 2.0):
+    """Inputs for the greedy rule built without ranking anything: in each row
+    (with probability plant_prob) one uniformly drawn token is planted with the
+    value `top`, larger than every other entry; the draft copies the row's
+    planted token with probability `follow`, else takes a uniformly drawn token.
+    Returns (p with the planted values, int32 drafts [B][gamma])."""
+    p = p.copy()
+    bsz, g1, vocab = p.shape
+    planted = rng.integers(0, vocab, size=(bsz, g1))
+    mask = rng.random((bsz, g1)) < plant_prob
+    b_idx, i_idx = np.nonzero(mask)
+    p[b_idx, i_idx, planted[b_idx, i_idx]] = np.float32(top)
+    other = rng.integers(0, vocab, size=(bsz, g1 - 1))
+    keep = rng.random((bsz, g1 - 1)) < follow
+    draft = np.where(keep, planted[:, :g1 - 1], other).astype(np.int32)
+    return p, draft

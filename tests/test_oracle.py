@@ -174,6 +174,51 @@ def test_w4a4_accumulators_brute_force():
         assert abs(float(ex) - y[m, n]) <= 1e-14 * max(1.0, abs(float(ex)))
 
 
+# ---------------------------------------------------------------- W4A8 draft variant
+def test_quant_act8_brute_force_and_special_rows():
+    gi = synth.tiny_gemm_inputs()
+    x = gi.x.copy()
+    x[2, :] = 0.0                            # zero row
+    q, s_a = orc.quant_act8(x)
+    assert s_a[2] == 0 and np.all(q[2] == 0)
+    for m in (0, 1, 3):
+        a = Fraction(float(np.abs(x[m]).max()))
+        j = int(np.abs(x[m]).argmax())
+        assert q[m, j] == (127 if x[m, j] > 0 else -127)
+        for k in range(x.shape[1]):
+            exact = Fraction(float(x[m, k])) * 127 / a
+            want = max(-128, min(127, _half_even(exact)))
+            if want != q[m, k]:
+                assert _near_half(exact)
+        # the 8-bit codes resolve the row 127/7 times finer than the 4-bit ones
+        err8 = np.abs(q[m].astype(np.float64) * float(s_a[m]) - x[m]).max()
+        assert err8 <= float(a) / 127 / 2 * (1 + 1e-6)
+    assert q.min() >= -128 and q.max() <= 127
+
+
+def test_w4a8_accumulators_brute_force_and_closed_form():
+    gi = synth.tiny_gemm_inputs()
+    qw, s_h = orc.quantize_weights(gi.w, gi.group)
+    packed = orc.pack_int4(qw)
+    qa, s_a = orc.quant_act8(gi.x)
+    y, acc = orc.gemm_w4a8(gi.x, qw, s_h, gi.group, return_acc=True)
+    rows = [[_decode_nibble(packed[n], k) for k in range(qw.shape[1])] for n in (0, 5, 200)]
+    qa_l = qa.tolist()
+    for m in range(qa.shape[0]):
+        for ni, n in enumerate((0, 5, 200)):
+            for g in range(acc.shape[2]):
+                s = sum(qa_l[m][k] * rows[ni][k] for k in range(g * gi.group, (g + 1) * gi.group))
+                assert acc[m, n, g] == s
+    assert np.abs(acc).max() <= 128 * 8 * gi.group
+    deq_a = qa.astype(np.float64) * s_a.astype(np.float64)[:, None]
+    plain = deq_a @ orc.dequantize(qw, s_h, gi.group).T
+    assert np.allclose(y, plain, rtol=1e-12, atol=1e-12 * np.abs(plain).max())
+    # closer to the verifying mode than the 4-bit draft on the outlier-heavy inputs
+    y16 = orc.gemm_w4a16(gi.x, qw, s_h, gi.group)
+    y4 = orc.gemm_w4a4(gi.x, qw, s_h, gi.group)
+    assert np.linalg.norm(y - y16) < 0.5 * np.linalg.norm(y4 - y16)
+
+
 # ---------------------------------------------------------------- W4A16
 def test_w4a16_exact_rational_and_integer_special_case():
     gi = synth.tiny_gemm_inputs()
