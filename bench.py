@@ -59,6 +59,8 @@ def parse():
                     help="skip the Llama-3-8B-shaped M sweep report")
     ap.add_argument("--no-accept-report", action="store_true",
                     help="skip the vocab-128256 accept/resample report")
+    ap.add_argument("--no-chained", action="store_true",
+                    help="skip the chained-round report (layers fed by the previous layer)")
     ap.add_argument("--profile-gemm", metavar="MODE:SHAPE", default=None,
                     help="profiling driver: three calls of one GEMM (MODE w4a4|w4a16, SHAPE "
                          "qkv|o_proj|gate_up|down of the workload) on seeded weights, then exit")
@@ -537,6 +539,10 @@ def main():
     acc_rep = None
     if rank == 0 and world == 1 and not args.no_accept_report:
         acc_rep = accept_report(torch, qspec, peaks)
+    chained = None
+    if rank == 0 and world == 1 and not args.no_chained:
+        chained = chained_round_report(torch, qspec, peaks, wq, ws, L, x16, p, q, draft, u_acc,
+                                       u_res, n_acc, tokens, acc_work, bytes_step, ms_step)
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
@@ -548,7 +554,7 @@ def main():
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps,
                 "clocks": clk.summary(), "kernels": kern, "large_m": large,
-                "m_sweep": sweep, "accept_large_vocab": acc_rep}
+                "m_sweep": sweep, "accept_large_vocab": acc_rep, "round_chained": chained}
         print(json.dumps(line))
     if world > 1:
         del graph
@@ -748,6 +754,76 @@ def accept_report(torch, qspec, peaks, sigmas=(0.1, 0.5, 1.0), batch=64, gamma=5
             "bytes": "per sequence: 2 gathered elements per tested position + one vocab row of p "
                      "and q (rejection) or of p (all accepted) + outputs",
             "peak_hbm_gbs": hbm, "sigmas": out}
+
+
+def chained_round_report(torch, qspec, peaks, wq, ws, L, x16, p, q, draft, u_acc, u_res, n_acc,
+                         tokens, acc_work, bytes_unchained, ms_unchained):
+    """The round with its layers chained: in every pass each of the L layers' four GEMMs
+    takes the previous GEMM's fp32 output (its first K columns, cast to bf16 by the glue
+    kernel) as input: gamma W4A4 drafting passes at M = 16 (each from its own input),
+    one W4A16 verifying pass at M = 80, then accept.  Captured once as a CUDA graph.
+    Also the mode-switch cost: the same weights called W4A4 then W4A16 alternately,
+    against the same calls grouped by mode (CUDA graphs of back-to-back calls)."""
+    dev = x16[0].device
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(rank_seed(0) + 17)
+    hbm = float(peaks.get("hbm_gbs", 6650.0))
+    layers = [(wq[li][si], ws[li][si]) for li in range(L) for si in range(len(LAYERS))]
+    x0 = [torch.randn((M_DRAFT, 4096), generator=gen, device=dev).to(torch.bfloat16)
+          for _ in range(GAMMA)]
+    x0v = torch.randn((M_VERIFY, 4096), generator=gen, device=dev).to(torch.bfloat16)
+
+    def bufs(m):
+        ys = [torch.empty((m, wq_.shape[0]), dtype=torch.float32, device=dev) for (wq_, _) in layers]
+        xs = [None] + [torch.empty((m, wq_.shape[1] * 2), dtype=torch.bfloat16, device=dev)
+                       for (wq_, _) in layers[1:]]
+        return ys, xs
+
+    dbufs = [bufs(M_DRAFT) for _ in range(GAMMA)]
+    vbufs = bufs(M_VERIFY)
+    need = max(qspec.workspace_size(op, m, n, k, GROUP) for (_, n, k) in LAYERS
+               for (op, m) in ((qspec.OP_GEMM_W4A4, M_DRAFT), (qspec.OP_GEMM_W4A16, M_VERIFY)))
+    work = torch.zeros(need, dtype=torch.uint8, device=dev)
+
+    def round_():
+        for pss in range(GAMMA):
+            qspec.linear_chain(x0[pss], layers, "w4a4", GROUP, ys=dbufs[pss][0], xs=dbufs[pss][1],
+                               work=work, weights_ready=True)
+        qspec.linear_chain(x0v, layers, "w4a16", GROUP, ys=vbufs[0], xs=vbufs[1], work=work,
+                           weights_ready=True)
+        qspec.spec_accept(p, q, draft, u_acc, u_res, n_accepted=n_acc, tokens=tokens, work=acc_work)
+
+    t_round = _graph_time_per_call(torch, [round_], reps=5)
+    if qspec.workspace_status(work) != 0:
+        raise RuntimeError("device status reported a fault in the chained round")
+    glue = sum((GAMMA * M_DRAFT + M_VERIFY) * k * (4 + 2)
+               for (wq_, _) in layers[1:] for k in (wq_.shape[1] * 2,))
+    byts = bytes_unchained + glue
+    # mode switch: layer-0 gate_up weights, W4A4 at M=16 and W4A16 at M=80
+    wq0, ws0 = wq[0][2], ws[0][2]
+    xa = x16[2]
+    xv = torch.randn((M_VERIFY, 4096), generator=gen, device=dev).to(torch.bfloat16)
+    ya = torch.empty((M_DRAFT, 22016), dtype=torch.float32, device=dev)
+    yv = torch.empty((M_VERIFY, 22016), dtype=torch.float32, device=dev)
+    a = lambda: qspec.gemm_w4a4(xa, wq0, ws0, GROUP, y=ya, work=work, weights_ready=True)
+    v = lambda: qspec.gemm_w4a16(xv, wq0, ws0, GROUP, y=yv, work=work, weights_ready=True)
+    t_alt = _graph_time_per_call(torch, [a, v] * 10)
+    t_grp = _graph_time_per_call(torch, [a] * 10 + [v] * 10)
+    return {"workload": f"{L} Llama-2-7B-shaped layers chained (QKV -> first 4096 columns -> o_proj "
+                        "-> gate_up -> first 11008 columns -> down -> next layer), gamma="
+                        f"{GAMMA} W4A4 drafting passes at M={M_DRAFT} from their own inputs, one "
+                        f"W4A16 verifying pass at M={M_VERIFY}, accept B={BATCH} V={VOCAB}",
+            "glue": "qspec_cast_bf16 between consecutive GEMMs (fp32 output -> bf16 input)",
+            "ms_per_round": t_round * 1e3, "bytes": byts, "gbs": byts / t_round / 1e9,
+            "frac_hbm": byts / t_round / 1e9 / hbm,
+            "ms_per_round_unchained": ms_unchained,
+            "mode_switch": {
+                "shape": "gate_up 22016x4096 of layer 0, W4A4 at M=16 and W4A16 at M=80, one weight set",
+                "us_per_call_alternating": t_alt * 1e6, "us_per_call_grouped": t_grp * 1e6,
+                "switch_cost_us": (t_alt - t_grp) * 20 / 18 * 1e6,
+                "note": "20 calls alternating W4A4/W4A16 on the same wq/ws (19 switches) against "
+                        "the same 20 calls grouped by mode (1 switch): the time difference over "
+                        "the 18 extra switches"}}
 
 
 def measure_e2e(torch, stream, graph, acts, accept_in, outs, steps, bytes_step):

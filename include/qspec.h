@@ -83,7 +83,8 @@ enum {
   QSPEC_OP_QUANT_ACT = 1,
   QSPEC_OP_GEMM_W4A4 = 2,
   QSPEC_OP_GEMM_W4A16 = 3,
-  QSPEC_OP_SPEC_ACCEPT = 4
+  QSPEC_OP_SPEC_ACCEPT = 4,
+  QSPEC_OP_GEMM_W4A8 = 5
 };
 
 /*
@@ -119,6 +120,18 @@ qspec_status qspec_quant_act(const uint16_t* x, int64_t m, int64_t k, uint8_t* x
                              void* stream);
 
 /*
+ * Glue between chained linear layers (the synthetic draft-verify round runs
+ * the same layers back to back, each on the previous one's output): writes
+ * x[i][j] = bf16(y[i][j]) (round to nearest even) for i < m, j < k.
+ *  y   [m][ldy] fp32, the previous layer's output; its first k columns are read.
+ *  x   [m][k] bf16 bit patterns out.
+ * Requires m >= 1, k >= 8 and a multiple of 8, ldy >= k and a multiple of 4,
+ * y and x 16-byte aligned.
+ */
+qspec_status qspec_cast_bf16(const float* y, int64_t m, int64_t ldy, int64_t k, uint16_t* x,
+                             void* stream);
+
+/*
  * W4A4 drafting GEMM: y = x . deq(wq, ws)^T with the activations quantized
  * per token first (QSpec abstract: "low-precision joint quantization for
  * fast drafting").  Per group g, acc[m][n][g] = sum_{k in g} qa[m][k] qw[n][k]
@@ -140,6 +153,22 @@ qspec_status qspec_quant_act(const uint16_t* x, int64_t m, int64_t k, uint8_t* x
  * tile T is m rounded up to a multiple of 16 for m <= 96, else 128.
  */
 qspec_status qspec_gemm_w4a4(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
+                             const uint16_t* ws, int64_t n, int32_t group, float* y,
+                             void* workspace, size_t workspace_bytes, int32_t* dbg_acc,
+                             uint32_t flags, void* stream);
+
+/*
+ * W4A8 drafting variant: the W4A4 GEMM with 8-bit per-token activation codes
+ * (a higher-precision draft activation; the SpecQuant abstract builds INT4 /
+ * FP8 / FP16 model copies, and the QSpec page ties draft quality to how the
+ * activations are quantized).  For each row m: a = max_k |x|,
+ * s_a = a / 127, inv = 127 / a (fp32 divisions), qa = clamp(rint(x * inv),
+ * -128, 127); per group g, acc[m][n][g] = sum_{k in g} qa[m][k] qw[n][k]
+ * (exact, int32), y[m][n] = s_a[m] * sum_g s_h[n][g] * acc[m][n][g].
+ * Same weights, arguments, requirements and workspace layout as
+ * qspec_gemm_w4a4 (workspace sized for QSPEC_OP_GEMM_W4A8).
+ */
+qspec_status qspec_gemm_w4a8(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
                              const uint16_t* ws, int64_t n, int32_t group, float* y,
                              void* workspace, size_t workspace_bytes, int32_t* dbg_acc,
                              uint32_t flags, void* stream);
@@ -186,6 +215,29 @@ qspec_status qspec_spec_accept(const float* p, const float* q, const int32_t* dr
                                int32_t gamma, int32_t vocab, int32_t* n_accepted,
                                int32_t* tokens, void* workspace, size_t workspace_bytes,
                                void* stream);
+
+/*
+ * Greedy verification for a batch of sequences (SpecQuant review, paragraph
+ * 5: a draft that matches in full is kept and the first mismatch is replaced
+ * by the target model's own choice).  The target's choice at position i is
+ * t_i = argmax_j p[b][i][j], ties to the lowest index; draft position i is
+ * accepted while draft[b][i] == t_i; n = first mismatch (gamma if none); the
+ * new token is t_n.  Only rows 0..n of p are read.
+ *  p          [batch][gamma+1][vocab] fp32 target scores (probabilities or
+ *             logits: only their order matters); finite.
+ *  draft      [batch][gamma] int32 draft tokens.
+ *  n_accepted [batch] int32 out.
+ *  tokens     [batch][gamma+1] int32 out: accepted draft tokens, then t_n,
+ *             then -1 padding.
+ *  workspace  optional, as for qspec_spec_accept: a draft token outside
+ *             [0, vocab) never matches and is reported as BAD_INPUT there.
+ * Requires 1 <= batch <= 65535, 1 <= gamma <= 16, 4 <= vocab <= 409600, vocab % 4 == 0,
+ * p 16-byte aligned.
+ */
+qspec_status qspec_spec_accept_greedy(const float* p, const int32_t* draft, int32_t batch,
+                                      int32_t gamma, int32_t vocab, int32_t* n_accepted,
+                                      int32_t* tokens, void* workspace, size_t workspace_bytes,
+                                      void* stream);
 
 /*
  * W4A16 verifying GEMM that allocates nothing and takes no workspace.
@@ -243,8 +295,8 @@ size_t qspec_workspace_size(int32_t op, int64_t m, int64_t n, int64_t k, int32_t
  * for the next call. */
 qspec_status qspec_workspace_status(void* workspace, void* stream);
 
-/* Version of this ABI (3: adds QSPEC_GEMM_TEST_STALL and
- * qspec_gemm_w4a16_noalloc_status). */
+/* Version of this ABI (3: adds QSPEC_GEMM_TEST_STALL, qspec_gemm_w4a8, qspec_cast_bf16,
+ * qspec_spec_accept_greedy and qspec_gemm_w4a16_noalloc_status). */
 #define QSPEC_ABI_VERSION 3
 int32_t qspec_abi_version(void);
 

@@ -294,3 +294,32 @@ def greedy_accept(p: np.ndarray, draft: np.ndarray):
         tokens[b, :n] = draft[b, :n]
         tokens[b, n] = int(np.argmax(p[b, n]))
     return n_acc, tokens
+
+
+# --------------------------------------------------------------------------
+# A chained pass over linear layers (the synthetic draft-verify round: QSpec
+# abstract, the drafter and the verifier run the same layers on the same
+# quantized weights).  Each layer's input is the previous layer's fp32 output,
+# its first k columns (the next layer's input width), rounded to bf16;
+# `mode` picks the GEMM of every layer.  The pages describe no model around
+# the linear layers, so nothing else (attention, norms, activations) is in
+# the chain.
+# --------------------------------------------------------------------------
+def round_to_bf16(y: np.ndarray) -> np.ndarray:
+    """fp64/fp32 values -> fp32 (RN) -> bf16 (RN, ties to even), returned as fp32."""
+    b = np.asarray(y, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    b = (b + 0x7FFF + ((b >> 16) & 1)) >> 16
+    return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+def linear_chain(x0: np.ndarray, layers, mode: str, group: int):
+    """x0: bf16-valued fp32 [M][K0]; layers: [(q, s_h)] per GEMM in order.
+    Returns the float64 output of every layer."""
+    gemm = {"w4a4": gemm_w4a4, "w4a8": gemm_w4a8, "w4a16": gemm_w4a16}[mode]
+    outs = []
+    x = np.asarray(x0, dtype=np.float32)
+    for (q, s_h) in layers:
+        k = q.shape[1]
+        x = round_to_bf16(outs[-1][:, :k]) if outs else x
+        outs.append(gemm(x, q, s_h, group))
+    return outs

@@ -26,7 +26,10 @@
 
 namespace qspec {
 
-constexpr int kAcceptCluster = 8;
+// 16 CTAs per sequence (a non-portable cluster size, allowed on B200): at vocab
+// 128256 a CTA's chunk is 32 KB of shared memory, so the 64-sequence batch
+// (1024 CTAs) is resident in one wave.
+constexpr int kAcceptCluster = 16;
 constexpr int kAcceptThreads = 256;
 
 __device__ __forceinline__ uint64_t fixed_point_weight(float r) {
@@ -70,7 +73,6 @@ __device__ __forceinline__ uint64_t block_sum_u64(uint64_t v, uint64_t* red) {
 struct AcceptShared {
   uint64_t chunk_sum[2];                    // per pass; read by the other CTAs of the cluster
   uint64_t red[kAcceptThreads / 32];
-  uint64_t scan[kAcceptThreads];
   int n_acc;
   int token;
 };
@@ -90,25 +92,30 @@ __global__ void __cluster_dims__(kAcceptCluster, 1, 1) __launch_bounds__(kAccept
   const int crank = static_cast<int>(cluster.block_rank());
   const int tid = threadIdx.x;
 
-  // Phase 1: ratio test along the draft (a few scattered reads).
-  if (tid == 0) {
-    int n = gamma;
-    for (int i = 0; i < gamma; ++i) {
-      const int x = draft[b * gamma + i];
+  // Phase 1: ratio test at every draft position at once (lane i of the first
+  // warp takes position i: one round of scattered reads instead of gamma
+  // dependent ones); n = the first failing position, found by a ballot.
+  if (tid < 32) {
+    bool fail = false;
+    bool bad = false;
+    if (tid < gamma) {
+      const int x = draft[b * gamma + tid];
       if (x < 0 || x >= vocab) {
-        if (status && crank == 0) atomicOr(status, kDevBadInput);
-        n = i;
-        break;
-      }
-      const double pv = p[(static_cast<int64_t>(b) * (gamma + 1) + i) * vocab + x];
-      const double qv = q[(static_cast<int64_t>(b) * gamma + i) * vocab + x];
-      if (!(static_cast<double>(u_acc[b * gamma + i]) * qv < pv)) {
-        n = i;
-        break;
+        fail = bad = true;
+      } else {
+        const double pv = p[(static_cast<int64_t>(b) * (gamma + 1) + tid) * vocab + x];
+        const double qv = q[(static_cast<int64_t>(b) * gamma + tid) * vocab + x];
+        fail = !(static_cast<double>(u_acc[b * gamma + tid]) * qv < pv);
       }
     }
-    sh.n_acc = n;
-    sh.token = -1;
+    const uint32_t fails = __ballot_sync(0xffffffffu, fail);
+    const int n_first = fails ? (__ffs(fails) - 1) : gamma;
+    // only an invalid draft the rule actually reached counts as bad input
+    if (bad && tid == n_first && status && crank == 0) atomicOr(status, kDevBadInput);
+    if (tid == 0) {
+      sh.n_acc = n_first;
+      sh.token = -1;
+    }
   }
   __syncthreads();
   const int n = sh.n_acc;
@@ -172,21 +179,24 @@ __global__ void __cluster_dims__(kAcceptCluster, 1, 1) __launch_bounds__(kAccept
     const int a1 = min(len, a0 + per);
     uint64_t s = 0;
     for (int j = a0; j < a1; ++j) s += fixed_point_weight(r_s[j]);
-    sh.scan[tid] = s;
-    __syncthreads();
-    // Exclusive scan of the per-thread sums (256 entries, simple and exact).
-    if (tid == 0) {
-      uint64_t run = 0;
-      for (int i = 0; i < kAcceptThreads; ++i) {
-        const uint64_t v = sh.scan[i];
-        sh.scan[i] = run;
-        run += v;
-      }
+    // Exclusive scan of the per-thread sums: inclusive scans inside each warp
+    // by shuffles, then the warp totals (exact integer sums, any order).
+    const int lane = tid & 31, wid = tid >> 5;
+    uint64_t incl = s;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint64_t o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
     }
+    if (lane == 31) sh.red[wid] = incl;
     __syncthreads();
+    uint64_t warp_base = 0;
+#pragma unroll
+    for (int w = 0; w < kAcceptThreads / 32; ++w)
+      if (w < wid) warp_base += sh.red[w];
     uint64_t t = fixed_point_threshold(u_res[b], total);
     if (t >= total) t = total - 1;
-    const uint64_t base = prefix + sh.scan[tid];
+    const uint64_t base = prefix + warp_base + (incl - s);
     if (s != 0 && base <= t && t < base + s) {
       uint64_t c = base;
       for (int j = a0; j < a1; ++j) {
@@ -206,6 +216,103 @@ __global__ void __cluster_dims__(kAcceptCluster, 1, 1) __launch_bounds__(kAccept
       if (i < n) tokens[static_cast<int64_t>(b) * (gamma + 1) + i] = draft[b * gamma + i];
       if (i > n || (i == n && total == 0)) tokens[static_cast<int64_t>(b) * (gamma + 1) + i] = -1;
     }
+    if (tid == 0) n_accepted[b] = n;
+  }
+  // Keep this CTA's shared memory alive until every CTA of the cluster has read it.
+  cluster.sync();
+}
+
+// ---------------------------------------------------------------------------
+// Greedy verification (SpecQuant review, paragraph 5: a draft that matches in
+// full is kept; at the first mismatch the target model's own choice replaces
+// the draft token).  The target's choice at position i is t_i = argmax_j
+// p[b][i][j], ties to the lowest index; n = first i < gamma with
+// draft[b][i] != t_i (gamma if none); the new token is t_n.
+//
+// One cluster of kAcceptCluster CTAs per sequence walks the rows in order and
+// stops at the first mismatch, so only rows 0..n are read from HBM.  Each CTA
+// reduces its chunk of a row to (largest value, lowest index holding it),
+// publishes the pair in distributed shared memory, and after one cluster
+// barrier every CTA combines the same eight pairs into the same t_i, so the
+// whole cluster takes the same branch without further communication.
+struct ArgMax {
+  float v;
+  int i;
+};
+
+// The better of two candidates: larger value, or equal value and lower index.
+__device__ __forceinline__ ArgMax argmax_pick(ArgMax a, ArgMax b) {
+  return (b.v > a.v || (b.v == a.v && b.i < a.i)) ? b : a;
+}
+
+struct GreedyShared {
+  ArgMax part[2];                      // this CTA's pair for the current row (by parity)
+  ArgMax red[kAcceptThreads / 32];
+};
+
+__global__ void __cluster_dims__(kAcceptCluster, 1, 1) __launch_bounds__(kAcceptThreads)
+    greedy_accept_kernel(const float* __restrict__ p, const int32_t* __restrict__ draft, int gamma,
+                         int vocab, int chunk, int32_t* __restrict__ n_accepted,
+                         int32_t* __restrict__ tokens, uint32_t* __restrict__ status) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  __shared__ GreedyShared sh;
+  const int b = blockIdx.x / kAcceptCluster;
+  const int crank = static_cast<int>(cluster.block_rank());
+  const int tid = threadIdx.x;
+  const int lo = crank * chunk;
+  const int len = max(0, min(vocab, lo + chunk) - lo);
+
+  int n = gamma;
+  int token = -1;
+  bool bad = false;
+  for (int i = 0; i <= gamma; ++i) {
+    const float* row = p + (static_cast<int64_t>(b) * (gamma + 1) + i) * vocab + lo;
+    // thread-local scan: increasing indices, strict '>' keeps the first maximum
+    ArgMax best{-__int_as_float(0x7f800000), 0x7fffffff};
+    for (int j = tid * 4; j < len; j += kAcceptThreads * 4) {
+      const float4 v = *reinterpret_cast<const float4*>(row + j);
+      if (v.x > best.v) best = ArgMax{v.x, lo + j};
+      if (v.y > best.v) best = ArgMax{v.y, lo + j + 1};
+      if (v.z > best.v) best = ArgMax{v.z, lo + j + 2};
+      if (v.w > best.v) best = ArgMax{v.w, lo + j + 3};
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      ArgMax o;
+      o.v = __shfl_xor_sync(0xffffffffu, best.v, off);
+      o.i = __shfl_xor_sync(0xffffffffu, best.i, off);
+      best = argmax_pick(best, o);
+    }
+    if ((tid & 31) == 0) sh.red[tid >> 5] = best;
+    __syncthreads();
+    if (tid == 0) {
+      ArgMax c = sh.red[0];
+#pragma unroll
+      for (int w = 1; w < kAcceptThreads / 32; ++w) c = argmax_pick(c, sh.red[w]);
+      sh.part[i & 1] = c;
+    }
+    cluster.sync();
+    ArgMax t{-__int_as_float(0x7f800000), 0x7fffffff};
+    for (int c = 0; c < kAcceptCluster; ++c)
+      t = argmax_pick(t, *cluster.map_shared_rank(&sh.part[i & 1], c));
+    if (i == gamma) {
+      token = t.i;
+      break;
+    }
+    const int x = draft[b * gamma + i];
+    if (x < 0 || x >= vocab) bad = true;
+    if (x != t.i) {
+      n = i;
+      token = t.i;
+      break;
+    }
+  }
+  if (crank == 0) {
+    if (bad && status && tid == 0) atomicOr(status, kDevBadInput);
+    for (int i = tid; i <= gamma; i += kAcceptThreads)
+      tokens[static_cast<int64_t>(b) * (gamma + 1) + i] =
+          (i < n) ? draft[b * gamma + i] : (i == n ? token : -1);
     if (tid == 0) n_accepted[b] = n;
   }
   // Keep this CTA's shared memory alive until every CTA of the cluster has read it.

@@ -36,11 +36,24 @@ static __device__ unsigned long long* g_qspec_timeline = nullptr;
       for (int q_ = threadIdx.x; q_ < 16 * 64; q_ += blockDim.x)                        \
         g_qspec_timeline[blockIdx.x * 1024u + q_] = s_qspec_stamps[q_];                 \
   } while (0)
-// Coarse phase stamps (global timer, ns, comparable across SMs): [cta][16].
-static __device__ unsigned long long* g_qspec_phases = nullptr;
+// Coarse phase events (global timer, ns, comparable across SMs and launches),
+// appended to a log: {time, kind << 56 | launch << 32 | cta << 16 | event}.
+// `kTraceKind` names the kernel and `trace_launch` (24 bits) the launch; each
+// kernel defines both.
+static __device__ unsigned long long* g_qspec_events = nullptr;
+static __device__ unsigned int g_qspec_event_count = 0;
+constexpr unsigned kQspecEventCap = 1u << 20;
 #define QSPEC_PHASE(ev)                                                                 \
   do {                                                                                  \
-    if (g_qspec_phases) g_qspec_phases[blockIdx.x * 16u + (ev)] = global_timer_ns();    \
+    if (g_qspec_events) {                                                               \
+      const unsigned i_ = atomicAdd(&g_qspec_event_count, 1u);                          \
+      if (i_ < kQspecEventCap) {                                                        \
+        g_qspec_events[2u * i_] = global_timer_ns();                                    \
+        g_qspec_events[2u * i_ + 1u] = (static_cast<unsigned long long>(kTraceKind) << 56) | \
+                                       (static_cast<unsigned long long>(trace_launch & 0xFFFFFFu) << 32) | \
+                                       (static_cast<unsigned long long>(blockIdx.x) << 16) | (ev); \
+      }                                                                                 \
+    }                                                                                   \
   } while (0)
 #define QSPEC_ALIGN_OK(addr, a)                                                          \
   ((static_cast<unsigned long long>(addr) % (a)) == 0 ||                                 \

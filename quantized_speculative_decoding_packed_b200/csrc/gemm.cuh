@@ -294,6 +294,10 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
                  const __grid_constant__ CUtensorMap tmap_s, const __grid_constant__ GemmArgs args) {
   using C = GemmCfg<kInt8, MT>;
   constexpr int NPK = C::kNumPk, NA = C::kNumA, NX = C::kNumX, NACC = C::kNumAcc;
+  constexpr unsigned kTraceKind = kInt8 ? 1u : 2u;   // trace builds: event-log tags
+  const unsigned trace_launch = static_cast<unsigned>(reinterpret_cast<uintptr_t>(args.status) >> 8);
+  (void)kTraceKind;
+  (void)trace_launch;
   extern __shared__ uint8_t smem_raw[];
   QSPEC_STAMP_DECL
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -422,6 +426,8 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
         mbar_arrive_expect_tx(smem_u32(&pk_full[s]), C::kPkBytes);
         tma_load_2d(smem_u32(pk_buf + s * C::kPkBytes), &tmap_w, smem_u32(&pk_full[s]),
                     cur.kc * (C::kUnitK / 2), cur.n_tile * kTileN);
+        if (i == 0) QSPEC_PHASE(4);
+        if (u + 1 == u_end) QSPEC_PHASE(9);
       }
       __syncwarp();
       QSPEC_STAMP(0, i);
@@ -524,6 +530,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------ activation producer
     grid_dependency_wait();   // activations may come from the preceding kernel
+    if (lane == 0) QSPEC_PHASE(10);
     int i = 0;
     UnitCursor cur;
     cur.init(u_begin, ku, args.m_tiles);

@@ -222,10 +222,13 @@ qspec_status launch_qgemm(int mt, const CUtensorMap& tw, const CUtensorMap& tx, 
   }
 }
 
+// kInt8: the drafting modes (integer MMA on per-token activation codes of
+// act_bits = 4 (W4A4) or 8 (W4A8)); else the W4A16 verifying mode.
 template <bool kInt8>
 qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
                       const uint16_t* ws, int64_t n, int32_t group, float* y, void* workspace,
-                      size_t workspace_bytes, int32_t* dbg_acc, uint32_t flags, void* stream_v) {
+                      size_t workspace_bytes, int32_t* dbg_acc, uint32_t flags, void* stream_v,
+                      int act_bits = 4) {
   if (!x || !wq || !ws || !y || !workspace) return QSPEC_ERR_INVALID_ARG;
   if ((flags & ~(QSPEC_GEMM_WEIGHTS_READY | QSPEC_GEMM_TEST_STALL)) != 0u) return QSPEC_ERR_INVALID_ARG;
   const bool weights_ready = (flags & QSPEC_GEMM_WEIGHTS_READY) != 0u;
@@ -285,8 +288,13 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
     qc.numAttrs = 1;
     void* qout = xq;
     const int early = weights_ready ? 1 : 0;
-    if (cudaLaunchKernelEx(&qc, quant_act_kernel<false>, x, static_cast<int64_t>(k), qout, sa,
-                           early) != cudaSuccess) {
+    const cudaError_t qe =
+        (act_bits == 8)
+            ? cudaLaunchKernelEx(&qc, quant_act_kernel<false, 127>, x, static_cast<int64_t>(k), qout,
+                                 sa, early)
+            : cudaLaunchKernelEx(&qc, quant_act_kernel<false, 7>, x, static_cast<int64_t>(k), qout,
+                                 sa, early);
+    if (qe != cudaSuccess) {
       cudaGetLastError();
       return QSPEC_ERR_CUDA;
     }
@@ -307,6 +315,25 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
   return launch_qgemm<kInt8>(p.mt, tw, tx, ts, a, p.grid, dev, stream);
 }
 
+// Launch attributes of the accept kernels, set once per device (concurrent
+// first calls may both set them; idempotent): the residual sampler's dynamic
+// shared memory, and the 16-CTA clusters of both kernels.
+bool accept_attrs_set(int dev) {
+  static std::atomic<bool> done[kMaxDevices];
+  if (done[dev].load(std::memory_order_acquire)) return true;
+  if (cudaFuncSetAttribute(spec_accept_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           204800) != cudaSuccess ||
+      cudaFuncSetAttribute(spec_accept_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(greedy_accept_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                           1) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  done[dev].store(true, std::memory_order_release);
+  return true;
+}
+
 }  // namespace
 }  // namespace qspec
 
@@ -316,8 +343,12 @@ using namespace qspec;
 extern "C" int qspec_debug_set_trace(void* host_mapped) {
   return cudaMemcpyToSymbol(g_qspec_trace, &host_mapped, sizeof(void*)) == cudaSuccess ? 0 : 1;
 }
-extern "C" int qspec_debug_set_phases(void* dev_buffer) {
-  return cudaMemcpyToSymbol(g_qspec_phases, &dev_buffer, sizeof(void*)) == cudaSuccess ? 0 : 1;
+extern "C" int qspec_debug_set_events(void* dev_buffer) {
+  const unsigned zero = 0;
+  return (cudaMemcpyToSymbol(g_qspec_events, &dev_buffer, sizeof(void*)) == cudaSuccess &&
+          cudaMemcpyToSymbol(g_qspec_event_count, &zero, sizeof(zero)) == cudaSuccess)
+             ? 0
+             : 1;
 }
 extern "C" int qspec_debug_set_timeline(void* dev_buffer) {
   return cudaMemcpyToSymbol(g_qspec_timeline, &dev_buffer, sizeof(void*)) == cudaSuccess ? 0 : 1;
@@ -357,12 +388,36 @@ qspec_status qspec_quant_act(const uint16_t* x, int64_t m, int64_t k, uint8_t* x
   return cudaGetLastError() == cudaSuccess ? QSPEC_OK : QSPEC_ERR_CUDA;
 }
 
+qspec_status qspec_cast_bf16(const float* y, int64_t m, int64_t ldy, int64_t k, uint16_t* x,
+                             void* stream) {
+  if (!y || !x) return QSPEC_ERR_INVALID_ARG;
+  if (m < 1 || k < 8 || (k % 8) != 0 || ldy < k || (ldy % 4) != 0 || m * (k / 8) > (1ll << 40))
+    return QSPEC_ERR_INVALID_ARG;
+  if (!aligned(y, 16) || !aligned(x, 16)) return QSPEC_ERR_INVALID_ARG;
+  qspec_status st = current_device(nullptr, nullptr);
+  if (st != QSPEC_OK) return st;
+  const long long threads = m * (k / 8);
+  const long long blocks = (threads + 255) / 256;
+  if (blocks > 0x7FFFFFFFll) return QSPEC_ERR_INVALID_ARG;
+  cast_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      y, m, ldy, k, x);
+  return cudaGetLastError() == cudaSuccess ? QSPEC_OK : QSPEC_ERR_CUDA;
+}
+
 qspec_status qspec_gemm_w4a4(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
                              const uint16_t* ws, int64_t n, int32_t group, float* y,
                              void* workspace, size_t workspace_bytes, int32_t* dbg_acc,
                              uint32_t flags, void* stream) {
   return run_gemm<true>(x, m, k, wq, ws, n, group, y, workspace, workspace_bytes, dbg_acc, flags,
                         stream);
+}
+
+qspec_status qspec_gemm_w4a8(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
+                             const uint16_t* ws, int64_t n, int32_t group, float* y,
+                             void* workspace, size_t workspace_bytes, int32_t* dbg_acc,
+                             uint32_t flags, void* stream) {
+  return run_gemm<true>(x, m, k, wq, ws, n, group, y, workspace, workspace_bytes, dbg_acc, flags,
+                        stream, 8);
 }
 
 qspec_status qspec_gemm_w4a16(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
@@ -395,19 +450,34 @@ qspec_status qspec_spec_accept(const float* p, const float* q, const int32_t* dr
   if (st != QSPEC_OK) return st;
   const int chunk = ((vocab + 4 * kAcceptCluster - 1) / (4 * kAcceptCluster)) * 4;
   const size_t smem = static_cast<size_t>(chunk) * 4;
-  static std::atomic<bool> attr_set[kMaxDevices];   // as for the GEMM kernels
-  if (!attr_set[dev].load(std::memory_order_acquire)) {
-    if (cudaFuncSetAttribute(spec_accept_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             204800) != cudaSuccess) {
-      cudaGetLastError();
-      return QSPEC_ERR_CUDA;
-    }
-    attr_set[dev].store(true, std::memory_order_release);
-  }
+  if (!accept_attrs_set(dev)) return QSPEC_ERR_CUDA;
   spec_accept_kernel<<<batch * kAcceptCluster, kAcceptThreads, smem,
                        static_cast<cudaStream_t>(stream)>>>(
       p, q, draft, u_acc, u_res, gamma, vocab, chunk, n_accepted, tokens,
       static_cast<uint32_t*>(workspace));
+  return cudaGetLastError() == cudaSuccess ? QSPEC_OK : QSPEC_ERR_CUDA;
+}
+
+qspec_status qspec_spec_accept_greedy(const float* p, const int32_t* draft, int32_t batch,
+                                      int32_t gamma, int32_t vocab, int32_t* n_accepted,
+                                      int32_t* tokens, void* workspace, size_t workspace_bytes,
+                                      void* stream) {
+  if (!p || !draft || !n_accepted || !tokens) return QSPEC_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 65535 || gamma < 1 || gamma > 16 || vocab < 4 || vocab > 409600 ||
+      (vocab % 4) != 0)
+    return QSPEC_ERR_INVALID_ARG;
+  if (!aligned(p, 16) || !aligned(draft, 4) || !aligned(n_accepted, 4) || !aligned(tokens, 4))
+    return QSPEC_ERR_INVALID_ARG;
+  if (workspace && (workspace_bytes < 256 || !aligned(workspace, 16)))
+    return QSPEC_ERR_WORKSPACE_TOO_SMALL;
+  int dev = 0;
+  qspec_status st = current_device(&dev, nullptr);
+  if (st != QSPEC_OK) return st;
+  if (!accept_attrs_set(dev)) return QSPEC_ERR_CUDA;
+  const int chunk = ((vocab + 4 * kAcceptCluster - 1) / (4 * kAcceptCluster)) * 4;
+  greedy_accept_kernel<<<batch * kAcceptCluster, kAcceptThreads, 0,
+                         static_cast<cudaStream_t>(stream)>>>(
+      p, draft, gamma, vocab, chunk, n_accepted, tokens, static_cast<uint32_t*>(workspace));
   return cudaGetLastError() == cudaSuccess ? QSPEC_OK : QSPEC_ERR_CUDA;
 }
 
@@ -423,11 +493,12 @@ size_t qspec_workspace_size(int32_t op, int64_t m, int64_t n, int64_t k, int32_t
     case QSPEC_OP_SPEC_ACCEPT:
       return 256;
     case QSPEC_OP_GEMM_W4A4:
+    case QSPEC_OP_GEMM_W4A8:
     case QSPEC_OP_GEMM_W4A16: {
       if (!gemm_shape_ok(m, n, k, group)) return 0;
       DeviceInfo info;
       if (current_device(nullptr, &info) != QSPEC_OK) return 0;
-      return plan_gemm(op == QSPEC_OP_GEMM_W4A4, m, n, k, info.sm_count).total;
+      return plan_gemm(op != QSPEC_OP_GEMM_W4A16, m, n, k, info.sm_count).total;
     }
     default:
       return 0;

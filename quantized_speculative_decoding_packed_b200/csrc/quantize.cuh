@@ -8,6 +8,7 @@
 // compiler flags and forbid contraction into FMAs.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cstdint>
 
@@ -75,8 +76,10 @@ __device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) {
 
 // One CTA per token row.  kPacked: write two nibbles per byte (the ABI
 // format); otherwise write one int8 per element (the layout the W4A4 GEMM
-// streams into its tensor-core operand tiles).
-template <bool kPacked>
+// streams into its tensor-core operand tiles).  kQMax: 7 for the 4-bit codes
+// of the W4A4 drafter, 127 for the 8-bit codes of the W4A8 drafting variant
+// (s_a = absmax / kQMax, inv = kQMax / absmax, q clamped to [-kQMax-1, kQMax]).
+template <bool kPacked, int kQMax = 7>
 __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restrict__ x,
                                                         int64_t k, void* __restrict__ out,
                                                         float* __restrict__ scales,
@@ -85,7 +88,12 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
   const int64_t row = blockIdx.x;
   const uint16_t* xr = x + row * k;
   const int tid = threadIdx.x;
+  constexpr unsigned kTraceKind = 3u;   // trace builds: event-log tags
+  const unsigned trace_launch = static_cast<unsigned>(reinterpret_cast<uintptr_t>(out) >> 8);
+  (void)kTraceKind;
+  (void)trace_launch;
   QSPEC_TRACE_AT(1);
+  if (tid == 0) QSPEC_PHASE(0);
   // This kernel may be launched as a programmatic dependent of the previous
   // grid: wait for it (complete, memory flushed; a no-op otherwise) and let
   // the GEMM that consumes our output launch.  By default the GEMM launches
@@ -100,6 +108,7 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   }
+  if (tid == 0) QSPEC_PHASE(1);
   if (!QSPEC_ALIGN_OK(reinterpret_cast<uintptr_t>(xr), 16) ||
       !QSPEC_ALIGN_OK(reinterpret_cast<uintptr_t>(out), 8))
     return;
@@ -137,9 +146,12 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
 #pragma unroll
   for (int i = 1; i < 8; ++i) a = fmaxf(a, red[i]);
 
-  const float s = __fdiv_rn(a, 7.0f);
-  const float inv = __fdiv_rn(7.0f, a);
+  static_assert(!kPacked || kQMax == 7, "packed output holds 4-bit codes");
+  constexpr float kLevels = static_cast<float>(kQMax);
+  const float s = __fdiv_rn(a, kLevels);
+  const float inv = __fdiv_rn(kLevels, a);
   if (tid == 0) scales[row] = s;
+  auto clamp_code = [](int v) { return v < -kQMax - 1 ? -kQMax - 1 : (v > kQMax ? kQMax : v); };
 
   auto emit = [&](int64_t c, const uint4& u) {
     const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
@@ -148,8 +160,8 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
     for (int j = 0; j < 4; ++j) {
       const float lo = bf16_bits_to_float(w4[j] & 0xFFFFu);
       const float hi = bf16_bits_to_float(w4[j] >> 16);
-      q[2 * j] = (a == 0.f) ? 0 : clamp_q(__float2int_rn(__fmul_rn(lo, inv)));
-      q[2 * j + 1] = (a == 0.f) ? 0 : clamp_q(__float2int_rn(__fmul_rn(hi, inv)));
+      q[2 * j] = (a == 0.f) ? 0 : clamp_code(__float2int_rn(__fmul_rn(lo, inv)));
+      q[2 * j + 1] = (a == 0.f) ? 0 : clamp_code(__float2int_rn(__fmul_rn(hi, inv)));
     }
     if constexpr (kPacked) {
       uint32_t p = 0;
@@ -177,6 +189,29 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
   }
   for (int64_t c = (static_cast<int64_t>(tid) + 256 * kCache) * 8; c < k; c += 256 * 8)
     emit(c, *reinterpret_cast<const uint4*>(xr + c));
+  if (tid == 0) QSPEC_PHASE(8);
+}
+
+// Glue between chained linear layers: x[i][j] = bf16_RN(y[i][j]) for j < k,
+// the next layer's bf16 input from a layer's fp32 output (its first k
+// columns, row stride ldy).  One thread per 8 outputs: two 16-byte loads, one
+// 16-byte store.
+__global__ void __launch_bounds__(256) cast_bf16_kernel(const float* __restrict__ y, int64_t m,
+                                                        int64_t ldy, int64_t k,
+                                                        uint16_t* __restrict__ x) {
+  const int64_t per_row = k / 8;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= m * per_row) return;
+  const int64_t i = t / per_row;
+  const int64_t j = (t - i * per_row) * 8;
+  const float4 a = *reinterpret_cast<const float4*>(y + i * ldy + j);
+  const float4 b = *reinterpret_cast<const float4*>(y + i * ldy + j + 4);
+  auto pack = [](float lo, float hi) {
+    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(lo))) |
+           (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(hi))) << 16);
+  };
+  *reinterpret_cast<uint4*>(x + i * k + j) =
+      make_uint4(pack(a.x, a.y), pack(a.z, a.w), pack(b.x, b.y), pack(b.z, b.w));
 }
 
 }  // namespace qspec

@@ -19,10 +19,13 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqspec.s
 OK = 0
 STATUS_NAMES = {0: "ok", 1: "invalid argument", 2: "unsupported device", 3: "CUDA error",
                 4: "workspace too small", 5: "timeout", 6: "bad input"}
-OP_QUANTIZE_WEIGHTS, OP_QUANT_ACT, OP_GEMM_W4A4, OP_GEMM_W4A16, OP_SPEC_ACCEPT = range(5)
+OP_QUANTIZE_WEIGHTS, OP_QUANT_ACT, OP_GEMM_W4A4, OP_GEMM_W4A16, OP_SPEC_ACCEPT, OP_GEMM_W4A8 = range(6)
 
-EXPORTED = ("qspec_quantize_weights", "qspec_quant_act", "qspec_gemm_w4a4", "qspec_gemm_w4a16",
-            "qspec_spec_accept", "qspec_workspace_size", "qspec_workspace_status",
+EXPORTED = ("qspec_quantize_weights", "qspec_quant_act", "qspec_cast_bf16", "qspec_gemm_w4a4",
+            "qspec_gemm_w4a8",
+            "qspec_gemm_w4a16",
+            "qspec_spec_accept", "qspec_spec_accept_greedy", "qspec_workspace_size",
+            "qspec_workspace_status",
             "qspec_status_string", "qspec_gemm_w4a16_noalloc", "qspec_gemm_w4a16_noalloc_status",
             "qspec_abi_version")
 ABI_VERSION = 3
@@ -46,20 +49,25 @@ def _load() -> ctypes.CDLL:
                             ctypes.c_size_t)
     lib.qspec_quantize_weights.argtypes = [P, I64, I64, I32, P, P, P]
     lib.qspec_quant_act.argtypes = [P, I64, I64, P, P, P]
+    lib.qspec_cast_bf16.argtypes = [P, I64, I64, I64, P, P]
     lib.qspec_gemm_w4a4.argtypes = [P, I64, I64, P, P, I64, I32, P, P, SZ, P, U32, P]
+    lib.qspec_gemm_w4a8.argtypes = [P, I64, I64, P, P, I64, I32, P, P, SZ, P, U32, P]
     lib.qspec_gemm_w4a16.argtypes = [P, I64, I64, P, P, I64, I32, P, P, SZ, U32, P]
     lib.qspec_gemm_w4a16_noalloc.argtypes = [P, I64, I64, P, P, I64, I32, P, U32, P]
     lib.qspec_gemm_w4a16_noalloc_status.argtypes = [P]
     lib.qspec_abi_version.argtypes = []
     lib.qspec_abi_version.restype = I32
     lib.qspec_spec_accept.argtypes = [P, P, P, P, P, I32, I32, I32, P, P, P, SZ, P]
+    lib.qspec_spec_accept_greedy.argtypes = [P, P, I32, I32, I32, P, P, P, SZ, P]
     lib.qspec_workspace_size.argtypes = [I32, I64, I64, I64, I32, I32, I32, I32]
     lib.qspec_workspace_size.restype = SZ
     lib.qspec_workspace_status.argtypes = [P, P]
     lib.qspec_status_string.argtypes = [I32]
     lib.qspec_status_string.restype = ctypes.c_char_p
-    for name in ("qspec_quantize_weights", "qspec_quant_act", "qspec_gemm_w4a4",
-                 "qspec_gemm_w4a16", "qspec_spec_accept", "qspec_workspace_status",
+    for name in ("qspec_quantize_weights", "qspec_quant_act", "qspec_cast_bf16", "qspec_gemm_w4a4",
+                 "qspec_gemm_w4a8",
+                 "qspec_gemm_w4a16", "qspec_spec_accept", "qspec_spec_accept_greedy",
+                 "qspec_workspace_status",
                  "qspec_gemm_w4a16_noalloc", "qspec_gemm_w4a16_noalloc_status"):
         getattr(lib, name).restype = ctypes.c_int
     if lib.qspec_abi_version() != ABI_VERSION:
@@ -157,6 +165,39 @@ def _flags(weights_ready: bool, flags: int) -> int:
     return (GEMM_WEIGHTS_READY if weights_ready else 0) | flags
 
 
+def cast_bf16(y: torch.Tensor, k: int | None = None, x: torch.Tensor | None = None,
+              stream=None) -> torch.Tensor:
+    """fp32 [M][N] -> bf16 [M][k]: the first k columns rounded to nearest even."""
+    _need(y, torch.float32, "y")
+    m, n = y.shape
+    k = n if k is None else k
+    if x is None:
+        x = torch.empty((m, k), dtype=torch.bfloat16, device=y.device)
+    _check(LIB.qspec_cast_bf16(_ptr(y), m, n, k, _ptr(x), _stream(stream)), "qspec_cast_bf16")
+    return x
+
+
+def linear_chain(x0: torch.Tensor, layers, mode: str = "w4a4", group: int = 128,
+                 ys=None, xs=None, work: torch.Tensor | None = None, stream=None,
+                 weights_ready: bool = False):
+    """Runs linear layers back to back on one token batch: layer j's input is
+    the first K_j columns of layer j-1's fp32 output, rounded to bf16 by
+    qspec_cast_bf16.  layers: [(wq, ws)]; mode: w4a4 | w4a8 | w4a16.  ys/xs:
+    optional preallocated outputs / intermediate inputs (for CUDA-graph
+    capture).  Returns the list of fp32 outputs."""
+    gemm = {"w4a4": gemm_w4a4, "w4a8": gemm_w4a8, "w4a16": gemm_w4a16}[mode]
+    m = x0.shape[0]
+    outs = []
+    x = x0
+    for j, (wq, ws) in enumerate(layers):
+        n, k = wq.shape[0], wq.shape[1] * 2
+        if j:
+            x = cast_bf16(outs[-1], k, x=None if xs is None else xs[j], stream=stream)
+        y = None if ys is None else ys[j]
+        outs.append(gemm(x, wq, ws, group, y=y, work=work, stream=stream, weights_ready=weights_ready))
+    return outs
+
+
 def gemm_w4a4(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor, group: int = 128,
               y: torch.Tensor | None = None, work: torch.Tensor | None = None,
               dbg_acc: torch.Tensor | None = None, stream=None,
@@ -178,6 +219,25 @@ def gemm_w4a4(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor, group: int = 
     _check(LIB.qspec_gemm_w4a4(_ptr(x), m, k, _ptr(wq), _ptr(ws), n, group, _ptr(y), _ptr(work),
                                work.numel(), _ptr(dbg_acc), _flags(weights_ready, flags),
                                _stream(stream)), "qspec_gemm_w4a4")
+    return y
+
+
+def gemm_w4a8(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor, group: int = 128,
+              y: torch.Tensor | None = None, work: torch.Tensor | None = None,
+              dbg_acc: torch.Tensor | None = None, stream=None,
+              weights_ready: bool = False, flags: int = 0) -> torch.Tensor:
+    """W4A8 drafting variant: y[M][N] fp32 = quant8(x) . deq(wq, ws)^T (arguments as gemm_w4a4)."""
+    _need(x, torch.bfloat16, "x")
+    m, k = x.shape
+    n = wq.shape[0]
+    if y is None:
+        y = torch.empty((m, n), dtype=torch.float32, device=x.device)
+    need = workspace_size(OP_GEMM_W4A8, m, n, k, group)
+    if work is None:
+        work = workspace(need, x.device)
+    _check(LIB.qspec_gemm_w4a8(_ptr(x), m, k, _ptr(wq), _ptr(ws), n, group, _ptr(y), _ptr(work),
+                               work.numel(), _ptr(dbg_acc), _flags(weights_ready, flags),
+                               _stream(stream)), "qspec_gemm_w4a8")
     return y
 
 
@@ -243,4 +303,23 @@ def spec_accept(p: torch.Tensor, q: torch.Tensor, draft: torch.Tensor, u_acc: to
     _check(LIB.qspec_spec_accept(_ptr(p), _ptr(q), _ptr(draft), _ptr(u_acc), _ptr(u_res), b, gamma,
                                  v, _ptr(n_accepted), _ptr(tokens), _ptr(work), nbytes,
                                  _stream(stream)), "qspec_spec_accept")
+    return n_accepted, tokens
+
+
+def spec_accept_greedy(p: torch.Tensor, draft: torch.Tensor, n_accepted: torch.Tensor | None = None,
+                       tokens: torch.Tensor | None = None, work: torch.Tensor | None = None,
+                       stream=None):
+    """Greedy verification -> (n_accepted int32 [B], tokens int32 [B][gamma+1])."""
+    _need(p, torch.float32, "p")
+    _need(draft, torch.int32, "draft")
+    b, g1, v = p.shape
+    gamma = g1 - 1
+    if n_accepted is None:
+        n_accepted = torch.empty((b,), dtype=torch.int32, device=p.device)
+    if tokens is None:
+        tokens = torch.empty((b, gamma + 1), dtype=torch.int32, device=p.device)
+    nbytes = 0 if work is None else work.numel()
+    _check(LIB.qspec_spec_accept_greedy(_ptr(p), _ptr(draft), b, gamma, v, _ptr(n_accepted),
+                                        _ptr(tokens), _ptr(work), nbytes, _stream(stream)),
+           "qspec_spec_accept_greedy")
     return n_accepted, tokens

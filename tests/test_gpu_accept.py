@@ -85,3 +85,44 @@ def test_out_of_range_draft_is_reported(qs):
     assert n[1] <= 1
     assert qs.workspace_status(work) == 6
     assert qs.workspace_status(work) == 0           # reading clears it
+
+
+# ---------------------------------------------------------------- greedy verification
+def _run_greedy(qs, p, draft, work=None):
+    n, tok = qs.spec_accept_greedy(cuda_f32(p), cuda_i32(draft), work=work)
+    torch.cuda.synchronize()
+    return n.cpu().numpy(), tok.cpu().numpy()
+
+
+@pytest.mark.parametrize("sigma", synth.ACCEPT_SIGMAS)
+def test_greedy_vocab_128256_batch_64_identical(qs, sigma):
+    ai = synth.big_accept_inputs(sigma)
+    p, draft = synth.greedy_inputs(synth.rng_for("accept", 14, int(10 * sigma)), ai.p, follow=0.8)
+    n, tok = _run_greedy(qs, p, draft)
+    n_ref, tok_ref = orc.greedy_accept(p, draft)
+    assert np.array_equal(n, n_ref) and np.array_equal(tok, tok_ref)
+    assert 0 < n.mean() < 5
+
+
+@pytest.mark.parametrize("b,g,v", [(1, 1, 4), (2, 4, 32), (3, 16, 36), (5, 2, 1000), (130, 3, 2048)])
+def test_greedy_ragged_sizes_and_ties_identical(qs, b, g, v):
+    rng = synth.rng_for("accept", 15, b, g, v)
+    levels = rng.integers(0, 3, size=(b, g + 1, v)).astype(np.float32)   # many ties
+    p, draft = synth.greedy_inputs(rng, levels, follow=0.7, plant_prob=0.6, top=3.0)
+    n, tok = _run_greedy(qs, p, draft)
+    n_ref, tok_ref = orc.greedy_accept(p, draft)
+    assert np.array_equal(n, n_ref) and np.array_equal(tok, tok_ref)
+
+
+def test_greedy_all_match_takes_bonus_and_bad_draft_is_reported(qs):
+    ai = synth.accept_inputs(synth.rng_for("accept", 16), 4, 3, 4096, 2.0, 0.5)
+    p, draft = synth.greedy_inputs(synth.rng_for("accept", 17), ai.p, follow=1.0)
+    n, tok = _run_greedy(qs, p, draft)
+    n_ref, tok_ref = orc.greedy_accept(p, draft)
+    assert np.all(n == 3) and np.array_equal(tok, tok_ref)
+    draft[2, 1] = 4096                                # == vocab: invalid, never matches
+    work = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    n, tok = _run_greedy(qs, p, draft, work=work)
+    n_ref, tok_ref = orc.greedy_accept(p, draft)
+    assert n[2] == 1 and np.array_equal(tok, tok_ref)
+    assert qs.workspace_status(work) == 6

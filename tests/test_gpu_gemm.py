@@ -262,3 +262,35 @@ def test_weights_rewritten_just_before_the_call(qs, mode):
         assert torch.equal(y, want)
         qs.quantize_weights(cuda_f32(g_old.w), 128, wq=wq, ws=ws)
     assert qs.workspace_status(work) == 0
+
+
+# ---------------------------------------------------------------- W4A8 drafting variant
+@pytest.mark.parametrize("m,n,k,group", SHAPES[:8] + [(130, 384, 512, 128)])
+def test_w4a8_accumulators_exact_and_output(qs, m, n, k, group):
+    gi = synth.gemm_inputs("llama3_8b", m, n, k, group, stream=97)
+    wq, ws, q, s_h = _prep(qs, gi)
+    dbg = torch.zeros((m, n, k // group), dtype=torch.int32, device="cuda")
+    y = qs.gemm_w4a8(cuda_bf16(gi.x_bits), wq, ws, group, dbg_acc=dbg)
+    torch.cuda.synchronize()
+    y_ref, acc = orc.gemm_w4a8(gi.x, q, s_h, group, return_acc=True)
+    assert np.array_equal(dbg.cpu().numpy(), acc)
+    assert_close_1e3(y.cpu().numpy(), y_ref)
+
+
+@pytest.mark.parametrize("name,n,k", synth.LLAMA2_7B_LAYERS)
+def test_w4a8_llama2_7b_sampled_and_closer_to_verify(qs, name, n, k):
+    """Full 7B decode shapes at M = 16 on sampled columns; the 8-bit draft's outputs sit
+    closer to the verifying mode's than the 4-bit draft's (outlier channels x20)."""
+    gi = synth.gemm_inputs("llama2_7b", 16, n, k, 128)
+    wq, ws = qs.quantize_weights(cuda_f32(gi.w), 128)
+    x = cuda_bf16(gi.x_bits)
+    cols = np.sort(synth.rng_for("llama2_7b", 9, n).choice(n, size=256, replace=False))
+    q, s_h = orc.quantize_weights(gi.w[cols], 128)
+    y8 = qs.gemm_w4a8(x, wq, ws, 128)
+    y4 = qs.gemm_w4a4(x, wq, ws, 128)
+    y16 = qs.gemm_w4a16(x, wq, ws, 128)
+    torch.cuda.synchronize()
+    assert_close_1e3(y8.cpu().numpy()[:, cols], orc.gemm_w4a8(gi.x, q, s_h, 128))
+    d8 = float((y8 - y16).norm())
+    d4 = float((y4 - y16).norm())
+    assert d8 < 0.5 * d4

@@ -28,7 +28,8 @@ def test_header_declares_the_boundary():
     syms = declared_symbols()
     for name in ("qspec_quantize_weights", "qspec_quant_act", "qspec_gemm_w4a4",
                  "qspec_gemm_w4a16", "qspec_spec_accept", "qspec_workspace_size",
-                 "qspec_workspace_status", "qspec_status_string", "qspec_abi_version"):
+                 "qspec_workspace_status", "qspec_status_string", "qspec_abi_version",
+                 "qspec_spec_accept_greedy", "qspec_gemm_w4a16_noalloc_status"):
         assert name in syms
 
 
@@ -117,3 +118,9 @@ def test_stream_k_schedule_invariants(tmp_path):
     assert res.returncode == 0, res.stderr
     run = subprocess.run([str(exe)], capture_output=True, text=True)
     assert run.returncode == 0 and run.stdout.startswith("ok"), run.stdout
+
+
+@pytest.mark.parametrize("b,g,v", [(0, 4, 32), (2, 0, 32), (2, 17, 32), (2, 4, 30), (2, 4, 0)])
+def test_greedy_accept_rejects(lib, b, g, v):
+    assert lib.LIB.qspec_spec_accept_greedy(FAKE, FAKE, b, g, v, FAKE, FAKE, None, 0, None) == 1
+    assert lib.LIB.qspec_spec_accept_greedy(None, FAKE, 2, 4, 32, FAKE, FAKE, None, 0, None) == 1

@@ -452,3 +452,33 @@ def test_greedy_equals_sampling_rule_for_deterministic_models():
     n_g, tok_g = orc.greedy_accept(p, draft.astype(np.int32))
     assert np.array_equal(n_s, n_g) and np.array_equal(tok_s, tok_g)
     assert n_g.tolist() == [0, 1, 2, 3, 4, 0]
+
+
+# ---------------------------------------------------------------- chained pass
+def test_round_to_bf16_matches_a_library_conversion():
+    rng = np.random.default_rng(41)
+    y = np.concatenate([rng.standard_normal(4000) * 10.0 ** rng.integers(-30, 30, 4000),
+                        [0.0, -0.0, 1.0, 1.00390625, 1.0078125, 3.0e38]])
+    got = orc.round_to_bf16(y).view(np.uint32) >> 16
+    want = synth.to_bf16_bits(y.astype(np.float32)).astype(np.uint32)
+    assert np.array_equal(got, want)
+
+
+def test_linear_chain_is_the_composition_of_the_pinned_gemms():
+    rng = np.random.default_rng(42)
+    m, group = 5, 64
+    shapes = [(384, 256), (256, 256), (512, 256)]   # (N, K): slices 384 -> 256, 256 -> 256, ...
+    layers = []
+    for (n, k) in shapes:
+        w = (rng.standard_normal((n, k)) * 0.02).astype(np.float32)
+        layers.append(orc.quantize_weights(w, group))
+    x0 = synth.bf16_bits_to_f32(synth.to_bf16_bits(rng.standard_normal((m, 256)).astype(np.float32)))
+    for mode, fn in (("w4a4", orc.gemm_w4a4), ("w4a16", orc.gemm_w4a16)):
+        outs = orc.linear_chain(x0, layers, mode, group)
+        x = x0
+        for j, (q, s_h) in enumerate(layers):
+            if j:
+                # the next input: the first K columns, to fp32 then bf16 (textbook RNE on the bits)
+                x = synth.bf16_bits_to_f32(synth.to_bf16_bits(outs[j - 1][:, :q.shape[1]].astype(np.float32)))
+            assert np.array_equal(outs[j], fn(x, q, s_h, group)), (mode, j)
+        assert outs[-1].shape == (m, 512)
