@@ -61,6 +61,9 @@ def parse():
                     help="skip the vocab-128256 accept/resample report")
     ap.add_argument("--no-chained", action="store_true",
                     help="skip the chained-round report (layers fed by the previous layer)")
+    ap.add_argument("--profile-accept", metavar="RULE", default=None,
+                    help="profiling driver: three calls of the accept step (RULE sampling|greedy) "
+                         "at vocab 128256, batch 64, gamma 5, sigma 0.5, then exit")
     ap.add_argument("--profile-gemm", metavar="MODE:SHAPE", default=None,
                     help="profiling driver: three calls of one GEMM (MODE w4a4|w4a16, SHAPE "
                          "qkv|o_proj|gate_up|down of the workload) on seeded weights, then exit")
@@ -68,12 +71,18 @@ def parse():
 
 
 def profile_gemm(spec):
-    """Three calls of one GEMM of the workload, for a profiler to capture one of them."""
+    """Three calls of one GEMM of the workload, for a profiler to capture one of them.
+    SHAPE is a Llama-2-7B layer (decode M), or one of the Llama-2-70B layers with a
+    "70b_" prefix (M = 2048)."""
     import torch
     from quantized_speculative_decoding_packed_b200 import qspec
     mode, shape = spec.split(":")
-    n, k = {name: (n, k) for name, n, k in LAYERS}[shape]
-    m = M_DRAFT if mode == "w4a4" else M_VERIFY
+    if shape.startswith("70b_"):
+        n, k = {name: (n, k) for name, n, k in LARGE_SHAPES}[shape[4:]]
+        m = LARGE_M
+    else:
+        n, k = {name: (n, k) for name, n, k in LAYERS}[shape]
+        m = M_DRAFT if mode == "w4a4" else M_VERIFY
     gen = torch.Generator(device="cuda")
     gen.manual_seed(rank_seed(0))
     w = torch.randn((n, k), generator=gen, device="cuda", dtype=torch.float32) * 0.02
@@ -85,6 +94,30 @@ def profile_gemm(spec):
         y = fn(x, wq, ws, GROUP)
     torch.cuda.synchronize()
     print(f"{mode} {shape}: y[{m}][{n}] sum |y| = {float(y.abs().sum()):.6g}")
+
+
+def profile_accept(rule, batch=64, gamma=5, vocab=128256, sigma=0.5):
+    """Three calls of the accept step on seeded inputs, for a profiler to capture one."""
+    import torch
+    from quantized_speculative_decoding_packed_b200 import qspec
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(rank_seed(0) + 13)
+    lp = torch.randn((batch, gamma + 1, vocab), generator=gen, device="cuda", dtype=torch.float64) * 2
+    lq = lp[:, :gamma] + torch.randn((batch, gamma, vocab), generator=gen, device="cuda",
+                                     dtype=torch.float64) * sigma
+    p = torch.softmax(lp, -1).float().contiguous()
+    q = torch.softmax(lq, -1).float().contiguous()
+    draft = torch.multinomial(q.reshape(-1, vocab).double(), 1, generator=gen).reshape(
+        batch, gamma).to(torch.int32)
+    u_acc = torch.rand((batch, gamma), generator=gen, device="cuda")
+    u_res = torch.rand((batch,), generator=gen, device="cuda")
+    for _ in range(3):
+        if rule == "greedy":
+            n, tok = qspec.spec_accept_greedy(p, draft)
+        else:
+            n, tok = qspec.spec_accept(p, q, draft, u_acc, u_res)
+    torch.cuda.synchronize()
+    print(f"accept {rule}: mean accepted {float(n.float().mean()):.3f}")
 
 
 # ---------------------------------------------------------------- algorithmic bytes / ops
@@ -336,6 +369,9 @@ def main():
     if args.profile_gemm:
         profile_gemm(args.profile_gemm)
         return
+    if args.profile_accept:
+        profile_accept(args.profile_accept)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -539,6 +575,9 @@ def main():
     acc_rep = None
     if rank == 0 and world == 1 and not args.no_accept_report:
         acc_rep = accept_report(torch, qspec, peaks)
+    fused_ab = None
+    if rank == 0 and world == 1 and not args.no_chained:
+        fused_ab = fused_quant_report(torch, qspec, wq, ws, L, x16)
     chained = None
     if rank == 0 and world == 1 and not args.no_chained:
         chained = chained_round_report(torch, qspec, peaks, wq, ws, L, x16, p, q, draft, u_acc,
@@ -554,7 +593,8 @@ def main():
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps,
                 "clocks": clk.summary(), "kernels": kern, "large_m": large,
-                "m_sweep": sweep, "accept_large_vocab": acc_rep, "round_chained": chained}
+                "m_sweep": sweep, "accept_large_vocab": acc_rep, "round_chained": chained,
+                "fused_quant_ab": fused_ab}
         print(json.dumps(line))
     if world > 1:
         del graph
@@ -754,6 +794,29 @@ def accept_report(torch, qspec, peaks, sigmas=(0.1, 0.5, 1.0), batch=64, gamma=5
             "bytes": "per sequence: 2 gathered elements per tested position + one vocab row of p "
                      "and q (rejection) or of p (all accepted) + outputs",
             "peak_hbm_gbs": hbm, "sigmas": out}
+
+
+def fused_quant_report(torch, qspec, wq, ws, L, x16):
+    """One W4A4 drafting pass of the step (L layers x 4 GEMMs at M = 16), timed as a CUDA
+    graph with the activations quantized by the separate per-token pre-pass kernel (the
+    default) and inside the GEMM kernel (QSPEC_GEMM_FUSED_QUANT)."""
+    dev = x16[0].device
+    need = max(qspec.workspace_size(qspec.OP_GEMM_W4A4, M_DRAFT, n, k, GROUP) for (_, n, k) in LAYERS)
+    work = torch.zeros(need, dtype=torch.uint8, device=dev)
+    ys = [torch.empty((M_DRAFT, n), dtype=torch.float32, device=dev) for (_, n, k) in LAYERS]
+    out = {}
+    for name, flags in (("pre_pass", 0), ("fused", qspec.GEMM_FUSED_QUANT)):
+        def pass_(flags=flags):
+            for li in range(L):
+                for si in range(len(LAYERS)):
+                    qspec.gemm_w4a4(x16[si], wq[li][si], ws[li][si], GROUP, y=ys[si], work=work,
+                                    weights_ready=True, flags=flags)
+        t = _graph_time_per_call(torch, [pass_], reps=5)
+        out[name] = {"us_per_pass": t * 1e6, "us_per_gemm": t * 1e6 / (L * len(LAYERS))}
+    if qspec.workspace_status(work) != 0:
+        raise RuntimeError("device status reported a fault in the fused-quantization pass")
+    return {"workload": f"one W4A4 drafting pass: {L} layers x 4 GEMMs at M={M_DRAFT}",
+            "pre_pass": out["pre_pass"], "fused": out["fused"]}
 
 
 def chained_round_report(torch, qspec, peaks, wq, ws, L, x16, p, q, draft, u_acc, u_res, n_acc,

@@ -66,6 +66,17 @@ typedef enum qspec_status {
  */
 #define QSPEC_GEMM_WEIGHTS_READY 1u
 /*
+ *  QSPEC_GEMM_FUSED_QUANT (drafting modes, m <= 32; ignored otherwise): the
+ *    GEMM kernel quantizes the activations itself instead of a separate
+ *    per-token pre-pass kernel: the epilogue warps of CTA c quantize token
+ *    rows c, c + grid, ... into the workspace and count them done, and every
+ *    CTA's activation producer waits (bounded) for all rows before loading
+ *    them.  Same codes, scales and results as without the flag.  Measured on
+ *    B200 it is slower than the pre-pass (the cross-CTA hand-off costs about
+ *    what the kernel boundary does), so it is not the default.
+ */
+#define QSPEC_GEMM_FUSED_QUANT 2u
+/*
  *  QSPEC_GEMM_TEST_STALL: a test hook for the failure path, not for normal
  *    use.  The GEMM's weight producer first waits, for 10 ms at most, on a
  *    barrier that nothing signals; the wait runs out and every CTA gives up

@@ -88,6 +88,11 @@ constexpr int kMmaDone = kAccEmpty + kMaxAcc, kScFull = kMmaDone + 1, kScEmpty =
 constexpr int kFlush = kScEmpty + kNumSc, kTicket = kFlush + 2, kTail = kTicket + 2;
 constexpr int kStall = kTail + 1;   // never signalled: the test hook's wait
 constexpr int kCount = kStall + 1;
+// Fused activation quantization only, in a block of their own: the barrier
+// that hands the token scales to the epilogue, the one on which the epilogue
+// warps combine a row's absmax, then the row partials and the token scales.
+constexpr int kScaleReady = 0, kRowAmax = 1;
+constexpr int kFusedCount = kRowAmax + 1;
 }  // namespace bar
 constexpr int kNumBars = bar::kCount;
 // The flag words follow the barriers on a 16-byte boundary: with them 8 bytes
@@ -95,6 +100,12 @@ constexpr int kNumBars = bar::kCount;
 // longer on B200 (measured: +17 to +35 % per decode GEMM call).
 constexpr int kMiscOffset = (kNumBars * 8 + 15) / 16 * 16;
 static_assert(kMiscOffset + 8 * 4 <= 1024, "barrier block overflow");
+// The fused block: its barriers, the row absmax partials of up to 4 epilogue
+// warps (double-buffered), then the token scales (token tiles <= 32).
+constexpr int kRowPartOffset = (bar::kFusedCount * 8 + 15) / 16 * 16;
+constexpr int kTokScaleOffset = kRowPartOffset + 2 * 4 * 4;
+constexpr int kFusedBlockBytes = 1024;
+static_assert(kTokScaleOffset + 32 * 4 <= kFusedBlockBytes, "fused block overflow");
 
 // Arrival count of barrier b in that order.
 __device__ __forceinline__ uint32_t bar_count(int b, int epi_warps) {
@@ -105,12 +116,17 @@ __device__ __forceinline__ uint32_t bar_count(int b, int epi_warps) {
   return 1;
 }
 
+
 __host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 __host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
 
-template <bool kInt8, int MT>
+// kFused (drafting modes, token tiles of 16 or 32): the kernel quantizes the
+// bf16 activations itself (see qgemm_kernel) instead of a separate pre-pass
+// kernel doing it.
+template <bool kInt8, int MT, bool kFused = false>
 struct GemmCfg {
   static_assert(MT % 16 == 0 && MT >= 16 && MT <= 128, "token tile must be 16..128, step 16");
+  static_assert(!kFused || (kInt8 && MT <= 32), "fused activation quantization: int8, MT <= 32");
   static constexpr int kUnitK = unit_k(kInt8);
   static constexpr int kPkBytes = kTileN * kUnitK / 2;           // packed bytes per unit
   static constexpr int kElem = kInt8 ? 1 : 2;                    // bytes per widened element
@@ -138,7 +154,7 @@ struct GemmCfg {
   static constexpr int kConvWarps = kConvTeamWarps * kConvTeams;
   static constexpr int kWarps = kCtlWarps + kConvWarps + kEpiWarps;
   static constexpr int kThreads = 32 * kWarps;
-  static constexpr int kBarBytes = 1024;
+  static constexpr int kBarBytes = 1024 + (kFused ? kFusedBlockBytes : 0);
   static constexpr int kScaleBytes = kNumSc * kScaleTileBytes;
   // Ring depths from the shared-memory budget: packed weights first (they
   // cover HBM latency), activations (an L2 hit) with what is left.
@@ -160,8 +176,12 @@ struct GemmArgs {
   int weights_ready;       // wq/ws may be read before the preceding grid completes
   uint32_t test_stall_ns;  // test hook (0 = off): the weight producer first waits this
                            // long on a barrier that nothing signals, then gives up
+  float qmax;              // activation codes: 7 (4-bit) or 127 (8-bit)
+  const uint16_t* x;       // fused: bf16 activations [M][K]
+  int8_t* xq;              // fused: int8 codes [M][K] written by this kernel (workspace)
+  uint32_t* qsync;         // fused: [0] rows quantized, [1] CTAs that have seen them all
   const uint16_t* ws;      // fp16 scales [N][K/group]
-  const float* s_a;        // W4A4: per-token scales [M]
+  const float* s_a;        // drafting modes: per-token scales [M] (fused: written by this kernel)
   float* y;                // [M][N]
   int32_t* dbg_acc;        // optional W4A4 per-group accumulators [M][N][K/group]
   uint32_t* status;        // device status word
@@ -289,14 +309,90 @@ __device__ __forceinline__ void st_release_cta(uint32_t* p, uint32_t v) {
   asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
 }
 
+// Fused activation quantization of one token row by the NW epilogue warps of
+// a CTA, with the arithmetic of quant_act_kernel: a = max_k |x|, s_a = a / qmax
+// and inv = qmax / a (IEEE fp32 divisions), q = clamp(rint(x * inv), -qmax-1,
+// qmax) with the product rounded to fp32, a zero row giving 0; the codes are
+// stored as the GEMM reads them, each 8 channels in the order 0,2,4,6,1,3,5,7.
+// Each thread keeps up to kCache 16-byte chunks of the row in registers between
+// the two passes (all its loads in flight at once); rows longer than
+// 8 * kCache * 32 * NW elements read the rest twice.  The warps combine their
+// absmax partials through shared memory and the barrier `row_bar` (count NW,
+// one phase per row; `part` is double-buffered by that phase).  Returns false
+// if the wait gave up.  K is a multiple of 8; rows are 16-byte aligned.
+template <int NW>
+__device__ __forceinline__ bool quantize_row_team(const uint16_t* xr, int K, int8_t* qr,
+                                                  float* s_out, float qmax, int ew, int lane,
+                                                  float* part, uint32_t row_bar, uint32_t phase,
+                                                  volatile int* abort_flag, uint32_t* status) {
+  constexpr int T = NW * 32;
+  constexpr int kCache = 8;
+  const int t = ew * 32 + lane;
+  auto bf = [](uint32_t bits16) { return __uint_as_float(bits16 << 16); };
+  auto absmax8 = [&](const uint4& u, float m) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) m = fmaxf(m, fmaxf(fabsf(bf(w[j] & 0xFFFFu)), fabsf(bf(w[j] >> 16))));
+    return m;
+  };
+  uint4 cache[kCache];
+#pragma unroll
+  for (int j = 0; j < kCache; ++j) {
+    const int c = (t + T * j) * 8;
+    if (c < K) cache[j] = __ldcg(reinterpret_cast<const uint4*>(xr + c));   // written by the preceding grid
+  }
+  float a = 0.f;
+#pragma unroll
+  for (int j = 0; j < kCache; ++j)
+    if ((t + T * j) * 8 < K) a = absmax8(cache[j], a);
+  for (int c = (t + T * kCache) * 8; c < K; c += T * 8)
+    a = absmax8(__ldcg(reinterpret_cast<const uint4*>(xr + c)), a);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+  float* pp = part + (phase & 1u) * 4;
+  if (lane == 0) pp[ew] = a;
+  __syncwarp();
+  if (lane == 0) mbar_arrive(row_bar);
+  if (!warp_wait(row_bar, phase & 1u, abort_flag, status)) return false;
+  a = pp[0];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) a = fmaxf(a, pp[w]);
+  const float inv = __fdiv_rn(qmax, a);
+  if (t == 0) *s_out = __fdiv_rn(a, qmax);
+  const int qm = static_cast<int>(qmax);
+  auto emit = [&](int c, const uint4& u) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t ev = 0, od = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      int lo = __float2int_rn(__fmul_rn(bf(w[j] & 0xFFFFu), inv));
+      int hi = __float2int_rn(__fmul_rn(bf(w[j] >> 16), inv));
+      lo = (a == 0.f) ? 0 : (lo < -qm - 1 ? -qm - 1 : (lo > qm ? qm : lo));
+      hi = (a == 0.f) ? 0 : (hi < -qm - 1 ? -qm - 1 : (hi > qm ? qm : hi));
+      ev |= (static_cast<uint32_t>(lo) & 0xFFu) << (8 * j);
+      od |= (static_cast<uint32_t>(hi) & 0xFFu) << (8 * j);
+    }
+    *reinterpret_cast<uint2*>(qr + c) = make_uint2(ev, od);
+  };
+#pragma unroll
+  for (int j = 0; j < kCache; ++j) {
+    const int c = (t + T * j) * 8;
+    if (c < K) emit(c, cache[j]);
+  }
+  for (int c = (t + T * kCache) * 8; c < K; c += T * 8)
+    emit(c, __ldcg(reinterpret_cast<const uint4*>(xr + c)));
+  return true;
+}
+
 // kDbg (int8 mode only): also write the per-group integer accumulators.  A
 // separate instantiation keeps those stores out of the hot loop's code.
-template <bool kInt8, int MT, bool kDbg>
-__global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
+// kFused: see GemmCfg.
+template <bool kInt8, int MT, bool kDbg, bool kFused>
+__global__ void __launch_bounds__(GemmCfg<kInt8, MT, kFused>::kThreads, 1)
     qgemm_kernel(const __grid_constant__ CUtensorMap tmap_w,
                  const __grid_constant__ CUtensorMap tmap_x,
                  const __grid_constant__ CUtensorMap tmap_s, const __grid_constant__ GemmArgs args) {
-  using C = GemmCfg<kInt8, MT>;
+  using C = GemmCfg<kInt8, MT, kFused>;
   constexpr int NPK = C::kNumPk, NA = C::kNumA, NX = C::kNumX, NACC = C::kNumAcc;
   constexpr unsigned kTraceKind = kInt8 ? 1u : 2u;   // trace builds: event-log tags
   const unsigned trace_launch = static_cast<unsigned>(reinterpret_cast<uintptr_t>(args.status) >> 8);
@@ -325,6 +421,11 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
   uint64_t* flush_bar = bars + bar::kFlush;
   uint64_t* ticket_bar = bars + bar::kTicket;  // ... and its ticket taken (misc[3], misc[6])
   uint64_t* tail_bar = bars + bar::kTail;      // the other contributor's tail share is out
+  uint64_t* fbars = bars + 1024 / 8;                // the fused block (fused configurations only)
+  uint64_t* scale_ready = fbars + bar::kScaleReady;  // the token scales are in s_tok_scale
+  uint64_t* row_amax = fbars + bar::kRowAmax;        // the epilogue warps' row partials are in
+  float* s_row_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(fbars) + kRowPartOffset);
+  float* s_tok_scale = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(fbars) + kTokScaleOffset);
   uint32_t* misc = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(bars) + kMiscOffset);
   // misc[0]: tensor-memory base; misc[1]: abort flag; misc[3]: this CTA is the
   // last contributor of its head split tile; misc[5]: some epilogue warp left
@@ -356,14 +457,27 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
 
   if (threadIdx.x == 0) QSPEC_PHASE(0);
   if (threadIdx.x == 0) QSPEC_STAMP(8, 0);
-  if (threadIdx.x == 0) {
-    for (int b = 0; b < kNumBars; ++b) mbar_init(smem_u32(&bars[b]), bar_count(b, C::kEpiWarps));
-    misc[1] = 0;
-    misc[3] = 0;
-    misc[5] = 0;
-    misc[6] = 0;
-    misc[7] = 0;
-    fence_barrier_init();
+  if (warp == 0) {
+    // The 32 lanes of warp 0 initialise the barriers in a compact loop.  (One
+    // thread walking all of them compiled, depending on their number, into a
+    // set-up several microseconds long: +20 to +45 % per decode call.)
+#pragma unroll 1
+    for (int b = lane; b < kNumBars; b += 32) mbar_init(smem_u32(&bars[b]), bar_count(b, C::kEpiWarps));
+    if constexpr (kFused) {
+      if (lane == 0) {
+        mbar_init(smem_u32(scale_ready), 1);
+        mbar_init(smem_u32(row_amax), C::kEpiWarps);
+      }
+    }
+    fence_barrier_init();   // each lane's inits, before the async proxy uses them
+    if (lane == 0) {
+      misc[1] = 0;
+      misc[3] = 0;
+      misc[5] = 0;
+      misc[6] = 0;
+      misc[7] = 0;
+    }
+    __syncwarp();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmap_w);
@@ -397,9 +511,9 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     const long long head_end = (u_end < (t_head + 1) * ku) ? u_end : (t_head + 1) * ku;
     bool head_pending = (u_begin < u_end) && head_end < u_end && u_begin != t_head * ku;
     // The weights may come from the preceding grid unless the caller vouches
-    // otherwise.  W4A4 runs behind its own activation quantization, which
-    // then launches this grid only after the grid before it has completed.
-    if constexpr (!kInt8) {
+    // otherwise.  W4A4 with the activation pre-pass runs behind that kernel,
+    // which then launches this grid only after the grid before it has completed.
+    if constexpr (!kInt8 || kFused) {
       if (!args.weights_ready) grid_dependency_wait();
     }
     // Test hook: a wait that nothing completes runs out, and the CTA gives up
@@ -535,15 +649,43 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     // ------------------------------------------------ activation producer
     grid_dependency_wait();   // activations may come from the preceding kernel
     if (lane == 0) QSPEC_PHASE(10);
+    bool xok = true;
+    if constexpr (kFused) {
+      // Every token row is quantized by the epilogue warps of CTA (row mod
+      // grid), each warp counting its share: wait (bounded) until all M rows
+      // are in the workspace, hand the token scales to the epilogue, and count
+      // this CTA as having seen them; the last CTA to do so returns the
+      // counters to zero for the next call.
+      const uint64_t start = global_timer_ns();
+      for (;;) {
+        uint32_t v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(args.qsync) : "memory");
+        if (v >= static_cast<uint32_t>(args.M * C::kEpiWarps)) break;
+        if (*abort_flag || global_timer_ns() - start > kWaitLimitNs) {
+          if (lane == 0) {
+            *abort_flag = 1;
+            if (args.status) atomicOr(args.status, kDevTimeout);
+          }
+          xok = false;
+          break;
+        }
+        __nanosleep(64);
+      }
+      xok = __all_sync(0xffffffffu, xok);
+      if (lane == 0) QSPEC_PHASE(13);
+      // the codes were written by other CTAs' generic stores; TMA reads them
+      if (xok) asm volatile("fence.proxy.async.global;" ::: "memory");
+    }
     int i = 0;
     UnitCursor cur;
     cur.init(u_begin, ku, args.m_tiles);
-    for (long long u = u_begin; u < u_end; ++u, ++i, cur.next(ku, args.m_tiles)) {
+    for (long long u = u_begin; xok && u < u_end; ++u, ++i, cur.next(ku, args.m_tiles)) {
       const int s = i % NX;
       const uint32_t ph = (i / NX) & 1;
       if (!warp_wait(smem_u32(&x_empty[s]), ph ^ 1, abort_flag, args.status)) break;
       if (elect_one_lane()) {
         mbar_arrive_expect_tx(smem_u32(&x_full[s]), C::kXBytes);
+        if (i == 0) QSPEC_PHASE(14);
 #pragma unroll
         for (int a = 0; a < C::kAtoms; ++a) {
           tma_load_2d(smem_u32(x_buf + s * C::kXBytes + a * MT * 128), &tmap_x,
@@ -553,6 +695,24 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
       }
       __syncwarp();
       QSPEC_STAMP(7, i);
+      if constexpr (kFused) {
+        // Off the critical path (the first activation tiles are on their way):
+        // hand the token scales to the epilogue, and count this CTA as having
+        // seen every row; the last CTA to do so zeroes the counters for the
+        // next call.
+        if (i == 0) {
+          if (lane < args.M) s_tok_scale[lane] = __ldcg(args.s_a + lane);
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(smem_u32(scale_ready));
+            if (atomicAdd(args.qsync + 1, 1u) == gridDim.x - 1) {
+              args.qsync[0] = 0u;
+              args.qsync[1] = 0u;
+            }
+          }
+          __syncwarp();
+        }
+      }
     }
     if (*abort_flag) {
       for (int j = (i > NX ? i - NX : 0); j < i; ++j)
@@ -722,6 +882,27 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     const int G = args.groups_per_row;
     grid_dependency_wait();   // no global write before the preceding grid is done
     if (et == 0) st_release_cta(&misc[7], 1u);   // ... and its tickets are settled
+    bool epi_ok = true;
+    if constexpr (kFused) {
+      // Fused activation quantization: this CTA's epilogue warps together
+      // quantize token rows blockIdx.x, blockIdx.x + grid, ... into the
+      // workspace; each warp counts its share of a row as done (every lane's
+      // stores fenced, then one release of the count), M * kEpiWarps in all.
+      static_assert(C::kEpiWarps <= 4, "row partials for up to 4 epilogue warps");
+      uint32_t rphase = 0;
+      for (long long m = cta; epi_ok && m < args.M; m += grid, ++rphase) {
+        if (et == 0) QSPEC_PHASE(11);
+        epi_ok = quantize_row_team<C::kEpiWarps>(
+            args.x + m * args.K, args.K, args.xq + m * args.K, const_cast<float*>(args.s_a) + m,
+            args.qmax, ew, lane, s_row_part, smem_u32(row_amax), rphase, abort_flag, args.status);
+        __threadfence();
+        __syncwarp();
+        if (epi_ok && lane == 0)
+          asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(args.qsync) : "memory");
+        if (et == 0) QSPEC_PHASE(12);
+      }
+      epi_ok = epi_ok && warp_wait(smem_u32(scale_ready), 0, abort_flag, args.status);
+    }
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
 
     // Group scales come as TMA tiles of 8 groups x 128 rows from the weight
@@ -737,14 +918,15 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     // y rows m0 .. m0+kCols-1 of output column n from run[]
     auto write_y = [&](int n, int m0) {
       if (n >= args.N) return;
-      if constexpr (kInt8) grid_dependency_wait();   // s_a comes from the preceding kernel
+      if constexpr (kInt8 && !kFused) grid_dependency_wait();   // s_a comes from the preceding kernel
 #pragma unroll
       for (int c = 0; c < C::kCols; ++c) {
         const int m = m0 + c;
         if (m < args.M) {
           // int8 mode: run holds 16 x the sums; s_a / 16 is exact and so is
           // the product's rounding relative to the unscaled one
-          const float v = kInt8 ? (args.s_a[m] * 0.0625f) * run[c] : run[c];
+          const float sa = kFused ? s_tok_scale[m] : (kInt8 ? args.s_a[m] : 1.f);
+          const float v = kInt8 ? (sa * 0.0625f) * run[c] : run[c];
           args.y[static_cast<long long>(m) * args.N + n] = v;
         }
       }
@@ -775,7 +957,7 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT>::kThreads, 1)
     const bool head_handoff = (u_begin < u_end) && head_end < u_end && u_begin != t_head * ku;
     RingPos acc;              // accumulator ring position of the next group
     acc.init(0, NACC);
-    bool ok = true;
+    bool ok = epi_ok;
     bool tail_slow = false;   // this warp left its tail-tile share for the ticket
     long long u = u_begin;
     UnitCursor tc;            // the tile of the next segment (no divisions per segment)

@@ -127,6 +127,11 @@ bool gemm_shape_ok(int64_t m, int64_t n, int64_t k, int32_t group) {
   return units < kMaxUnits;
 }
 
+// Decode-sized drafting GEMMs (m <= 32) can quantize their activations in the
+// GEMM kernel itself (QSPEC_GEMM_FUSED_QUANT); otherwise the separate
+// per-token pre-pass kernel does.
+bool fused_act_quant(bool int8_mode, int64_t m) { return int8_mode && m <= 32; }
+
 GemmPlan plan_gemm(bool int8_mode, int64_t m, int64_t n, int64_t k, int sm_count) {
   GemmPlan p;
   p.mt = pick_mt(m);
@@ -155,15 +160,15 @@ GemmPlan plan_gemm(bool int8_mode, int64_t m, int64_t n, int64_t k, int sm_count
   return p;
 }
 
-template <bool kInt8, int MT, bool kDbg>
+template <bool kInt8, int MT, bool kDbg, bool kFused = false>
 qspec_status launch_qgemm_t(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ts,
                             const GemmArgs& a,
                             int grid, int dev, cudaStream_t stream) {
-  using C = GemmCfg<kInt8, MT>;
+  using C = GemmCfg<kInt8, MT, kFused>;
   // Set once per device; concurrent first calls may both set it (idempotent).
   static std::atomic<bool> attr_set[kMaxDevices];
   if (!attr_set[dev].load(std::memory_order_acquire)) {
-    if (cudaFuncSetAttribute(qgemm_kernel<kInt8, MT, kDbg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(qgemm_kernel<kInt8, MT, kDbg, kFused>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess) {
       cudaGetLastError();
       return QSPEC_ERR_CUDA;
@@ -184,7 +189,7 @@ qspec_status launch_qgemm_t(const CUtensorMap& tw, const CUtensorMap& tx, const 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, qgemm_kernel<kInt8, MT, kDbg>, tw, tx, ts, a) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, qgemm_kernel<kInt8, MT, kDbg, kFused>, tw, tx, ts, a) != cudaSuccess) {
     cudaGetLastError();
     return QSPEC_ERR_CUDA;
   }
@@ -192,10 +197,23 @@ qspec_status launch_qgemm_t(const CUtensorMap& tw, const CUtensorMap& tx, const 
 }
 
 template <bool kInt8>
-qspec_status launch_qgemm(int mt, const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ts,
-                          const GemmArgs& a,
+qspec_status launch_qgemm(int mt, bool fused, const CUtensorMap& tw, const CUtensorMap& tx,
+                          const CUtensorMap& ts, const GemmArgs& a,
                           int grid, int dev, cudaStream_t stream) {
   const bool dbg = kInt8 && a.dbg_acc != nullptr;
+  if constexpr (kInt8) {
+    if (fused) {
+      switch (mt) {
+        case 16:
+          return dbg ? launch_qgemm_t<true, 16, true, true>(tw, tx, ts, a, grid, dev, stream)
+                     : launch_qgemm_t<true, 16, false, true>(tw, tx, ts, a, grid, dev, stream);
+        case 32:
+          return dbg ? launch_qgemm_t<true, 32, true, true>(tw, tx, ts, a, grid, dev, stream)
+                     : launch_qgemm_t<true, 32, false, true>(tw, tx, ts, a, grid, dev, stream);
+        default: return QSPEC_ERR_INVALID_ARG;
+      }
+    }
+  }
   switch (mt) {
     case 16:
       return dbg ? launch_qgemm_t<kInt8, 16, kInt8>(tw, tx, ts, a, grid, dev, stream)
@@ -230,7 +248,9 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
                       size_t workspace_bytes, int32_t* dbg_acc, uint32_t flags, void* stream_v,
                       int act_bits = 4) {
   if (!x || !wq || !ws || !y || !workspace) return QSPEC_ERR_INVALID_ARG;
-  if ((flags & ~(QSPEC_GEMM_WEIGHTS_READY | QSPEC_GEMM_TEST_STALL)) != 0u) return QSPEC_ERR_INVALID_ARG;
+  const uint32_t allowed = QSPEC_GEMM_WEIGHTS_READY | QSPEC_GEMM_TEST_STALL |
+                           (kInt8 ? QSPEC_GEMM_FUSED_QUANT : 0u);
+  if ((flags & ~allowed) != 0u) return QSPEC_ERR_INVALID_ARG;
   const bool weights_ready = (flags & QSPEC_GEMM_WEIGHTS_READY) != 0u;
   if (!gemm_shape_ok(m, n, k, group)) return QSPEC_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(wq, 16) || !aligned(ws, 16) || !aligned(y, 4) ||
@@ -264,6 +284,8 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
   a.units = p.units;
   a.weights_ready = weights_ready ? 1 : 0;
   a.test_stall_ns = (flags & QSPEC_GEMM_TEST_STALL) ? 10u * 1000u * 1000u : 0u;   // 10 ms
+  a.qmax = (act_bits == 8) ? 127.f : 7.f;
+  const bool fused = fused_act_quant(kInt8, m) && (flags & QSPEC_GEMM_FUSED_QUANT) != 0u;
   a.ws = ws;
   a.y = y;
   a.dbg_acc = dbg_acc;
@@ -271,7 +293,21 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
   a.counters = reinterpret_cast<uint32_t*>(wsp + p.off_counters);
   a.partials = reinterpret_cast<float*>(wsp + p.off_partials);
   a.s_a = nullptr;
-  if constexpr (kInt8) {
+  a.x = nullptr;
+  a.xq = nullptr;
+  a.qsync = nullptr;
+  if (fused) {
+    // the kernel quantizes the bf16 activations itself, into the same
+    // workspace regions the pre-pass would have written, and reads them back
+    // by TMA; the two counters live in the status block
+    a.x = x;
+    a.xq = reinterpret_cast<int8_t*>(wsp + p.off_xq);
+    a.s_a = reinterpret_cast<float*>(wsp + p.off_sa);
+    a.qsync = reinterpret_cast<uint32_t*>(wsp + 64);
+    if (!make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.xq, m, k, p.mt, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+      return QSPEC_ERR_CUDA;
+  } else if constexpr (kInt8) {
     int8_t* xq = reinterpret_cast<int8_t*>(wsp + p.off_xq);
     float* sa = reinterpret_cast<float*>(wsp + p.off_sa);
     // Also a programmatic dependent: it waits for the preceding grid itself,
@@ -312,7 +348,7 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
   if (!make_tmap(&ts, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, ws, n, scale_row_stride(k / group), kTileN, 8,
                  CU_TENSOR_MAP_SWIZZLE_NONE))
     return QSPEC_ERR_CUDA;
-  return launch_qgemm<kInt8>(p.mt, tw, tx, ts, a, p.grid, dev, stream);
+  return launch_qgemm<kInt8>(p.mt, fused, tw, tx, ts, a, p.grid, dev, stream);
 }
 
 // Launch attributes of the accept kernels, set once per device (concurrent

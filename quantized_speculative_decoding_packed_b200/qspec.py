@@ -31,6 +31,7 @@ EXPORTED = ("qspec_quantize_weights", "qspec_quant_act", "qspec_cast_bf16", "qsp
 ABI_VERSION = 3
 GEMM_WEIGHTS_READY = 1   # flag: wq/ws are not written by work still in flight
 GEMM_TEST_STALL = 0x100  # test hook: the GEMM's first wait runs out (QSPEC_GEMM_TEST_STALL)
+GEMM_FUSED_QUANT = 0x2   # drafting modes, m <= 32: activations quantized inside the GEMM kernel
 
 
 class QSpecError(RuntimeError):

@@ -49,6 +49,28 @@ def test_w4a4_accumulators_exact_and_output(qs, m, n, k, group):
     assert_close_1e3(y.cpu().numpy(), y_ref)
 
 
+@pytest.mark.parametrize("mode", ["w4a4", "w4a8"])
+@pytest.mark.parametrize("m,n,k,group", [s for s in SHAPES if s[0] <= 32] + [(16, 12288, 4096, 128)])
+def test_fused_quantization_exact(qs, mode, m, n, k, group):
+    """Activations quantized inside the GEMM kernel (QSPEC_GEMM_FUSED_QUANT):
+    accumulators bit-exact and outputs within the bar, twice in a row on one
+    workspace (its counters return to zero after every call)."""
+    gi = synth.gemm_inputs("llama3_8b", m, n, k, group, stream=96)
+    wq, ws, q, s_h = _prep(qs, gi)
+    fn = qs.gemm_w4a4 if mode == "w4a4" else qs.gemm_w4a8
+    ref = orc.gemm_w4a4 if mode == "w4a4" else orc.gemm_w4a8
+    op = qs.OP_GEMM_W4A4 if mode == "w4a4" else qs.OP_GEMM_W4A8
+    work = torch.zeros(qs.workspace_size(op, m, n, k, group), dtype=torch.uint8, device="cuda")
+    y_ref, acc = ref(gi.x, q, s_h, group, return_acc=True)
+    for _ in range(2):
+        dbg = torch.zeros((m, n, k // group), dtype=torch.int32, device="cuda")
+        y = fn(cuda_bf16(gi.x_bits), wq, ws, group, dbg_acc=dbg, work=work, flags=qs.GEMM_FUSED_QUANT)
+        torch.cuda.synchronize()
+        assert np.array_equal(dbg.cpu().numpy(), acc)
+        assert_close_1e3(y.cpu().numpy(), y_ref)
+    assert qs.workspace_status(work) == 0
+
+
 @pytest.mark.parametrize("m,n,k,group", SHAPES)
 def test_w4a16_output(qs, m, n, k, group):
     gi = synth.gemm_inputs("llama3_8b", m, n, k, group, stream=98)
