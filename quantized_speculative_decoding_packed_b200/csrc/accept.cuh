@@ -26,10 +26,11 @@
 
 namespace qspec {
 
-// 16 CTAs per sequence (a non-portable cluster size, allowed on B200): at vocab
-// 128256 a CTA's chunk is 32 KB of shared memory, so the 64-sequence batch
-// (1024 CTAs) is resident in one wave.
-constexpr int kAcceptCluster = 16;
+// 8 CTAs per sequence (16, a non-portable size, measured 1.7x slower at vocab
+// 128256, batch 64).
+constexpr int kAcceptCluster = 8;
+// Vocabulary iterations whose loads a thread keeps in flight together.
+constexpr int kAcceptUnroll = 8;
 constexpr int kAcceptThreads = 256;
 
 __device__ __forceinline__ uint64_t fixed_point_weight(float r) {
@@ -135,20 +136,35 @@ __global__ void __cluster_dims__(kAcceptCluster, 1, 1) __launch_bounds__(kAccept
 
   uint64_t total = 0, prefix = 0;
   for (int pass = 0; pass < 2; ++pass) {
-    // Stream this CTA's chunk once: r into shared memory, F summed on the fly.
+    // Stream this CTA's chunk once: r into shared memory, F summed on the
+    // fly; each thread keeps kAcceptUnroll iterations' loads in flight.
     uint64_t part = 0;
-    for (int j = tid * 4; j < len; j += kAcceptThreads * 4) {
-      float4 pv = *reinterpret_cast<const float4*>(prow + lo + j);
-      if (qrow) {
-        const float4 qv = *reinterpret_cast<const float4*>(qrow + lo + j);
-        pv.x = fmaxf(0.f, __fsub_rn(pv.x, qv.x));
-        pv.y = fmaxf(0.f, __fsub_rn(pv.y, qv.y));
-        pv.z = fmaxf(0.f, __fsub_rn(pv.z, qv.z));
-        pv.w = fmaxf(0.f, __fsub_rn(pv.w, qv.w));
+    for (int j0 = tid * 4; j0 < len; j0 += kAcceptThreads * 4 * kAcceptUnroll) {
+      float4 pv[kAcceptUnroll], qv[kAcceptUnroll];
+#pragma unroll
+      for (int t = 0; t < kAcceptUnroll; ++t) {
+        const int j = j0 + t * kAcceptThreads * 4;
+        if (j < len) {
+          pv[t] = __ldcs(reinterpret_cast<const float4*>(prow + lo + j));
+          if (qrow) qv[t] = __ldcs(reinterpret_cast<const float4*>(qrow + lo + j));
+        }
       }
-      *reinterpret_cast<float4*>(r_s + j) = pv;
-      part += fixed_point_weight(pv.x) + fixed_point_weight(pv.y) + fixed_point_weight(pv.z) +
-              fixed_point_weight(pv.w);
+#pragma unroll
+      for (int t = 0; t < kAcceptUnroll; ++t) {
+        const int j = j0 + t * kAcceptThreads * 4;
+        if (j < len) {
+          float4 v = pv[t];
+          if (qrow) {
+            v.x = fmaxf(0.f, __fsub_rn(v.x, qv[t].x));
+            v.y = fmaxf(0.f, __fsub_rn(v.y, qv[t].y));
+            v.z = fmaxf(0.f, __fsub_rn(v.z, qv[t].z));
+            v.w = fmaxf(0.f, __fsub_rn(v.w, qv[t].w));
+          }
+          *reinterpret_cast<float4*>(r_s + j) = v;
+          part += fixed_point_weight(v.x) + fixed_point_weight(v.y) + fixed_point_weight(v.z) +
+                  fixed_point_weight(v.w);
+        }
+      }
     }
     const uint64_t mine = block_sum_u64(part, sh.red);
     if (tid == 0) sh.chunk_sum[pass] = mine;
@@ -268,14 +284,27 @@ __global__ void __cluster_dims__(kAcceptCluster, 1, 1) __launch_bounds__(kAccept
   bool bad = false;
   for (int i = 0; i <= gamma; ++i) {
     const float* row = p + (static_cast<int64_t>(b) * (gamma + 1) + i) * vocab + lo;
-    // thread-local scan: increasing indices, strict '>' keeps the first maximum
+    // thread-local scan: increasing indices, strict '>' keeps the first
+    // maximum; kAcceptUnroll iterations' loads in flight together
     ArgMax best{-__int_as_float(0x7f800000), 0x7fffffff};
-    for (int j = tid * 4; j < len; j += kAcceptThreads * 4) {
-      const float4 v = *reinterpret_cast<const float4*>(row + j);
-      if (v.x > best.v) best = ArgMax{v.x, lo + j};
-      if (v.y > best.v) best = ArgMax{v.y, lo + j + 1};
-      if (v.z > best.v) best = ArgMax{v.z, lo + j + 2};
-      if (v.w > best.v) best = ArgMax{v.w, lo + j + 3};
+    for (int j0 = tid * 4; j0 < len; j0 += kAcceptThreads * 4 * kAcceptUnroll) {
+      float4 vv[kAcceptUnroll];
+#pragma unroll
+      for (int t = 0; t < kAcceptUnroll; ++t) {
+        const int j = j0 + t * kAcceptThreads * 4;
+        if (j < len) vv[t] = __ldcs(reinterpret_cast<const float4*>(row + j));
+      }
+#pragma unroll
+      for (int t = 0; t < kAcceptUnroll; ++t) {
+        const int j = j0 + t * kAcceptThreads * 4;
+        if (j < len) {
+          const float4 v = vv[t];
+          if (v.x > best.v) best = ArgMax{v.x, lo + j};
+          if (v.y > best.v) best = ArgMax{v.y, lo + j + 1};
+          if (v.z > best.v) best = ArgMax{v.z, lo + j + 2};
+          if (v.w > best.v) best = ArgMax{v.w, lo + j + 3};
+        }
+      }
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {

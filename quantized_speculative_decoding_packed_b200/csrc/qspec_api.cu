@@ -353,16 +353,12 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
 
 // Launch attributes of the accept kernels, set once per device (concurrent
 // first calls may both set them; idempotent): the residual sampler's dynamic
-// shared memory, and the 16-CTA clusters of both kernels.
+// shared memory.
 bool accept_attrs_set(int dev) {
   static std::atomic<bool> done[kMaxDevices];
   if (done[dev].load(std::memory_order_acquire)) return true;
   if (cudaFuncSetAttribute(spec_accept_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           204800) != cudaSuccess ||
-      cudaFuncSetAttribute(spec_accept_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
-          cudaSuccess ||
-      cudaFuncSetAttribute(greedy_accept_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed,
-                           1) != cudaSuccess) {
+                           204800) != cudaSuccess) {
     cudaGetLastError();
     return false;
   }
