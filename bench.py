@@ -143,6 +143,15 @@ def accept_bytes(n_acc, gamma, vocab):
     return total
 
 
+def greedy_bytes(n_acc, gamma, vocab):
+    """Per sequence (greedy rule): the draft tokens it compares, rows 0..n of p
+    (the first mismatch's row, or the bonus row when all match), plus the outputs."""
+    total = 0
+    for n in n_acc:
+        total += min(int(n) + 1, gamma) * 4 + (int(n) + 1) * vocab * 4 + (gamma + 2) * 4
+    return total
+
+
 def step_work(layers):
     b = 0
     ops = 0
@@ -773,6 +782,23 @@ def accept_report(torch, qspec, peaks, sigmas=(0.1, 0.5, 1.0), batch=64, gamma=5
         t = statistics.median(ts)
         na = n_acc.cpu().numpy()
         byts = accept_bytes(na, gamma, vocab)
+        # the greedy rule on the same target rows and drafts
+        tg = []
+        for rep in range(8):
+            flush.fill_(rep & 0xFF)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            ng, _ = qspec.spec_accept_greedy(p, draft, work=work)
+            e1.record()
+            e1.synchronize()
+            if rep >= 2:
+                tg.append(e0.elapsed_time(e1) * 1e-3)
+        if qspec.workspace_status(work) != 0:
+            raise RuntimeError("greedy accept kernel reported bad input")
+        t_g = statistics.median(tg)
+        ng = ng.cpu().numpy()
+        byts_g = greedy_bytes(ng, gamma, vocab)
         # near-tie count over the positions the rule tested
         idx = draft.long().unsqueeze(-1)
         pv = p[:, :gamma].gather(2, idx).squeeze(-1).double()
@@ -784,7 +810,11 @@ def accept_report(torch, qspec, peaks, sigmas=(0.1, 0.5, 1.0), batch=64, gamma=5
                                  "mean_accepted": float(na.mean()),
                                  "acceptance_per_position": float(
                                      (na.sum()) / (na.sum() + (na < gamma).sum())),
-                                 "near_ties": int(near.sum())}
+                                 "near_ties": int(near.sum()),
+                                 "greedy": {"us": t_g * 1e6, "bytes": byts_g,
+                                            "gbs": byts_g / t_g / 1e9,
+                                            "frac_hbm": byts_g / t_g / 1e9 / hbm,
+                                            "mean_accepted": float(ng.mean())}}
         del p, q
     del flush
     torch.cuda.empty_cache()
@@ -792,7 +822,8 @@ def accept_report(torch, qspec, peaks, sigmas=(0.1, 0.5, 1.0), batch=64, gamma=5
                         "target logits N(0, 2^2), draft = target + N(0, sigma^2)",
             "timing": "each call alone between CUDA events, L2 flushed (256 MB write) before it",
             "bytes": "per sequence: 2 gathered elements per tested position + one vocab row of p "
-                     "and q (rejection) or of p (all accepted) + outputs",
+                     "and q (rejection) or of p (all accepted) + outputs; greedy: the compared "
+                     "drafts + rows 0..n of p + outputs",
             "peak_hbm_gbs": hbm, "sigmas": out}
 
 

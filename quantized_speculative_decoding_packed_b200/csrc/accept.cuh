@@ -13,10 +13,13 @@
 // the order in which the vocabulary is summed.
 //
 // Layout on B200: one cluster of kAcceptCluster CTAs per sequence.  Each CTA
-// streams one contiguous chunk of the row(s) from HBM once, keeps r in shared
-// memory, and publishes its chunk total; the CTAs read each other's totals
-// through distributed shared memory, and the CTA whose chunk holds the
-// threshold finds the token with a block scan over its shared-memory copy.
+// streams one contiguous chunk of the row(s) from HBM once (each warp a
+// contiguous sub-chunk, coalesced), records the F sums of its blocks of 128 x
+// k floats in shared memory and publishes its chunk total; the CTAs read each
+// other's totals through distributed shared memory, and the CTA whose chunk
+// holds the threshold locates it among its recorded sums and re-reads only
+// that block (an L2 hit) to find the token.  Without a copy of the chunk in
+// shared memory a batch of 64 sequences (512 CTAs) is resident in one wave.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -29,8 +32,10 @@ namespace qspec {
 // 8 CTAs per sequence (16, a non-portable size, measured 1.7x slower at vocab
 // 128256, batch 64).
 constexpr int kAcceptCluster = 8;
-// Vocabulary iterations whose loads a thread keeps in flight together.
+// Vocabulary iterations whose loads a thread keeps in flight together (the
+// sampler keeps fewer: it runs four CTAs per SM, so within 64 registers).
 constexpr int kAcceptUnroll = 8;
+constexpr int kSampleUnroll = 4;
 constexpr int kAcceptThreads = 256;
 
 __device__ __forceinline__ uint64_t fixed_point_weight(float r) {
@@ -58,27 +63,59 @@ __device__ __forceinline__ uint64_t fixed_point_threshold(float u, uint64_t s) {
   return (lo >> shift) | (hi << (64 - shift));
 }
 
-__device__ __forceinline__ uint64_t block_sum_u64(uint64_t v, uint64_t* red) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-  const int w = threadIdx.x >> 5;
-  if ((threadIdx.x & 31) == 0) red[w] = v;
-  __syncthreads();
-  uint64_t t = 0;
-#pragma unroll
-  for (int i = 0; i < kAcceptThreads / 32; ++i) t += red[i];
-  __syncthreads();
-  return t;
-}
+// Block sums recorded per warp: a warp's sub-chunk is read as iterations of
+// 128 floats (one float4 per lane), and every AcceptSplit::per_blk
+// consecutive iterations (kSampleUnroll up to a vocabulary of 8 x 8 x 64 x 128
+// x kSampleUnroll) form one recorded block.
+constexpr int kAcceptWarps = kAcceptThreads / 32;
+constexpr int kAcceptMaxBlocks = 64;
 
 struct AcceptShared {
   uint64_t chunk_sum[2];                    // per pass; read by the other CTAs of the cluster
-  uint64_t red[kAcceptThreads / 32];
+  uint64_t red[kAcceptWarps];               // this CTA's warp totals
+  uint64_t blk[kAcceptWarps][kAcceptMaxBlocks];
   int n_acc;
   int token;
 };
 
-__global__ void __cluster_dims__(kAcceptCluster, 1, 1) __launch_bounds__(kAcceptThreads)
+__device__ __forceinline__ uint64_t warp_sum_u64(uint64_t v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+__device__ __forceinline__ uint64_t warp_incl_scan_u64(uint64_t v, int lane) {
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint64_t o = __shfl_up_sync(0xffffffffu, v, off);
+    if (lane >= off) v += o;
+  }
+  return v;
+}
+
+// Split of a CTA's chunk of `len` floats (a multiple of 4) among its warps:
+// warp w owns [w * wlen, min(len, (w + 1) * wlen)), read in `its` iterations
+// of 128 floats, recorded in blocks of `per_blk` iterations.
+struct AcceptSplit {
+  int wlen, its, per_blk;
+  __device__ __forceinline__ void init(int len) {
+    wlen = ((len + 4 * kAcceptWarps - 1) / (4 * kAcceptWarps)) * 4;
+    its = (wlen + 127) / 128;
+    // at least kSampleUnroll iterations per block: one warp reduction per
+    // batch of loads
+    per_blk = (its + kAcceptMaxBlocks - 1) / kAcceptMaxBlocks;
+    if (per_blk < kSampleUnroll) per_blk = kSampleUnroll;
+  }
+};
+
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__global__ void __cluster_dims__(kAcceptCluster, 1, 1) __launch_bounds__(kAcceptThreads, 4)
     spec_accept_kernel(const float* __restrict__ p, const float* __restrict__ q,
                        const int32_t* __restrict__ draft, const float* __restrict__ u_acc,
                        const float* __restrict__ u_res, int gamma, int vocab, int chunk,
@@ -86,12 +123,12 @@ __global__ void __cluster_dims__(kAcceptCluster, 1, 1) __launch_bounds__(kAccept
                        uint32_t* __restrict__ status) {
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
-  extern __shared__ __align__(16) float r_s[];
   __shared__ AcceptShared sh;
 
   const int b = blockIdx.x / kAcceptCluster;
   const int crank = static_cast<int>(cluster.block_rank());
   const int tid = threadIdx.x;
+  const int lane = tid & 31, wid = tid >> 5;
 
   // Phase 1: ratio test at every draft position at once (lane i of the first
   // warp takes position i: one round of scattered reads instead of gamma
@@ -123,6 +160,10 @@ __global__ void __cluster_dims__(kAcceptCluster, 1, 1) __launch_bounds__(kAccept
   const int lo = crank * chunk;
   const int hi = min(vocab, lo + chunk);
   const int len = max(0, hi - lo);
+  AcceptSplit sp;
+  sp.init(len);
+  const int w0 = min(len, wid * sp.wlen);
+  const int w1 = min(len, w0 + sp.wlen);
 
   const float* prow;
   const float* qrow;
@@ -133,40 +174,67 @@ __global__ void __cluster_dims__(kAcceptCluster, 1, 1) __launch_bounds__(kAccept
     prow = p + (static_cast<int64_t>(b) * (gamma + 1) + gamma) * vocab;
     qrow = nullptr;
   }
+  // r at chunk offset j (a multiple of 4), four at a time
+  auto r4 = [&](int j) {
+    float4 v = __ldcg(reinterpret_cast<const float4*>(prow + lo + j));
+    if (qrow) {
+      const float4 w = __ldcg(reinterpret_cast<const float4*>(qrow + lo + j));
+      v.x = fmaxf(0.f, __fsub_rn(v.x, w.x));
+      v.y = fmaxf(0.f, __fsub_rn(v.y, w.y));
+      v.z = fmaxf(0.f, __fsub_rn(v.z, w.z));
+      v.w = fmaxf(0.f, __fsub_rn(v.w, w.w));
+    }
+    return v;
+  };
 
-  uint64_t total = 0, prefix = 0;
+  uint64_t total = 0, prefix = 0, mine = 0;
   for (int pass = 0; pass < 2; ++pass) {
-    // Stream this CTA's chunk once: r into shared memory, F summed on the
-    // fly; each thread keeps kAcceptUnroll iterations' loads in flight.
-    uint64_t part = 0;
-    for (int j0 = tid * 4; j0 < len; j0 += kAcceptThreads * 4 * kAcceptUnroll) {
-      float4 pv[kAcceptUnroll], qv[kAcceptUnroll];
+    // Stream this CTA's chunk once, each warp its own sub-chunk, coalesced
+    // (lane l reads floats 4l..4l+3 of each 128), kSampleUnroll iterations'
+    // loads in flight; record the warp's F sum per block of iterations.
+    uint64_t wsum = 0, lsum = 0;
+    for (int k0 = 0; k0 < sp.its; k0 += kSampleUnroll) {
+      float4 pv[kSampleUnroll], qv[kSampleUnroll];
 #pragma unroll
-      for (int t = 0; t < kAcceptUnroll; ++t) {
-        const int j = j0 + t * kAcceptThreads * 4;
-        if (j < len) {
+      for (int t = 0; t < kSampleUnroll; ++t) {
+        const int j = w0 + (k0 + t) * 128 + lane * 4;
+        if (k0 + t < sp.its && j < w1) {
           pv[t] = __ldcs(reinterpret_cast<const float4*>(prow + lo + j));
           if (qrow) qv[t] = __ldcs(reinterpret_cast<const float4*>(qrow + lo + j));
         }
       }
 #pragma unroll
-      for (int t = 0; t < kAcceptUnroll; ++t) {
-        const int j = j0 + t * kAcceptThreads * 4;
-        if (j < len) {
-          float4 v = pv[t];
-          if (qrow) {
-            v.x = fmaxf(0.f, __fsub_rn(v.x, qv[t].x));
-            v.y = fmaxf(0.f, __fsub_rn(v.y, qv[t].y));
-            v.z = fmaxf(0.f, __fsub_rn(v.z, qv[t].z));
-            v.w = fmaxf(0.f, __fsub_rn(v.w, qv[t].w));
+      for (int t = 0; t < kSampleUnroll; ++t) {
+        const int it = k0 + t;
+        if (it < sp.its) {   // warp-uniform
+          const int j = w0 + it * 128 + lane * 4;
+          uint64_t f = 0;
+          if (j < w1) {
+            float4 v = pv[t];
+            if (qrow) {
+              v.x = fmaxf(0.f, __fsub_rn(v.x, qv[t].x));
+              v.y = fmaxf(0.f, __fsub_rn(v.y, qv[t].y));
+              v.z = fmaxf(0.f, __fsub_rn(v.z, qv[t].z));
+              v.w = fmaxf(0.f, __fsub_rn(v.w, qv[t].w));
+            }
+            f = fixed_point_weight(v.x) + fixed_point_weight(v.y) + fixed_point_weight(v.z) +
+                fixed_point_weight(v.w);
           }
-          *reinterpret_cast<float4*>(r_s + j) = v;
-          part += fixed_point_weight(v.x) + fixed_point_weight(v.y) + fixed_point_weight(v.z) +
-                  fixed_point_weight(v.w);
+          lsum += f;
+          if ((it + 1) % sp.per_blk == 0 || it + 1 == sp.its) {
+            const uint64_t bsum = warp_sum_u64(lsum);
+            if (lane == 0) sh.blk[wid][it / sp.per_blk] = bsum;
+            wsum += bsum;
+            lsum = 0;
+          }
         }
       }
     }
-    const uint64_t mine = block_sum_u64(part, sh.red);
+    if (lane == 0) sh.red[wid] = wsum;
+    __syncthreads();
+    mine = 0;
+#pragma unroll
+    for (int w = 0; w < kAcceptWarps; ++w) mine += sh.red[w];
     if (tid == 0) sh.chunk_sum[pass] = mine;
     cluster.sync();
     total = 0;
@@ -181,50 +249,79 @@ __global__ void __cluster_dims__(kAcceptCluster, 1, 1) __launch_bounds__(kAccept
     // Empty residual (possible only through fp32 rounding): draw from p[b][n].
     prow = p + (static_cast<int64_t>(b) * (gamma + 1) + n) * vocab;
     qrow = nullptr;
-    __syncthreads();
   }
+  // Done with the other CTAs' shared memory (they wait for this arrival
+  // before exiting, so theirs stays readable until here).
+  cluster_arrive_release();
 
-  // The CTA whose chunk holds the threshold finds the token: per-thread
-  // contiguous sub-ranges of the shared-memory copy, an exclusive scan of
-  // their sums, then a sequential search inside the one sub-range that
-  // straddles the threshold.
-  __syncthreads();
-  if (total != 0) {
-    const int per = (len + kAcceptThreads - 1) / kAcceptThreads;
-    const int a0 = min(len, tid * per);
-    const int a1 = min(len, a0 + per);
-    uint64_t s = 0;
-    for (int j = a0; j < a1; ++j) s += fixed_point_weight(r_s[j]);
-    // Exclusive scan of the per-thread sums: inclusive scans inside each warp
-    // by shuffles, then the warp totals (exact integer sums, any order).
-    const int lane = tid & 31, wid = tid >> 5;
-    uint64_t incl = s;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const uint64_t o = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += o;
-    }
-    if (lane == 31) sh.red[wid] = incl;
-    __syncthreads();
-    uint64_t warp_base = 0;
-#pragma unroll
-    for (int w = 0; w < kAcceptThreads / 32; ++w)
-      if (w < wid) warp_base += sh.red[w];
+  // The CTA whose chunk holds the threshold T draws the token: its first warp
+  // finds the warp sub-chunk and the recorded block holding T, then re-reads
+  // that one block (from L2) and finds the lane and the element.
+  if (total != 0 && wid == 0) {
     uint64_t t = fixed_point_threshold(u_res[b], total);
     if (t >= total) t = total - 1;
-    const uint64_t base = prefix + warp_base + (incl - s);
-    if (s != 0 && base <= t && t < base + s) {
-      uint64_t c = base;
-      for (int j = a0; j < a1; ++j) {
-        c += fixed_point_weight(r_s[j]);
-        if (c > t) {
-          sh.token = lo + j;
-          break;
+    if (prefix <= t && t < prefix + mine) {
+      // warp sub-chunk: lanes 0..7 hold the warp totals
+      uint64_t v = (lane < kAcceptWarps) ? sh.red[lane] : 0;
+      uint64_t incl = warp_incl_scan_u64(v, lane);
+      uint32_t hit = __ballot_sync(0xffffffffu, lane < kAcceptWarps && prefix + incl > t);
+      const int ws = hit ? __ffs(hit) - 1 : 0;   // T < prefix + mine: always a hit
+      uint64_t base = prefix + __shfl_sync(0xffffffffu, incl - v, ws);
+      // recorded block inside that sub-chunk
+      const int sw0 = min(len, ws * sp.wlen), sw1 = min(len, sw0 + sp.wlen);
+      const int nblk = (sp.its + sp.per_blk - 1) / sp.per_blk;
+      int blk = -1;
+      for (int b0 = 0; b0 < nblk && blk < 0; b0 += 32) {
+        v = (b0 + lane < nblk) ? sh.blk[ws][b0 + lane] : 0;
+        incl = warp_incl_scan_u64(v, lane);
+        hit = __ballot_sync(0xffffffffu, b0 + lane < nblk && base + incl > t);
+        if (hit) {
+          const int l = __ffs(hit) - 1;
+          blk = b0 + l;
+          base += __shfl_sync(0xffffffffu, incl - v, l);
+        } else {
+          base += __shfl_sync(0xffffffffu, incl, 31);
+        }
+      }
+      // re-read the block's iterations (loads of kSampleUnroll of them in
+      // flight) and walk them in order
+      const int it1 = min(sp.its, (blk + 1) * sp.per_blk);
+      bool done = blk < 0;
+      for (int i0 = blk * sp.per_blk; !done && i0 < it1; i0 += kSampleUnroll) {
+        float4 rv[kSampleUnroll];
+#pragma unroll
+        for (int u = 0; u < kSampleUnroll; ++u) {
+          const int j = sw0 + (i0 + u) * 128 + lane * 4;
+          rv[u] = (i0 + u < it1 && j < sw1) ? r4(j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < kSampleUnroll; ++u) {
+          if (done || i0 + u >= it1) break;   // warp-uniform
+          const float e[4] = {rv[u].x, rv[u].y, rv[u].z, rv[u].w};
+          const uint64_t s = fixed_point_weight(e[0]) + fixed_point_weight(e[1]) +
+                             fixed_point_weight(e[2]) + fixed_point_weight(e[3]);
+          incl = warp_incl_scan_u64(s, lane);
+          hit = __ballot_sync(0xffffffffu, base + incl > t);
+          if (hit) {
+            if (lane == __ffs(hit) - 1) {
+              const int j = sw0 + (i0 + u) * 128 + lane * 4;
+              uint64_t c = base + incl - s;
+#pragma unroll
+              for (int e4 = 0; e4 < 4; ++e4) {
+                c += fixed_point_weight(e[e4]);
+                if (c > t) {
+                  tokens[static_cast<int64_t>(b) * (gamma + 1) + n] = lo + j + e4;
+                  break;
+                }
+              }
+            }
+            done = true;
+          } else {
+            base += __shfl_sync(0xffffffffu, incl, 31);
+          }
         }
       }
     }
-    __syncthreads();
-    if (tid == 0 && sh.token >= 0) tokens[static_cast<int64_t>(b) * (gamma + 1) + n] = sh.token;
   }
 
   if (crank == 0) {
@@ -234,8 +331,7 @@ __global__ void __cluster_dims__(kAcceptCluster, 1, 1) __launch_bounds__(kAccept
     }
     if (tid == 0) n_accepted[b] = n;
   }
-  // Keep this CTA's shared memory alive until every CTA of the cluster has read it.
-  cluster.sync();
+  cluster_wait_acquire();
 }
 
 // ---------------------------------------------------------------------------

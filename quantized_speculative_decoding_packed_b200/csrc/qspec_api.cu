@@ -351,21 +351,6 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
   return launch_qgemm<kInt8>(p.mt, fused, tw, tx, ts, a, p.grid, dev, stream);
 }
 
-// Launch attributes of the accept kernels, set once per device (concurrent
-// first calls may both set them; idempotent): the residual sampler's dynamic
-// shared memory.
-bool accept_attrs_set(int dev) {
-  static std::atomic<bool> done[kMaxDevices];
-  if (done[dev].load(std::memory_order_acquire)) return true;
-  if (cudaFuncSetAttribute(spec_accept_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           204800) != cudaSuccess) {
-    cudaGetLastError();
-    return false;
-  }
-  done[dev].store(true, std::memory_order_release);
-  return true;
-}
-
 }  // namespace
 }  // namespace qspec
 
@@ -477,13 +462,10 @@ qspec_status qspec_spec_accept(const float* p, const float* q, const int32_t* dr
     return QSPEC_ERR_INVALID_ARG;
   if (workspace && (workspace_bytes < 256 || !aligned(workspace, 16)))
     return QSPEC_ERR_WORKSPACE_TOO_SMALL;
-  int dev = 0;
-  qspec_status st = current_device(&dev, nullptr);
+  qspec_status st = current_device(nullptr, nullptr);
   if (st != QSPEC_OK) return st;
   const int chunk = ((vocab + 4 * kAcceptCluster - 1) / (4 * kAcceptCluster)) * 4;
-  const size_t smem = static_cast<size_t>(chunk) * 4;
-  if (!accept_attrs_set(dev)) return QSPEC_ERR_CUDA;
-  spec_accept_kernel<<<batch * kAcceptCluster, kAcceptThreads, smem,
+  spec_accept_kernel<<<batch * kAcceptCluster, kAcceptThreads, 0,
                        static_cast<cudaStream_t>(stream)>>>(
       p, q, draft, u_acc, u_res, gamma, vocab, chunk, n_accepted, tokens,
       static_cast<uint32_t*>(workspace));
@@ -502,10 +484,8 @@ qspec_status qspec_spec_accept_greedy(const float* p, const int32_t* draft, int3
     return QSPEC_ERR_INVALID_ARG;
   if (workspace && (workspace_bytes < 256 || !aligned(workspace, 16)))
     return QSPEC_ERR_WORKSPACE_TOO_SMALL;
-  int dev = 0;
-  qspec_status st = current_device(&dev, nullptr);
+  qspec_status st = current_device(nullptr, nullptr);
   if (st != QSPEC_OK) return st;
-  if (!accept_attrs_set(dev)) return QSPEC_ERR_CUDA;
   const int chunk = ((vocab + 4 * kAcceptCluster - 1) / (4 * kAcceptCluster)) * 4;
   greedy_accept_kernel<<<batch * kAcceptCluster, kAcceptThreads, 0,
                          static_cast<cudaStream_t>(stream)>>>(

@@ -53,6 +53,16 @@ def test_accept_bytes_closed_forms(gamma, vocab):
     assert bench.accept_bytes([0, gamma], gamma, vocab) == reject_first + accept_all
 
 
+@pytest.mark.parametrize("gamma,vocab", [(4, 32000), (5, 128256)])
+def test_greedy_bytes_closed_forms(gamma, vocab):
+    out = (gamma + 2) * 4
+    first_mismatch = 1 * 4 + 1 * vocab * 4 + out          # draft 0 compared, row 0 read
+    all_match = gamma * 4 + (gamma + 1) * vocab * 4 + out  # every draft compared, rows 0..gamma
+    assert bench.greedy_bytes([0], gamma, vocab) == first_mismatch
+    assert bench.greedy_bytes([gamma], gamma, vocab) == all_match
+    assert bench.greedy_bytes([0, gamma], gamma, vocab) == first_mismatch + all_match
+
+
 def test_job_throughput_is_whole_job():
     one = bench.job_throughput(1e9, 1, 10.0)
     assert one == pytest.approx(100.0)                  # 1 GB in 10 ms = 100 GB/s
