@@ -39,8 +39,9 @@ constexpr int kSampleUnroll = 4;
 constexpr int kAcceptThreads = 256;
 
 __device__ __forceinline__ uint64_t fixed_point_weight(float r) {
-  // r * 2^62 is exact in fp64; truncation toward zero is floor for r >= 0.
-  return (r > 0.f) ? __double2ull_rz(static_cast<double>(r) * 4611686018427387904.0) : 0ull;
+  // r * 2^62 only moves the exponent (exact in fp32 for 0 <= r < 4); the
+  // conversion truncates toward zero, which is floor for r >= 0.
+  return (r > 0.f) ? __float2ull_rz(__fmul_rn(r, 4611686018427387904.0f)) : 0ull;
 }
 
 // floor(u * s) for an fp32 u in [0, 1), computed exactly with a 128-bit product.
