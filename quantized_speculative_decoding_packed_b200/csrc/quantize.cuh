@@ -4,6 +4,7 @@
 // All decisions are taken in IEEE fp32 with round-to-nearest-even:
 //   weights:     s = absmax / 7, s_h = fp16(s), q = clamp(rint(w / s_h), -8, 7)
 //   activations: s_a = absmax / 7, inv = 7 / absmax, q = clamp(rint(x * inv), -8, 7)
+//                (the clamp never binds for finite x; codes of non-finite x are unspecified)
 // The explicit __fdiv_rn / __fmul_rn intrinsics pin the rounding regardless of
 // compiler flags and forbid contraction into FMAs.
 #pragma once
@@ -118,26 +119,31 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
   // longer rows read the rest again.
   constexpr int kCache = 8;
   uint4 cache[kCache];
-  auto absmax8 = [](const uint4& u, float m) {
+  // |x| max on bf16 pairs: clear both sign bits, then one packed bf16 max
+  // (a max is exact in any format, so this equals the fp32 max of |x|).
+  auto absmax8 = [](const uint4& u, __nv_bfloat162 m) {
     const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      m = fmaxf(m, fabsf(bf16_bits_to_float(w4[j] & 0xFFFFu)));
-      m = fmaxf(m, fabsf(bf16_bits_to_float(w4[j] >> 16)));
+      const uint32_t b = w4[j] & 0x7FFF7FFFu;
+      __nv_bfloat162 v;
+      memcpy(&v, &b, 4);
+      m = __hmax2(m, v);
     }
     return m;
   };
-  float a = 0.f;
+  __nv_bfloat162 m2 = __float2bfloat162_rn(0.f);
 #pragma unroll
   for (int j = 0; j < kCache; ++j) {
     const int64_t c = (static_cast<int64_t>(tid) + 256 * j) * 8;
     if (c < k) {
       cache[j] = *reinterpret_cast<const uint4*>(xr + c);
-      a = absmax8(cache[j], a);
+      m2 = absmax8(cache[j], m2);
     }
   }
   for (int64_t c = (static_cast<int64_t>(tid) + 256 * kCache) * 8; c < k; c += 256 * 8)
-    a = absmax8(*reinterpret_cast<const uint4*>(xr + c), a);
+    m2 = absmax8(*reinterpret_cast<const uint4*>(xr + c), m2);
+  float a = fmaxf(__low2float(m2), __high2float(m2));
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
   if ((tid & 31) == 0) red[tid >> 5] = a;
@@ -149,37 +155,47 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
   static_assert(!kPacked || kQMax == 7, "packed output holds 4-bit codes");
   constexpr float kLevels = static_cast<float>(kQMax);
   const float s = __fdiv_rn(a, kLevels);
-  const float inv = __fdiv_rn(kLevels, a);
+  // an all-zero row quantizes to zeros: inv = 0 gives t = 0 for every element
+  const float inv = (a == 0.f) ? 0.f : __fdiv_rn(kLevels, a);
   if (tid == 0) scales[row] = s;
-  auto clamp_code = [](int v) { return v < -kQMax - 1 ? -kQMax - 1 : (v > kQMax ? kQMax : v); };
 
+  // t = x * inv rounded to fp32, then rint(t) by adding 1.5 x 2^23: for
+  // |t| < 2^22 the sum lies where the float spacing is 1, so it rounds t to
+  // the nearest integer, ties to even (1.5 x 2^23 is even), and the sum's bit
+  // pattern is 0x4B400000 + rint(t): its low byte is the two's-complement
+  // code.  For finite x, |t| <= kQMax (1 + 2^-23), so rint(t) already lies in
+  // [-kQMax, kQMax] and no clamp is needed.
+  auto code_bits = [inv](float v) {
+    return __float_as_uint(__fadd_rn(__fmul_rn(v, inv), 12582912.0f));
+  };
+  // bytes [a.0, b.0, c.0, d.0]
+  auto low_bytes = [](uint32_t a4, uint32_t b4, uint32_t c4, uint32_t d4) {
+    return __byte_perm(__byte_perm(a4, b4, 0x0040), __byte_perm(c4, d4, 0x0040), 0x5410);
+  };
   auto emit = [&](int64_t c, const uint4& u) {
     const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-    int q[8];
+    uint32_t e[8];   // element 2j: low half of word j, element 2j + 1: high half
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const float lo = bf16_bits_to_float(w4[j] & 0xFFFFu);
-      const float hi = bf16_bits_to_float(w4[j] >> 16);
-      q[2 * j] = (a == 0.f) ? 0 : clamp_code(__float2int_rn(__fmul_rn(lo, inv)));
-      q[2 * j + 1] = (a == 0.f) ? 0 : clamp_code(__float2int_rn(__fmul_rn(hi, inv)));
+      e[2 * j] = code_bits(__uint_as_float(w4[j] << 16));
+      e[2 * j + 1] = code_bits(__uint_as_float(w4[j] & 0xFFFF0000u));
     }
     if constexpr (kPacked) {
-      uint32_t p = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) p |= (static_cast<uint32_t>(q[j]) & 0xFu) << (4 * j);
-      *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(out) + row * (k / 2) + c / 2) = p;
+      // nibble j = code j; bytes -> nibbles: byte i's low nibble joins byte
+      // i - 1's high nibble, then bytes 0 and 2 of each half are kept
+      uint32_t lo = low_bytes(e[0], e[1], e[2], e[3]) & 0x0F0F0F0Fu;
+      uint32_t hi = low_bytes(e[4], e[5], e[6], e[7]) & 0x0F0F0F0Fu;
+      lo |= lo >> 4;
+      hi |= hi >> 4;
+      *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(out) + row * (k / 2) + c / 2) =
+          __byte_perm(lo, hi, 0x6420);
     } else {
       // int8 operand for the GEMM, each block of 8 channels stored in the
       // order (0,2,4,6,1,3,5,7): the GEMM widens packed weight nibbles into
       // the same order with masks alone, and a dot product does not depend
       // on the order of its terms.
-      uint32_t ev = 0, od = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        ev |= (static_cast<uint32_t>(q[2 * j]) & 0xFFu) << (8 * j);
-        od |= (static_cast<uint32_t>(q[2 * j + 1]) & 0xFFu) << (8 * j);
-      }
-      *reinterpret_cast<uint2*>(static_cast<int8_t*>(out) + row * k + c) = make_uint2(ev, od);
+      *reinterpret_cast<uint2*>(static_cast<int8_t*>(out) + row * k + c) =
+          make_uint2(low_bytes(e[0], e[2], e[4], e[6]), low_bytes(e[1], e[3], e[5], e[7]));
     }
   };
 #pragma unroll
