@@ -58,6 +58,19 @@ def test_ragged_sizes_identical(qs, b, g, v):
     assert np.array_equal(n, n_ref) and np.array_equal(tok, tok_ref)
 
 
+@pytest.mark.parametrize("sigma", [0.3, 3.0])
+def test_largest_vocab_identical(qs, sigma):
+    """The largest vocabulary the entry points accept (409600): the most blocks a warp records."""
+    ai = synth.accept_inputs(synth.rng_for("accept", 18, int(10 * sigma)), 3, 4, 409600, 2.0, sigma)
+    n, tok = _run(qs, ai)
+    n_ref, tok_ref = orc.spec_accept(ai.p, ai.q, ai.draft, ai.u_acc, ai.u_res)
+    assert np.array_equal(n, n_ref) and np.array_equal(tok, tok_ref)
+    p, draft = synth.greedy_inputs(synth.rng_for("accept", 19, int(10 * sigma)), ai.p, follow=0.7)
+    n, tok = _run_greedy(qs, p, draft)
+    n_ref, tok_ref = orc.greedy_accept(p, draft)
+    assert np.array_equal(n, n_ref) and np.array_equal(tok, tok_ref)
+
+
 def test_p_equals_q_accepts_all_and_draws_bonus(qs):
     ai = synth.accept_inputs(synth.rng_for("accept", 12), 8, 5, 5000, 2.0, 0.5)
     ai.q = ai.p[:, :5, :].copy()
