@@ -137,7 +137,9 @@ qspec_status qspec_quant_act(const uint16_t* x, int64_t m, int64_t k, uint8_t* x
  *  y   [m][ldy] fp32, the previous layer's output; its first k columns are read.
  *  x   [m][k] bf16 bit patterns out.
  * Requires m >= 1, k >= 8 and a multiple of 8, ldy >= k and a multiple of 4,
- * y and x 16-byte aligned.
+ * y and x 16-byte aligned.  Launched as a programmatic dependent of the
+ * preceding kernel on the stream (it reads y only after that kernel has
+ * completed), so the kernel after it may launch while it waits.
  */
 qspec_status qspec_cast_bf16(const float* y, int64_t m, int64_t ldy, int64_t k, uint16_t* x,
                              void* stream);

@@ -416,8 +416,20 @@ qspec_status qspec_cast_bf16(const float* y, int64_t m, int64_t ldy, int64_t k, 
   const long long threads = m * (k / 8);
   const long long blocks = (threads + 255) / 256;
   if (blocks > 0x7FFFFFFFll) return QSPEC_ERR_INVALID_ARG;
-  cast_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      y, m, ldy, k, x);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.blockDim = dim3(256);
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, cast_bf16_kernel, y, static_cast<int64_t>(m), static_cast<int64_t>(ldy),
+                         static_cast<int64_t>(k), x) != cudaSuccess) {
+    cudaGetLastError();
+    return QSPEC_ERR_CUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? QSPEC_OK : QSPEC_ERR_CUDA;
 }
 

@@ -211,10 +211,14 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
 // Glue between chained linear layers: x[i][j] = bf16_RN(y[i][j]) for j < k,
 // the next layer's bf16 input from a layer's fp32 output (its first k
 // columns, row stride ldy).  One thread per 8 outputs: two 16-byte loads, one
-// 16-byte store.
+// 16-byte store.  Launched as a programmatic dependent: it lets the next
+// kernel launch at once, then waits for the preceding grid (complete, memory
+// flushed) before it reads y or writes x.
 __global__ void __launch_bounds__(256) cast_bf16_kernel(const float* __restrict__ y, int64_t m,
                                                         int64_t ldy, int64_t k,
                                                         uint16_t* __restrict__ x) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int64_t per_row = k / 8;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t >= m * per_row) return;
