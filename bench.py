@@ -890,7 +890,9 @@ def chained_round_report(torch, qspec, peaks, wq, ws, L, x16, p, q, draft, u_acc
     t_round = _graph_time_per_call(torch, [round_], reps=5)
     if qspec.workspace_status(work) != 0:
         raise RuntimeError("device status reported a fault in the chained round")
-    glue = sum((GAMMA * M_DRAFT + M_VERIFY) * k * (4 + 2)
+    # chained inputs: a drafting quantizer reads 4 bytes (fp32) instead of 2 per
+    # element; the verifying pass's cast reads 4 and writes 2
+    glue = sum((GAMMA * M_DRAFT * 2 + M_VERIFY * (4 + 2)) * k
                for (wq_, _) in layers[1:] for k in (wq_.shape[1] * 2,))
     byts = bytes_unchained + glue
     # mode switch: layer-0 gate_up weights, W4A4 at M=16 and W4A16 at M=80
@@ -907,7 +909,9 @@ def chained_round_report(torch, qspec, peaks, wq, ws, L, x16, p, q, draft, u_acc
                         "-> gate_up -> first 11008 columns -> down -> next layer), gamma="
                         f"{GAMMA} W4A4 drafting passes at M={M_DRAFT} from their own inputs, one "
                         f"W4A16 verifying pass at M={M_VERIFY}, accept B={BATCH} V={VOCAB}",
-            "glue": "qspec_cast_bf16 between consecutive GEMMs (fp32 output -> bf16 input)",
+            "glue": "drafting passes: the next W4A4 call reads the previous fp32 output and "
+                    "rounds it to bf16 in its activation quantizer (qspec_gemm_w4a4_f32in); "
+                    "verifying pass: qspec_cast_bf16 between consecutive GEMMs",
             "ms_per_round": t_round * 1e3, "bytes": byts, "gbs": byts / t_round / 1e9,
             "frac_hbm": byts / t_round / 1e9 / hbm,
             "ms_per_round_unchained": ms_unchained,

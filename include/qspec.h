@@ -187,6 +187,26 @@ qspec_status qspec_gemm_w4a8(const uint16_t* x, int64_t m, int64_t k, const uint
                              uint32_t flags, void* stream);
 
 /*
+ * The drafting GEMMs on a chained layer's fp32 output: the activations are
+ * x[i][j] = bf16(xf[i][j]) (round to nearest even) for i < m, j < k, rounded
+ * as the per-token quantizer reads them, so no separate bf16 copy (and no
+ * qspec_cast_bf16 launch) is needed between layers.  The result is
+ * bit-identical to qspec_cast_bf16 followed by qspec_gemm_w4a4 (resp. _w4a8).
+ *  xf   [m][ldx] fp32, 16-byte aligned; its first k columns are read.
+ *  ldx  row stride in elements: ldx >= k, a multiple of 4.
+ * Other arguments, workspace size (QSPEC_OP_GEMM_W4A4 resp. _W4A8) and
+ * errors as for qspec_gemm_w4a4; QSPEC_GEMM_FUSED_QUANT is not accepted here.
+ */
+qspec_status qspec_gemm_w4a4_f32in(const float* xf, int64_t ldx, int64_t m, int64_t k,
+                                   const uint8_t* wq, const uint16_t* ws, int64_t n, int32_t group,
+                                   float* y, void* workspace, size_t workspace_bytes,
+                                   int32_t* dbg_acc, uint32_t flags, void* stream);
+qspec_status qspec_gemm_w4a8_f32in(const float* xf, int64_t ldx, int64_t m, int64_t k,
+                                   const uint8_t* wq, const uint16_t* ws, int64_t n, int32_t group,
+                                   float* y, void* workspace, size_t workspace_bytes,
+                                   int32_t* dbg_acc, uint32_t flags, void* stream);
+
+/*
  * W4A16 verifying GEMM: y = x . deq(wq, ws)^T with bf16 activations and the
  * same packed weights as the drafting mode (QSpec abstract: "high-precision
  * weight-only quantization for accurate verification").  deq = q * s_h is
@@ -309,8 +329,9 @@ size_t qspec_workspace_size(int32_t op, int64_t m, int64_t n, int64_t k, int32_t
 qspec_status qspec_workspace_status(void* workspace, void* stream);
 
 /* Version of this ABI (3: adds QSPEC_GEMM_TEST_STALL, qspec_gemm_w4a8, qspec_cast_bf16,
- * qspec_spec_accept_greedy and qspec_gemm_w4a16_noalloc_status). */
-#define QSPEC_ABI_VERSION 3
+ * qspec_spec_accept_greedy and qspec_gemm_w4a16_noalloc_status; 4: adds
+ * qspec_gemm_w4a4_f32in and qspec_gemm_w4a8_f32in). */
+#define QSPEC_ABI_VERSION 4
 int32_t qspec_abi_version(void);
 
 /* Static, human-readable name of a status code. */

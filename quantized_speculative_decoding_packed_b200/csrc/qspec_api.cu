@@ -242,19 +242,22 @@ qspec_status launch_qgemm(int mt, bool fused, const CUtensorMap& tw, const CUten
 
 // kInt8: the drafting modes (integer MMA on per-token activation codes of
 // act_bits = 4 (W4A4) or 8 (W4A8)); else the W4A16 verifying mode.
+// xf (drafting modes only): fp32 input [m][ldx] instead of bf16 x, rounded
+// to bf16 as the activation quantizer reads it.
 template <bool kInt8>
 qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,
                       const uint16_t* ws, int64_t n, int32_t group, float* y, void* workspace,
                       size_t workspace_bytes, int32_t* dbg_acc, uint32_t flags, void* stream_v,
-                      int act_bits = 4) {
-  if (!x || !wq || !ws || !y || !workspace) return QSPEC_ERR_INVALID_ARG;
+                      int act_bits = 4, const float* xf = nullptr, int64_t ldx = 0) {
+  if ((!x && !xf) || !wq || !ws || !y || !workspace) return QSPEC_ERR_INVALID_ARG;
   const uint32_t allowed = QSPEC_GEMM_WEIGHTS_READY | QSPEC_GEMM_TEST_STALL |
-                           (kInt8 ? QSPEC_GEMM_FUSED_QUANT : 0u);
+                           ((kInt8 && !xf) ? QSPEC_GEMM_FUSED_QUANT : 0u);
   if ((flags & ~allowed) != 0u) return QSPEC_ERR_INVALID_ARG;
   const bool weights_ready = (flags & QSPEC_GEMM_WEIGHTS_READY) != 0u;
   if (!gemm_shape_ok(m, n, k, group)) return QSPEC_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(wq, 16) || !aligned(ws, 16) || !aligned(y, 4) ||
-      !aligned(workspace, 16) || (dbg_acc && !aligned(dbg_acc, 4)))
+  if (xf && (!kInt8 || ldx < k || (ldx % 4) != 0 || ldx > (1ll << 40) / m)) return QSPEC_ERR_INVALID_ARG;
+  if ((x && !aligned(x, 16)) || (xf && !aligned(xf, 16)) || !aligned(wq, 16) || !aligned(ws, 16) ||
+      !aligned(y, 4) || !aligned(workspace, 16) || (dbg_acc && !aligned(dbg_acc, 4)))
     return QSPEC_ERR_INVALID_ARG;
   int dev = 0;
   DeviceInfo info;
@@ -324,12 +327,22 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
     qc.numAttrs = 1;
     void* qout = xq;
     const int early = weights_ready ? 1 : 0;
-    const cudaError_t qe =
-        (act_bits == 8)
-            ? cudaLaunchKernelEx(&qc, quant_act_kernel<false, 127>, x, static_cast<int64_t>(k), qout,
-                                 sa, early)
-            : cudaLaunchKernelEx(&qc, quant_act_kernel<false, 7>, x, static_cast<int64_t>(k), qout,
-                                 sa, early);
+    const void* xin = xf ? static_cast<const void*>(xf) : static_cast<const void*>(x);
+    const int64_t ld = xf ? ldx : k;
+    cudaError_t qe;
+    if (xf) {
+      qe = (act_bits == 8)
+               ? cudaLaunchKernelEx(&qc, quant_act_kernel<false, 127, true>, xin, ld,
+                                    static_cast<int64_t>(k), qout, sa, early)
+               : cudaLaunchKernelEx(&qc, quant_act_kernel<false, 7, true>, xin, ld,
+                                    static_cast<int64_t>(k), qout, sa, early);
+    } else {
+      qe = (act_bits == 8)
+               ? cudaLaunchKernelEx(&qc, quant_act_kernel<false, 127>, xin, ld,
+                                    static_cast<int64_t>(k), qout, sa, early)
+               : cudaLaunchKernelEx(&qc, quant_act_kernel<false, 7>, xin, ld,
+                                    static_cast<int64_t>(k), qout, sa, early);
+    }
     if (qe != cudaSuccess) {
       cudaGetLastError();
       return QSPEC_ERR_CUDA;
@@ -401,7 +414,7 @@ qspec_status qspec_quant_act(const uint16_t* x, int64_t m, int64_t k, uint8_t* x
   qspec_status st = current_device(nullptr, nullptr);
   if (st != QSPEC_OK) return st;
   quant_act_kernel<true><<<static_cast<unsigned>(m), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      x, k, xq, xs, 0);
+      x, k, k, xq, xs, 0);
   return cudaGetLastError() == cudaSuccess ? QSPEC_OK : QSPEC_ERR_CUDA;
 }
 
@@ -447,6 +460,22 @@ qspec_status qspec_gemm_w4a8(const uint16_t* x, int64_t m, int64_t k, const uint
                              uint32_t flags, void* stream) {
   return run_gemm<true>(x, m, k, wq, ws, n, group, y, workspace, workspace_bytes, dbg_acc, flags,
                         stream, 8);
+}
+
+qspec_status qspec_gemm_w4a4_f32in(const float* x, int64_t ldx, int64_t m, int64_t k,
+                                   const uint8_t* wq, const uint16_t* ws, int64_t n, int32_t group,
+                                   float* y, void* workspace, size_t workspace_bytes,
+                                   int32_t* dbg_acc, uint32_t flags, void* stream) {
+  return run_gemm<true>(nullptr, m, k, wq, ws, n, group, y, workspace, workspace_bytes, dbg_acc,
+                        flags, stream, 4, x, ldx);
+}
+
+qspec_status qspec_gemm_w4a8_f32in(const float* x, int64_t ldx, int64_t m, int64_t k,
+                                   const uint8_t* wq, const uint16_t* ws, int64_t n, int32_t group,
+                                   float* y, void* workspace, size_t workspace_bytes,
+                                   int32_t* dbg_acc, uint32_t flags, void* stream) {
+  return run_gemm<true>(nullptr, m, k, wq, ws, n, group, y, workspace, workspace_bytes, dbg_acc,
+                        flags, stream, 8, x, ldx);
 }
 
 qspec_status qspec_gemm_w4a16(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq,

@@ -80,14 +80,16 @@ __device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) {
 // streams into its tensor-core operand tiles).  kQMax: 7 for the 4-bit codes
 // of the W4A4 drafter, 127 for the 8-bit codes of the W4A8 drafting variant
 // (s_a = absmax / kQMax, inv = kQMax / absmax, q clamped to [-kQMax-1, kQMax]).
-template <bool kPacked, int kQMax = 7>
-__global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restrict__ x,
+// kF32In: x holds fp32 values (a layer's output, row stride ldx) and each one
+// is first rounded to bf16 (nearest even): the bf16 glue of chained layers
+// folded into the read.  Otherwise x holds bf16 bit patterns, row stride ldx.
+template <bool kPacked, int kQMax = 7, bool kF32In = false>
+__global__ void __launch_bounds__(256) quant_act_kernel(const void* __restrict__ x, int64_t ldx,
                                                         int64_t k, void* __restrict__ out,
                                                         float* __restrict__ scales,
                                                         int early_trigger) {
   __shared__ float red[8];
   const int64_t row = blockIdx.x;
-  const uint16_t* xr = x + row * k;
   const int tid = threadIdx.x;
   constexpr unsigned kTraceKind = 3u;   // trace builds: event-log tags
   const unsigned trace_launch = static_cast<unsigned>(reinterpret_cast<uintptr_t>(out) >> 8);
@@ -110,9 +112,26 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   }
   if (tid == 0) QSPEC_PHASE(1);
-  if (!QSPEC_ALIGN_OK(reinterpret_cast<uintptr_t>(xr), 16) ||
+  const uint16_t* xr = static_cast<const uint16_t*>(x) + row * ldx;
+  const float* xfr = static_cast<const float*>(x) + row * ldx;
+  if (!QSPEC_ALIGN_OK(kF32In ? reinterpret_cast<uintptr_t>(xfr) : reinterpret_cast<uintptr_t>(xr), 16) ||
       !QSPEC_ALIGN_OK(reinterpret_cast<uintptr_t>(out), 8))
     return;
+  // elements c .. c+7 of the row as 8 bf16 bit patterns (element 2j in the
+  // low half of word j)
+  auto load8 = [&](int64_t c) {
+    if constexpr (kF32In) {
+      const float4 a = *reinterpret_cast<const float4*>(xfr + c);
+      const float4 b = *reinterpret_cast<const float4*>(xfr + c + 4);
+      auto two = [](float lo, float hi) {
+        return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(lo))) |
+               (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(hi))) << 16);
+      };
+      return make_uint4(two(a.x, a.y), two(a.z, a.w), two(b.x, b.y), two(b.z, b.w));
+    } else {
+      return *reinterpret_cast<const uint4*>(xr + c);
+    }
+  };
 
   // Each thread's chunks of 8 elements stay in registers between the two
   // passes (up to kCache chunks: rows of up to 16384 elements are read once);
@@ -137,12 +156,12 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
   for (int j = 0; j < kCache; ++j) {
     const int64_t c = (static_cast<int64_t>(tid) + 256 * j) * 8;
     if (c < k) {
-      cache[j] = *reinterpret_cast<const uint4*>(xr + c);
+      cache[j] = load8(c);
       m2 = absmax8(cache[j], m2);
     }
   }
   for (int64_t c = (static_cast<int64_t>(tid) + 256 * kCache) * 8; c < k; c += 256 * 8)
-    m2 = absmax8(*reinterpret_cast<const uint4*>(xr + c), m2);
+    m2 = absmax8(load8(c), m2);
   float a = fmaxf(__low2float(m2), __high2float(m2));
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
@@ -204,7 +223,7 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
     if (c < k) emit(c, cache[j]);
   }
   for (int64_t c = (static_cast<int64_t>(tid) + 256 * kCache) * 8; c < k; c += 256 * 8)
-    emit(c, *reinterpret_cast<const uint4*>(xr + c));
+    emit(c, load8(c));
   if (tid == 0) QSPEC_PHASE(8);
 }
 

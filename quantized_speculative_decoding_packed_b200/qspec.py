@@ -28,7 +28,7 @@ EXPORTED = ("qspec_quantize_weights", "qspec_quant_act", "qspec_cast_bf16", "qsp
             "qspec_workspace_status",
             "qspec_status_string", "qspec_gemm_w4a16_noalloc", "qspec_gemm_w4a16_noalloc_status",
             "qspec_abi_version")
-ABI_VERSION = 3
+ABI_VERSION = 4
 GEMM_WEIGHTS_READY = 1   # flag: wq/ws are not written by work still in flight
 GEMM_TEST_STALL = 0x100  # test hook: the GEMM's first wait runs out (QSPEC_GEMM_TEST_STALL)
 GEMM_FUSED_QUANT = 0x2   # drafting modes, m <= 32: activations quantized inside the GEMM kernel
@@ -53,6 +53,8 @@ def _load() -> ctypes.CDLL:
     lib.qspec_cast_bf16.argtypes = [P, I64, I64, I64, P, P]
     lib.qspec_gemm_w4a4.argtypes = [P, I64, I64, P, P, I64, I32, P, P, SZ, P, U32, P]
     lib.qspec_gemm_w4a8.argtypes = [P, I64, I64, P, P, I64, I32, P, P, SZ, P, U32, P]
+    lib.qspec_gemm_w4a4_f32in.argtypes = [P, I64, I64, I64, P, P, I64, I32, P, P, SZ, P, U32, P]
+    lib.qspec_gemm_w4a8_f32in.argtypes = [P, I64, I64, I64, P, P, I64, I32, P, P, SZ, P, U32, P]
     lib.qspec_gemm_w4a16.argtypes = [P, I64, I64, P, P, I64, I32, P, P, SZ, U32, P]
     lib.qspec_gemm_w4a16_noalloc.argtypes = [P, I64, I64, P, P, I64, I32, P, U32, P]
     lib.qspec_gemm_w4a16_noalloc_status.argtypes = [P]
@@ -66,7 +68,7 @@ def _load() -> ctypes.CDLL:
     lib.qspec_status_string.argtypes = [I32]
     lib.qspec_status_string.restype = ctypes.c_char_p
     for name in ("qspec_quantize_weights", "qspec_quant_act", "qspec_cast_bf16", "qspec_gemm_w4a4",
-                 "qspec_gemm_w4a8",
+                 "qspec_gemm_w4a8", "qspec_gemm_w4a4_f32in", "qspec_gemm_w4a8_f32in",
                  "qspec_gemm_w4a16", "qspec_spec_accept", "qspec_spec_accept_greedy",
                  "qspec_workspace_status",
                  "qspec_gemm_w4a16_noalloc", "qspec_gemm_w4a16_noalloc_status"):
@@ -182,8 +184,9 @@ def linear_chain(x0: torch.Tensor, layers, mode: str = "w4a4", group: int = 128,
                  ys=None, xs=None, work: torch.Tensor | None = None, stream=None,
                  weights_ready: bool = False):
     """Runs linear layers back to back on one token batch: layer j's input is
-    the first K_j columns of layer j-1's fp32 output, rounded to bf16 by
-    qspec_cast_bf16.  layers: [(wq, ws)]; mode: w4a4 | w4a8 | w4a16.  ys/xs:
+    the first K_j columns of layer j-1's fp32 output, rounded to bf16 (by the
+    drafting GEMMs' quantizer as it reads them, or by qspec_cast_bf16 for the
+    verifying GEMM).  layers: [(wq, ws)]; mode: w4a4 | w4a8 | w4a16.  ys/xs:
     optional preallocated outputs / intermediate inputs (for CUDA-graph
     capture).  Returns the list of fp32 outputs."""
     gemm = {"w4a4": gemm_w4a4, "w4a8": gemm_w4a8, "w4a16": gemm_w4a16}[mode]
@@ -192,7 +195,9 @@ def linear_chain(x0: torch.Tensor, layers, mode: str = "w4a4", group: int = 128,
     x = x0
     for j, (wq, ws) in enumerate(layers):
         n, k = wq.shape[0], wq.shape[1] * 2
-        if j:
+        if j and mode != "w4a16":
+            x = outs[-1][:, :k]
+        elif j:
             x = cast_bf16(outs[-1], k, x=None if xs is None else xs[j], stream=stream)
         y = None if ys is None else ys[j]
         outs.append(gemm(x, wq, ws, group, y=y, work=work, stream=stream, weights_ready=weights_ready))
@@ -209,18 +214,7 @@ def gemm_w4a4(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor, group: int = 
     running (sets QSPEC_GEMM_WEIGHTS_READY; the weights then stream while the
     preceding kernel finishes).  flags: further QSPEC_GEMM_* bits.
     """
-    _need(x, torch.bfloat16, "x")
-    m, k = x.shape
-    n = wq.shape[0]
-    if y is None:
-        y = torch.empty((m, n), dtype=torch.float32, device=x.device)
-    need = workspace_size(OP_GEMM_W4A4, m, n, k, group)
-    if work is None:
-        work = workspace(need, x.device)
-    _check(LIB.qspec_gemm_w4a4(_ptr(x), m, k, _ptr(wq), _ptr(ws), n, group, _ptr(y), _ptr(work),
-                               work.numel(), _ptr(dbg_acc), _flags(weights_ready, flags),
-                               _stream(stream)), "qspec_gemm_w4a4")
-    return y
+    return _drafting("w4a4", x, wq, ws, group, y, work, dbg_acc, stream, weights_ready, flags)
 
 
 def gemm_w4a8(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor, group: int = 128,
@@ -228,17 +222,33 @@ def gemm_w4a8(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor, group: int = 
               dbg_acc: torch.Tensor | None = None, stream=None,
               weights_ready: bool = False, flags: int = 0) -> torch.Tensor:
     """W4A8 drafting variant: y[M][N] fp32 = quant8(x) . deq(wq, ws)^T (arguments as gemm_w4a4)."""
-    _need(x, torch.bfloat16, "x")
+    return _drafting("w4a8", x, wq, ws, group, y, work, dbg_acc, stream, weights_ready, flags)
+
+
+def _drafting(mode, x, wq, ws, group, y, work, dbg_acc, stream, weights_ready, flags):
+    """The drafting GEMMs: x bf16 [M][K] (contiguous), or fp32 [M][K] with unit column
+    stride (e.g. the first K columns of a layer's output), rounded to bf16 as it is
+    quantized (qspec_gemm_*_f32in)."""
     m, k = x.shape
     n = wq.shape[0]
+    op = OP_GEMM_W4A4 if mode == "w4a4" else OP_GEMM_W4A8
     if y is None:
         y = torch.empty((m, n), dtype=torch.float32, device=x.device)
-    need = workspace_size(OP_GEMM_W4A8, m, n, k, group)
+    need = workspace_size(op, m, n, k, group)
     if work is None:
         work = workspace(need, x.device)
-    _check(LIB.qspec_gemm_w4a8(_ptr(x), m, k, _ptr(wq), _ptr(ws), n, group, _ptr(y), _ptr(work),
-                               work.numel(), _ptr(dbg_acc), _flags(weights_ready, flags),
-                               _stream(stream)), "qspec_gemm_w4a8")
+    fl = _flags(weights_ready, flags)
+    if x.dtype == torch.float32:
+        if not x.is_cuda or x.stride(1) != 1:
+            raise ValueError("fp32 x must be a CUDA tensor with unit column stride")
+        fn = LIB.qspec_gemm_w4a4_f32in if mode == "w4a4" else LIB.qspec_gemm_w4a8_f32in
+        _check(fn(_ptr(x), x.stride(0), m, k, _ptr(wq), _ptr(ws), n, group, _ptr(y), _ptr(work),
+                  work.numel(), _ptr(dbg_acc), fl, _stream(stream)), f"qspec_gemm_{mode}_f32in")
+        return y
+    _need(x, torch.bfloat16, "x")
+    fn = LIB.qspec_gemm_w4a4 if mode == "w4a4" else LIB.qspec_gemm_w4a8
+    _check(fn(_ptr(x), m, k, _ptr(wq), _ptr(ws), n, group, _ptr(y), _ptr(work), work.numel(),
+              _ptr(dbg_acc), fl, _stream(stream)), f"qspec_gemm_{mode}")
     return y
 
 

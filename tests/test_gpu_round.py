@@ -3,7 +3,8 @@
 One Llama-2-7B-shaped layer (fused QKV -> o_proj -> gate+up -> down), run as
 gamma drafting passes (W4A4 at M = 16, each pass its own seeded input) and
 one verifying pass (W4A16 at M = 16 (gamma + 1)), every layer fed the
-previous layer's fp32 output cast to bf16 by the library's glue kernel, then
+previous layer's fp32 output rounded to bf16 (by the drafting GEMMs' quantizer
+as it reads it, by the library's glue kernel before the verifying GEMM), then
 the accept / resample step.  The oracle runs the same chain from the same
 inputs on its own.
 
@@ -46,6 +47,33 @@ def test_cast_glue_is_bit_exact(qs):
     got = x.view(torch.int16).cpu().numpy().view(np.uint16)
     want = (orc.round_to_bf16(y[:, :136]).view(np.uint32) >> 16).astype(np.uint16)
     assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("mode", ["w4a4", "w4a8"])
+@pytest.mark.parametrize("m,k,ldx,n", [(16, 4096, 12288, 1024), (5, 1024, 1028, 300), (33, 640, 640, 128)])
+def test_f32_input_drafting_equals_cast_then_gemm(qs, mode, m, k, ldx, n):
+    """The drafting GEMMs on a layer's fp32 output (a column slice of it) give bit-identical
+    accumulators and outputs to qspec_cast_bf16 followed by the bf16-input call, and
+    match the oracle's quantize-after-rounding chain."""
+    rng = synth.rng_for("llama2_7b", 62, m, k, ldx)
+    yprev = (rng.standard_normal((m, ldx)) * 3.0).astype(np.float32)
+    yprev[:, 7] *= 40.0                                   # an outlier channel
+    w = synth.layer_weights("llama2_7b", n, k, stream=63)
+    wq, ws = qs.quantize_weights(cuda_f32(w), 128)
+    gemm = qs.gemm_w4a4 if mode == "w4a4" else qs.gemm_w4a8
+    G = k // 128
+    yf = cuda_f32(yprev)
+    acc_a = torch.zeros((m, n, G), dtype=torch.int32, device="cuda")
+    acc_b = torch.zeros((m, n, G), dtype=torch.int32, device="cuda")
+    out_a = gemm(yf[:, :k], wq, ws, 128, dbg_acc=acc_a)
+    out_b = gemm(qs.cast_bf16(yf, k), wq, ws, 128, dbg_acc=acc_b)
+    torch.cuda.synchronize()
+    assert torch.equal(acc_a, acc_b)
+    assert torch.equal(out_a.view(torch.int32), out_b.view(torch.int32))
+    q_ref, s_ref = orc.quantize_weights(w, 128)
+    x_ref = orc.round_to_bf16(yprev[:, :k])
+    y_ref = (orc.gemm_w4a4 if mode == "w4a4" else orc.gemm_w4a8)(x_ref, q_ref, s_ref, 128)
+    assert_close_1e3(out_a.cpu().numpy(), y_ref)
 
 
 def test_chained_round_matches_oracle(qs):

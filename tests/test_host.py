@@ -29,12 +29,13 @@ def test_header_declares_the_boundary():
     for name in ("qspec_quantize_weights", "qspec_quant_act", "qspec_gemm_w4a4",
                  "qspec_gemm_w4a16", "qspec_spec_accept", "qspec_workspace_size",
                  "qspec_workspace_status", "qspec_status_string", "qspec_abi_version",
-                 "qspec_spec_accept_greedy", "qspec_gemm_w4a16_noalloc_status"):
+                 "qspec_spec_accept_greedy", "qspec_gemm_w4a16_noalloc_status",
+                 "qspec_gemm_w4a4_f32in", "qspec_gemm_w4a8_f32in"):
         assert name in syms
 
 
 def test_abi_version(lib):
-    assert lib.LIB.qspec_abi_version() == lib.ABI_VERSION == 3
+    assert lib.LIB.qspec_abi_version() == lib.ABI_VERSION == 4
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -84,6 +85,18 @@ def test_gemm_rejects_reserved_flags(lib):
     assert lib.LIB.qspec_gemm_w4a4(FAKE, 4, 256, FAKE, FAKE, 256, 64, FAKE, FAKE, 1 << 30, None,
                                    0x80000000, None) == 1
     assert lib.LIB.qspec_gemm_w4a16_noalloc(FAKE, 4, 256, FAKE, FAKE, 256, 64, FAKE, 4, None) == 1
+
+
+@pytest.mark.parametrize("fn", ["qspec_gemm_w4a4_f32in", "qspec_gemm_w4a8_f32in"])
+def test_f32_input_gemm_rejects(lib, fn):
+    f = getattr(lib.LIB, fn)
+    ok = (FAKE, 256, 4, 256, FAKE, FAKE, 256, 64, FAKE, FAKE, 1 << 30, None)
+    assert f(FAKE, 252, *ok[2:], 0, None) == 1            # ldx < k
+    assert f(FAKE, 258, *ok[2:], 0, None) == 1            # ldx not a multiple of 4
+    assert f(ctypes.c_void_p(0x10008), *ok[1:], 0, None) == 1   # x not 16-byte aligned
+    assert f(None, *ok[1:], 0, None) == 1                 # no input
+    assert f(*ok, 2, None) == 1                           # QSPEC_GEMM_FUSED_QUANT not accepted here
+    assert f(FAKE, 256, 4, 255, *ok[4:], 0, None) == 1    # k not a multiple of the group
 
 
 @pytest.mark.parametrize("b,g,v", [(0, 4, 32), (2, 0, 32), (2, 17, 32), (2, 4, 30), (2, 4, 0),
