@@ -22,20 +22,6 @@ static __device__ unsigned int* g_qspec_trace = nullptr;
       __threadfence_system();                                                           \
     }                                                                                   \
   } while (0)
-// Timeline stamps (SM clock, low 32 bits) per event and unit, kept in shared
-// memory (one st.shared each) and copied to [cta][16][64] at kernel exit.
-static __device__ unsigned long long* g_qspec_timeline = nullptr;
-#define QSPEC_STAMP_DECL __shared__ unsigned int s_qspec_stamps[16 * 64];
-#define QSPEC_STAMP(ev, unit)                                                           \
-  do {                                                                                  \
-    if ((unit) < 64) s_qspec_stamps[(ev) * 64 + (unit)] = static_cast<unsigned>(clock64()); \
-  } while (0)
-#define QSPEC_STAMP_FLUSH()                                                             \
-  do {                                                                                  \
-    if (g_qspec_timeline)                                                               \
-      for (int q_ = threadIdx.x; q_ < 16 * 64; q_ += blockDim.x)                        \
-        g_qspec_timeline[blockIdx.x * 1024u + q_] = s_qspec_stamps[q_];                 \
-  } while (0)
 // Coarse phase events (global timer, ns, comparable across SMs and launches),
 // appended to a log: {time, kind << 56 | launch << 32 | cta << 16 | event}.
 // `kTraceKind` names the kernel and `trace_launch` (24 bits) the launch; each
@@ -63,15 +49,8 @@ constexpr unsigned kQspecEventCap = 1u << 20;
   do {                       \
   } while (0)
 #define QSPEC_ALIGN_OK(addr, a) true
-#define QSPEC_STAMP(ev, unit) \
-  do {                        \
-  } while (0)
 #define QSPEC_PHASE(ev) \
   do {                  \
-  } while (0)
-#define QSPEC_STAMP_DECL
-#define QSPEC_STAMP_FLUSH() \
-  do {                      \
   } while (0)
 #endif
 

@@ -64,11 +64,7 @@ constexpr int kTileN = 128;                      // weight rows per tile (MMA M)
 __host__ __device__ constexpr int unit_k(bool int8_mode) { return int8_mode ? 256 : 128; }
 constexpr int kConvTeamWarps = 4;                // a converter team: one warp per lane quadrant
 constexpr int kCtlWarps = 4;
-#ifdef QSPEC_TRACE
-constexpr int kSmemLimit = 232448 - 4096;        // trace builds keep 4 KB of static stamps
-#else
 constexpr int kSmemLimit = 232448;               // sm_100 dynamic shared memory per CTA
-#endif
 constexpr int kMaxGrid = 1024;                   // ticket slots in the workspace
 constexpr int kMaxPk = 24, kMaxA = 8, kMaxAcc = 8, kMaxX = 8;
 // Group scales arrive by TMA, 8 groups x 128 rows (2 KB) per tile, into a ring.
@@ -399,7 +395,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kFused>::kThreads, 1)
   (void)kTraceKind;
   (void)trace_launch;
   extern __shared__ uint8_t smem_raw[];
-  QSPEC_STAMP_DECL
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* pk_buf = smem;
@@ -456,7 +451,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kFused>::kThreads, 1)
                          unit_owner(tail_u0 + ku - 1, units, grid) == cta + 1;
 
   if (threadIdx.x == 0) QSPEC_PHASE(0);
-  if (threadIdx.x == 0) QSPEC_STAMP(8, 0);
   if (warp == 0) {
     // The 32 lanes of warp 0 initialise the barriers in a compact loop.  (One
     // thread walking all of them compiled, depending on their number, into a
@@ -494,7 +488,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kFused>::kThreads, 1)
   const uint32_t tmem_base = misc[0];
   QSPEC_TRACE_AT(tmem_base & 0xFFFF);
   if (threadIdx.x == 0) QSPEC_PHASE(1);
-  if (threadIdx.x == 0) QSPEC_STAMP(8, 1);
   // The next grid may be scheduled as SMs free up; it waits for this one to
   // complete before it reads inputs or writes anything.
   if (threadIdx.x == 0) grid_launch_dependents();
@@ -538,7 +531,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kFused>::kThreads, 1)
     for (long long u = u_begin; run && u < u_end; ++u, ++i, cur.next(ku, args.m_tiles)) {
       const int s = i % NPK;
       const uint32_t ph = (i / NPK) & 1;
-      QSPEC_STAMP(13, i);
       if (!warp_wait(smem_u32(&pk_empty[s]), ph ^ 1, abort_flag, args.status)) break;
       if (elect_one_lane()) {
         mbar_arrive_expect_tx(smem_u32(&pk_full[s]), C::kPkBytes);
@@ -548,7 +540,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kFused>::kThreads, 1)
         if (u + 1 == u_end) QSPEC_PHASE(9);
       }
       __syncwarp();
-      QSPEC_STAMP(0, i);
       const int g0 = cur.kc * gpu;
       if (u == u_begin || (g0 & (kScaleTileGroups - 1)) == 0) {
         if (!warp_wait(smem_u32(&sc_empty[rs.slot]), rs.phase ^ 1u, abort_flag, args.status)) break;
@@ -694,7 +685,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kFused>::kThreads, 1)
         }
       }
       __syncwarp();
-      QSPEC_STAMP(7, i);
       if constexpr (kFused) {
         // Off the critical path (the first activation tiles are on their way):
         // hand the token scales to the epilogue, and count this CTA as having
@@ -736,11 +726,9 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kFused>::kThreads, 1)
       const int sa = ra.slot;
       const int sx = rx.slot;
       racc.init(i * gpu, NACC);
-      QSPEC_STAMP(15, i);
       ok = warp_wait(smem_u32(&a_full[sa]), ra.phase, abort_flag, args.status);
       ok = ok && warp_wait(smem_u32(&x_full[sx]), rx.phase, abort_flag, args.status);
       if (!ok) break;
-      QSPEC_STAMP(3, i);
       tc_fence_after();
       const uint32_t a_col = tmem_base + static_cast<uint32_t>(sa * C::kACols);
       const uint32_t b_base = smem_u32(x_buf + sx * C::kXBytes);
@@ -748,7 +736,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kFused>::kThreads, 1)
         const int b = racc.slot;
         ok = warp_wait(smem_u32(&acc_empty[b]), racc.phase ^ 1u, abort_flag, args.status);
         if (!ok) break;
-        QSPEC_STAMP(11, i * gpu + h);
         tc_fence_after();
         // One elected lane issues the group's MMAs and its commit back to back.
         if (elect_one_lane()) {
@@ -764,7 +751,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kFused>::kThreads, 1)
           mma_commit(smem_u32(&acc_full[b]));
         }
         __syncwarp();
-        QSPEC_STAMP(12, i * gpu + h);
       }
       if (!ok) break;
       if (elect_one_lane()) {
@@ -772,7 +758,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kFused>::kThreads, 1)
         mma_commit(smem_u32(&x_empty[sx]));
       }
       __syncwarp();
-      QSPEC_STAMP(4, i);
       if (i == 0 && lane == 0) QSPEC_PHASE(3);
     }
     // All MMAs this warp issued have finished once mma_done completes.
@@ -808,7 +793,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kFused>::kThreads, 1)
       ok = ok && warp_wait(smem_u32(&a_empty[sa]), ra.phase ^ 1u, abort_flag, args.status);
       if (!ok) break;
       if (i == 0 && r == 0) QSPEC_PHASE(2);
-      if (quad == 0) QSPEC_STAMP(cteam == 0 ? 1 : 9, i);
       const uint8_t* rowp = pk_buf + sp * C::kPkBytes + r * (C::kUnitK / 2);
       uint4 v[kChunks];
 #pragma unroll
@@ -869,7 +853,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kFused>::kThreads, 1)
       __syncwarp();
       if (elect_one_lane()) mbar_arrive(smem_u32(&a_full[sa]));
       __syncwarp();
-      if (quad == 0) QSPEC_STAMP(cteam == 0 ? 2 : 10, i);
     }
   } else if (warp >= kCtlWarps + C::kConvWarps) {
     // ------------------------------------------------ epilogue
@@ -983,9 +966,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kFused>::kThreads, 1)
       const int seg_groups = static_cast<int>(seg_end - seg_start) * gpu;
       int g = static_cast<int>(seg_start - tile_u0) * gpu;   // the row's scale group
       for (int jj = 0; jj < seg_groups; ++jj, ++g) {
-        const int gi = static_cast<int>(seg_start - u_begin) * gpu + jj;   // trace index
-        (void)gi;
-        if (ew == 0) QSPEC_STAMP(14, gi);
         if (sc_cur < 0 || (g & (kScaleTileGroups - 1)) == 0) {
           if (sc_cur >= 0) {   // done with the previous tile
             __syncwarp();
@@ -1005,7 +985,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kFused>::kThreads, 1)
         const float sc = __half2float(__ushort_as_half(hbits));
         ok = warp_wait(smem_u32(&acc_full[acc.slot]), acc.phase, abort_flag, args.status);
         if (!ok) break;
-        if (ew == 0) QSPEC_STAMP(5, gi);
         tc_fence_after();
         const uint32_t taddr =
             lane_addr + static_cast<uint32_t>(C::kAccCol0 + acc.slot * MT + col0);
@@ -1021,7 +1000,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kFused>::kThreads, 1)
             __syncwarp();
             if (elect_one_lane()) mbar_arrive(smem_u32(&acc_empty[acc.slot]));
             __syncwarp();
-            if (ew == 0) QSPEC_STAMP(6, gi);
           }
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -1047,7 +1025,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kFused>::kThreads, 1)
       if (!ok) break;
       u = seg_end;
       if (et == 0) QSPEC_PHASE(u >= u_end ? 5 : 7);
-      if (et == 0 && u >= u_end) QSPEC_STAMP(8, 4);
 
       if (full) {
         write_y(n, m0);
@@ -1086,7 +1063,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kFused>::kThreads, 1)
     }
     // The split tiles whose last ticket came to this CTA are added up here,
     // after the CTA's own tiles.
-    if (et == 0) QSPEC_STAMP(8, 7);
     if (ok && head_handoff) {
       ok = warp_wait(smem_u32(&ticket_bar[0]), 0, abort_flag, args.status);
       if (ok && misc[3] != 0u) reduce_tile(t_head);
@@ -1095,7 +1071,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kFused>::kThreads, 1)
       ok = warp_wait(smem_u32(&ticket_bar[1]), 0, abort_flag, args.status);
       if (ok && misc[6] != 0u) reduce_tile(t_tail);
     }
-    if (et == 0) QSPEC_STAMP(8, 2);
   }
 
   QSPEC_TRACE_AT(0xFFF0);
@@ -1104,8 +1079,6 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kFused>::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) QSPEC_PHASE(8);
-  if (threadIdx.x == 0) QSPEC_STAMP(8, 3);
-  QSPEC_STAMP_FLUSH();
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);

@@ -380,9 +380,6 @@ extern "C" int qspec_debug_set_events(void* dev_buffer) {
              ? 0
              : 1;
 }
-extern "C" int qspec_debug_set_timeline(void* dev_buffer) {
-  return cudaMemcpyToSymbol(g_qspec_timeline, &dev_buffer, sizeof(void*)) == cudaSuccess ? 0 : 1;
-}
 #endif
 
 extern "C" {
