@@ -61,6 +61,8 @@ def parse():
                     help="skip the vocab-128256 accept/resample report")
     ap.add_argument("--no-chained", action="store_true",
                     help="skip the chained-round report (layers fed by the previous layer)")
+    ap.add_argument("--no-draft-variants", action="store_true",
+                    help="skip the W4A4 / W4A8 drafting-variant report")
     ap.add_argument("--profile-accept", metavar="RULE", default=None,
                     help="profiling driver: three calls of the accept step (RULE sampling|greedy) "
                          "at vocab 128256, batch 64, gamma 5, sigma 0.5, then exit")
@@ -125,7 +127,7 @@ def gemm_bytes(m, n, k, mode):
     """Compulsory HBM bytes of one GEMM call: packed weights + fp16 scales +
     activations as the kernel reads them + fp32 output."""
     w = n * k // 2 + n * (k // GROUP) * 2
-    x = m * k * (1 if mode == "w4a4" else 2)
+    x = m * k * (1 if mode in ("w4a4", "w4a8") else 2)   # int8 codes, or bf16
     return w + x + m * n * 4
 
 
@@ -584,6 +586,9 @@ def main():
     acc_rep = None
     if rank == 0 and world == 1 and not args.no_accept_report:
         acc_rep = accept_report(torch, qspec, peaks)
+    variants = None
+    if rank == 0 and world == 1 and not args.no_draft_variants:
+        variants = draft_variants_report(torch, qspec, peaks)
     fused_ab = None
     if rank == 0 and world == 1 and not args.no_chained:
         fused_ab = fused_quant_report(torch, qspec, wq, ws, L, x16)
@@ -603,6 +608,7 @@ def main():
                 "gpu_launches": launches_per_step * args.steps,
                 "clocks": clk.summary(), "kernels": kern, "large_m": large,
                 "m_sweep": sweep, "accept_large_vocab": acc_rep, "round_chained": chained,
+                "draft_variants": variants,
                 "fused_quant_ab": fused_ab}
         print(json.dumps(line))
     if world > 1:
@@ -734,6 +740,57 @@ def m_sweep_report(torch, qspec, peaks):
             "peak_hbm_gbs": hbm, "peak_bf16_tflops": bf16, "peak_int8_tops": 2 * bf16,
             "frac": "roofline time / measured time for each bound (frac_hbm uses all compulsory "
                     "bytes: packed weights, scales, activations, output)",
+            "shapes": out}
+
+
+def draft_variants_report(torch, qspec, peaks):
+    """The two drafting variants on the Llama-2-7B decode shapes at M = 16: W4A4 (4-bit
+    per-token activation codes) and W4A8 (8-bit codes), on the same packed weights.
+    Speed: device time per call in a CUDA graph of back-to-back calls over weights
+    rotating past L2.  Draft quality: relative Frobenius distance of each draft's output
+    from the verifying (W4A16) output on the same weights and inputs, with the inputs'
+    outlier channels (x20) that make 4-bit activations lossy."""
+    from quantized_speculative_decoding_packed_b200 import synth
+    hbm = float(peaks.get("hbm_gbs", 6650.0))
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(rank_seed(0) + 19)
+    out = {}
+    for si, (name, n, k) in enumerate(LAYERS):
+        pb = packed_bytes(n, k)
+        copies = max(2, -(-3 * 126 * 2 ** 20 // pb))
+        wqs = []
+        for _ in range(copies):
+            w = torch.randn((n, k), generator=gen, device="cuda", dtype=torch.float32) * 0.02
+            wqs.append(qspec.quantize_weights(w, GROUP))
+            del w
+        bits = synth.layer_activations("llama2_7b", M_DRAFT, k, stream=70 + si)
+        x = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+        y = torch.empty((M_DRAFT, n), dtype=torch.float32, device="cuda")
+        ref = qspec.gemm_w4a16(x, wqs[0][0], wqs[0][1], GROUP)
+        row = {"n": n, "k": k, "m": M_DRAFT}
+        for mode in ("w4a4", "w4a8"):
+            fn = qspec.gemm_w4a4 if mode == "w4a4" else qspec.gemm_w4a8
+            op = qspec.OP_GEMM_W4A4 if mode == "w4a4" else qspec.OP_GEMM_W4A8
+            work = torch.zeros(qspec.workspace_size(op, M_DRAFT, n, k, GROUP), dtype=torch.uint8,
+                               device="cuda")
+            calls = [(lambda c=c: fn(x, wqs[c][0], wqs[c][1], GROUP, y=y, work=work,
+                                     weights_ready=True)) for c in range(copies)] * 2
+            t = _graph_time_per_call(torch, calls)
+            yd = fn(x, wqs[0][0], wqs[0][1], GROUP, work=work)
+            torch.cuda.synchronize()
+            err = float(torch.linalg.vector_norm(yd.double() - ref.double()) /
+                        torch.linalg.vector_norm(ref.double()))
+            row[mode] = {"us": t * 1e6, "gbs": gemm_bytes(M_DRAFT, n, k, mode) / t / 1e9,
+                         "frac_hbm": gemm_bytes(M_DRAFT, n, k, mode) / t / 1e9 / hbm,
+                         "rel_err_vs_verify": err}
+        out[name] = row
+        del wqs, x, y, ref
+        torch.cuda.empty_cache()
+    return {"workload": f"Llama-2-7B decode shapes, drafting at M={M_DRAFT}, group {GROUP}; "
+                        "inputs N(0,1) with round(0.01 K) outlier channels x20, bf16",
+            "timing": "CUDA graph of back-to-back calls, weights rotating past L2 (3x L2)",
+            "quality": "||y_draft - y_w4a16|| / ||y_w4a16|| (Frobenius) on the same weights "
+                       "and inputs: how far each draft is from the verifying model",
             "shapes": out}
 
 
