@@ -71,6 +71,26 @@ def test_largest_vocab_identical(qs, sigma):
     assert np.array_equal(n, n_ref) and np.array_equal(tok, tok_ref)
 
 
+def test_exact_ratio_ties_and_extreme_uniforms(qs):
+    """u * q(x) == p(x) exactly rejects (the strict reading), one ulp of u below it accepts;
+    u_res = 0 and the largest float below 1 draw the first and the last token of the CDF."""
+    ai = synth.accept_inputs(synth.rng_for("accept", 20), 8, 4, 64, 1.0, 0.5)
+    below = np.nextafter(np.float32(0.5), np.float32(0.0))
+    for b in range(8):
+        for i in range(4):
+            x = ai.draft[b, i]
+            ai.q[b, i, x] = np.float32(0.5)
+            ai.p[b, i, x] = np.float32(0.25)
+            # sequences 0..3 tie at position b % 4 (reject there), accept before it
+            ai.u_acc[b, i] = np.float32(0.5) if i == b % 4 else below
+    ai.u_res[0::2] = np.float32(0.0)
+    ai.u_res[1::2] = np.nextafter(np.float32(1.0), np.float32(0.0))
+    n, tok = _run(qs, ai)
+    n_ref, tok_ref = orc.spec_accept(ai.p, ai.q, ai.draft, ai.u_acc, ai.u_res)
+    assert np.array_equal(n, n_ref) and np.array_equal(tok, tok_ref)
+    assert np.array_equal(n, np.arange(8) % 4)
+
+
 def test_p_equals_q_accepts_all_and_draws_bonus(qs):
     ai = synth.accept_inputs(synth.rng_for("accept", 12), 8, 5, 5000, 2.0, 0.5)
     ai.q = ai.p[:, :5, :].copy()
