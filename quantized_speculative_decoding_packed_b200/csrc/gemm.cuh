@@ -307,8 +307,8 @@ __device__ __forceinline__ void st_release_cta(uint32_t* p, uint32_t v) {
 
 // Fused activation quantization of one token row by the NW epilogue warps of
 // a CTA, with the arithmetic of quant_act_kernel: a = max_k |x|, s_a = a / qmax
-// and inv = qmax / a (IEEE fp32 divisions), q = clamp(rint(x * inv), -qmax-1,
-// qmax) with the product rounded to fp32, a zero row giving 0; the codes are
+// and inv = qmax / a (IEEE fp32 divisions), q = rint(x * inv) with the product
+// rounded to fp32 (within [-qmax, qmax] for finite x), a zero row giving 0; the codes are
 // stored as the GEMM reads them, each 8 channels in the order 0,2,4,6,1,3,5,7.
 // Each thread keeps up to kCache 16-byte chunks of the row in registers between
 // the two passes (all its loads in flight at once); rows longer than
@@ -353,22 +353,24 @@ __device__ __forceinline__ bool quantize_row_team(const uint16_t* xr, int K, int
   a = pp[0];
 #pragma unroll
   for (int w = 1; w < NW; ++w) a = fmaxf(a, pp[w]);
-  const float inv = __fdiv_rn(qmax, a);
+  // rint(x * inv) by an fp32 add of 1.5 x 2^23 (the code lands in the low
+  // byte; finite x never needs the clamp), as in quant_act_kernel
+  const float inv = (a == 0.f) ? 0.f : __fdiv_rn(qmax, a);
   if (t == 0) *s_out = __fdiv_rn(a, qmax);
-  const int qm = static_cast<int>(qmax);
+  auto code = [inv](float v) { return __float_as_uint(__fadd_rn(__fmul_rn(v, inv), 12582912.0f)); };
+  auto low4 = [](uint32_t a4, uint32_t b4, uint32_t c4, uint32_t d4) {
+    return __byte_perm(__byte_perm(a4, b4, 0x0040), __byte_perm(c4, d4, 0x0040), 0x5410);
+  };
   auto emit = [&](int c, const uint4& u) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-    uint32_t ev = 0, od = 0;
+    uint32_t e[8];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      int lo = __float2int_rn(__fmul_rn(bf(w[j] & 0xFFFFu), inv));
-      int hi = __float2int_rn(__fmul_rn(bf(w[j] >> 16), inv));
-      lo = (a == 0.f) ? 0 : (lo < -qm - 1 ? -qm - 1 : (lo > qm ? qm : lo));
-      hi = (a == 0.f) ? 0 : (hi < -qm - 1 ? -qm - 1 : (hi > qm ? qm : hi));
-      ev |= (static_cast<uint32_t>(lo) & 0xFFu) << (8 * j);
-      od |= (static_cast<uint32_t>(hi) & 0xFFu) << (8 * j);
+      e[2 * j] = code(bf(w[j] & 0xFFFFu));
+      e[2 * j + 1] = code(bf(w[j] >> 16));
     }
-    *reinterpret_cast<uint2*>(qr + c) = make_uint2(ev, od);
+    *reinterpret_cast<uint2*>(qr + c) =
+        make_uint2(low4(e[0], e[2], e[4], e[6]), low4(e[1], e[3], e[5], e[7]));
   };
 #pragma unroll
   for (int j = 0; j < kCache; ++j) {
@@ -878,7 +880,8 @@ __global__ void __launch_bounds__(GemmCfg<kInt8, MT, kFused>::kThreads, 1)
         epi_ok = quantize_row_team<C::kEpiWarps>(
             args.x + m * args.K, args.K, args.xq + m * args.K, const_cast<float*>(args.s_a) + m,
             args.qmax, ew, lane, s_row_part, smem_u32(row_amax), rphase, abort_flag, args.status);
-        __threadfence();
+        // every lane's code stores are ordered before lane 0's release by the
+        // warp barrier (the release is cumulative over what lane 0 has seen)
         __syncwarp();
         if (epi_ok && lane == 0)
           asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(args.qsync) : "memory");
