@@ -66,7 +66,9 @@ constexpr int kConvTeamWarps = 4;                // a converter team: one warp p
 constexpr int kCtlWarps = 4;
 constexpr int kSmemLimit = 232448;               // sm_100 dynamic shared memory per CTA
 constexpr int kMaxGrid = 1024;                   // ticket slots in the workspace
-constexpr int kMaxPk = 24, kMaxA = 8, kMaxAcc = 8, kMaxX = 8;
+// (at most 7 activation slots: the int8 16-token tile then leaves an SM room
+// for a CTA of the activation quantizer beside it)
+constexpr int kMaxPk = 24, kMaxA = 8, kMaxAcc = 8, kMaxX = 7;
 // Group scales arrive by TMA, 8 groups x 128 rows (2 KB) per tile, into a ring.
 constexpr int kScaleTileGroups = 8;
 constexpr int kScaleTileBytes = kTileN * kScaleTileGroups * 2;

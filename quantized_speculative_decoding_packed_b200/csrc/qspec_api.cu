@@ -316,9 +316,11 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
     // Also a programmatic dependent: it waits for the preceding grid itself,
     // and lets the GEMM launch once it has (or, when the weights are ready,
     // at once: the GEMM then reads nothing else before its own waits).
+    // 128 threads beside the 16-token GEMM tile (they fit on its SMs), else 256
+    const bool small = p.mt == 16;
     cudaLaunchConfig_t qc = {};
     qc.gridDim = dim3(static_cast<unsigned>(m));
-    qc.blockDim = dim3(256);
+    qc.blockDim = dim3(small ? 128 : 256);
     qc.stream = stream;
     cudaLaunchAttribute qa[1];
     qa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -329,19 +331,22 @@ qspec_status run_gemm(const uint16_t* x, int64_t m, int64_t k, const uint8_t* wq
     const int early = weights_ready ? 1 : 0;
     const void* xin = xf ? static_cast<const void*>(xf) : static_cast<const void*>(x);
     const int64_t ld = xf ? ldx : k;
+    const int64_t kk = k;
     cudaError_t qe;
     if (xf) {
-      qe = (act_bits == 8)
-               ? cudaLaunchKernelEx(&qc, quant_act_kernel<false, 127, true>, xin, ld,
-                                    static_cast<int64_t>(k), qout, sa, early)
-               : cudaLaunchKernelEx(&qc, quant_act_kernel<false, 7, true>, xin, ld,
-                                    static_cast<int64_t>(k), qout, sa, early);
+      if (act_bits == 8)
+        qe = small ? cudaLaunchKernelEx(&qc, quant_act_kernel<false, 127, true, 128>, xin, ld, kk, qout, sa, early)
+                   : cudaLaunchKernelEx(&qc, quant_act_kernel<false, 127, true, 256>, xin, ld, kk, qout, sa, early);
+      else
+        qe = small ? cudaLaunchKernelEx(&qc, quant_act_kernel<false, 7, true, 128>, xin, ld, kk, qout, sa, early)
+                   : cudaLaunchKernelEx(&qc, quant_act_kernel<false, 7, true, 256>, xin, ld, kk, qout, sa, early);
     } else {
-      qe = (act_bits == 8)
-               ? cudaLaunchKernelEx(&qc, quant_act_kernel<false, 127>, xin, ld,
-                                    static_cast<int64_t>(k), qout, sa, early)
-               : cudaLaunchKernelEx(&qc, quant_act_kernel<false, 7>, xin, ld,
-                                    static_cast<int64_t>(k), qout, sa, early);
+      if (act_bits == 8)
+        qe = small ? cudaLaunchKernelEx(&qc, quant_act_kernel<false, 127, false, 128>, xin, ld, kk, qout, sa, early)
+                   : cudaLaunchKernelEx(&qc, quant_act_kernel<false, 127, false, 256>, xin, ld, kk, qout, sa, early);
+      else
+        qe = small ? cudaLaunchKernelEx(&qc, quant_act_kernel<false, 7, false, 128>, xin, ld, kk, qout, sa, early)
+                   : cudaLaunchKernelEx(&qc, quant_act_kernel<false, 7, false, 256>, xin, ld, kk, qout, sa, early);
     }
     if (qe != cudaSuccess) {
       cudaGetLastError();
@@ -410,7 +415,7 @@ qspec_status qspec_quant_act(const uint16_t* x, int64_t m, int64_t k, uint8_t* x
   if (!aligned(x, 16) || !aligned(xq, 4) || !aligned(xs, 4)) return QSPEC_ERR_INVALID_ARG;
   qspec_status st = current_device(nullptr, nullptr);
   if (st != QSPEC_OK) return st;
-  quant_act_kernel<true><<<static_cast<unsigned>(m), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+  quant_act_kernel<true, 7, false, 256><<<static_cast<unsigned>(m), 256, 0, static_cast<cudaStream_t>(stream)>>>(
       x, k, k, xq, xs, 0);
   return cudaGetLastError() == cudaSuccess ? QSPEC_OK : QSPEC_ERR_CUDA;
 }

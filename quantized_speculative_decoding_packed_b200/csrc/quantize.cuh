@@ -83,12 +83,20 @@ __device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) {
 // kF32In: x holds fp32 values (a layer's output, row stride ldx) and each one
 // is first rounded to bf16 (nearest even): the bf16 glue of chained layers
 // folded into the read.  Otherwise x holds bf16 bit patterns, row stride ldx.
-template <bool kPacked, int kQMax = 7, bool kF32In = false>
-__global__ void __launch_bounds__(256) quant_act_kernel(const void* __restrict__ x, int64_t ldx,
-                                                        int64_t k, void* __restrict__ out,
-                                                        float* __restrict__ scales,
-                                                        int early_trigger) {
-  __shared__ float red[8];
+// kThreads per row: 128 at most 56 registers each (launch bounds 128 x 9), or
+// 256.  The 128-thread CTA with its 16 bytes of static shared memory fits on an
+// SM beside a decode GEMM CTA of the 16-token tile (12 warps x 152 allocated
+// registers + 4 x 56 = 65536; shared memory 227 KB + 1 KB reserved each), so
+// the GEMM launched behind this kernel never waits for an SM it holds (with
+// 256 threads the last 16 GEMM CTAs of every drafting call started only when
+// these exited).  Rows of other sizes use 256 threads (fewer re-reads of long
+// rows).
+template <bool kPacked, int kQMax = 7, bool kF32In = false, int kThreads = 256>
+__global__ void __launch_bounds__(kThreads, kThreads == 128 ? 9 : 4)
+    quant_act_kernel(const void* __restrict__ x, int64_t ldx, int64_t k, void* __restrict__ out,
+                     float* __restrict__ scales, int early_trigger) {
+  constexpr int kQuantThreads = kThreads;
+  __shared__ float red[kQuantThreads / 32];
   const int64_t row = blockIdx.x;
   const int tid = threadIdx.x;
   constexpr unsigned kTraceKind = 3u;   // trace builds: event-log tags
@@ -154,13 +162,14 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const void* __restrict__
   __nv_bfloat162 m2 = __float2bfloat162_rn(0.f);
 #pragma unroll
   for (int j = 0; j < kCache; ++j) {
-    const int64_t c = (static_cast<int64_t>(tid) + 256 * j) * 8;
+    const int64_t c = (static_cast<int64_t>(tid) + kQuantThreads * j) * 8;
     if (c < k) {
       cache[j] = load8(c);
       m2 = absmax8(cache[j], m2);
     }
   }
-  for (int64_t c = (static_cast<int64_t>(tid) + 256 * kCache) * 8; c < k; c += 256 * 8)
+  for (int64_t c = (static_cast<int64_t>(tid) + kQuantThreads * kCache) * 8; c < k;
+       c += kQuantThreads * 8)
     m2 = absmax8(load8(c), m2);
   float a = fmaxf(__low2float(m2), __high2float(m2));
 #pragma unroll
@@ -169,7 +178,7 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const void* __restrict__
   __syncthreads();
   a = red[0];
 #pragma unroll
-  for (int i = 1; i < 8; ++i) a = fmaxf(a, red[i]);
+  for (int i = 1; i < kQuantThreads / 32; ++i) a = fmaxf(a, red[i]);
 
   static_assert(!kPacked || kQMax == 7, "packed output holds 4-bit codes");
   constexpr float kLevels = static_cast<float>(kQMax);
@@ -219,10 +228,11 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const void* __restrict__
   };
 #pragma unroll
   for (int j = 0; j < kCache; ++j) {
-    const int64_t c = (static_cast<int64_t>(tid) + 256 * j) * 8;
+    const int64_t c = (static_cast<int64_t>(tid) + kQuantThreads * j) * 8;
     if (c < k) emit(c, cache[j]);
   }
-  for (int64_t c = (static_cast<int64_t>(tid) + 256 * kCache) * 8; c < k; c += 256 * 8)
+  for (int64_t c = (static_cast<int64_t>(tid) + kQuantThreads * kCache) * 8; c < k;
+       c += kQuantThreads * 8)
     emit(c, load8(c));
   if (tid == 0) QSPEC_PHASE(8);
 }
