@@ -68,34 +68,39 @@ def parse():
                          "at vocab 128256, batch 64, gamma 5, sigma 0.5, then exit")
     ap.add_argument("--profile-gemm", metavar="MODE:SHAPE", default=None,
                     help="profiling driver: three calls of one GEMM (MODE w4a4|w4a16, SHAPE "
-                         "qkv|o_proj|gate_up|down of the workload) on seeded weights, then exit")
+                         "qkv|o_proj|gate_up|down of the workload, 'decode' for all four in "
+                         "turn, or 70b_qkv|70b_gate_up|70b_down at M=2048) on seeded weights, "
+                         "then exit")
     return ap.parse_args()
 
 
 def profile_gemm(spec):
     """Three calls of one GEMM of the workload, for a profiler to capture one of them.
-    SHAPE is a Llama-2-7B layer (decode M), or one of the Llama-2-70B layers with a
-    "70b_" prefix (M = 2048)."""
+    SHAPE is a Llama-2-7B layer (decode M), "decode" for each of the four Llama-2-7B
+    layers in turn, or one of the Llama-2-70B layers with a "70b_" prefix (M = 2048)."""
     import torch
     from quantized_speculative_decoding_packed_b200 import qspec
-    mode, shape = spec.split(":")
-    if shape.startswith("70b_"):
-        n, k = {name: (n, k) for name, n, k in LARGE_SHAPES}[shape[4:]]
-        m = LARGE_M
-    else:
-        n, k = {name: (n, k) for name, n, k in LAYERS}[shape]
-        m = M_DRAFT if mode == "w4a4" else M_VERIFY
+    mode, spec_shape = spec.split(":")
+    shapes = [name for name, _, _ in LAYERS] if spec_shape == "decode" else [spec_shape]
     gen = torch.Generator(device="cuda")
     gen.manual_seed(rank_seed(0))
-    w = torch.randn((n, k), generator=gen, device="cuda", dtype=torch.float32) * 0.02
-    wq, ws = qspec.quantize_weights(w, GROUP)
-    del w
-    x = torch.randn((m, k), generator=gen, device="cuda").to(torch.bfloat16)
     fn = qspec.gemm_w4a4 if mode == "w4a4" else qspec.gemm_w4a16
-    for _ in range(3):
-        y = fn(x, wq, ws, GROUP)
-    torch.cuda.synchronize()
-    print(f"{mode} {shape}: y[{m}][{n}] sum |y| = {float(y.abs().sum()):.6g}")
+    for shape in shapes:
+        if shape.startswith("70b_"):
+            n, k = {name: (n, k) for name, n, k in LARGE_SHAPES}[shape[4:]]
+            m = LARGE_M
+        else:
+            n, k = {name: (n, k) for name, n, k in LAYERS}[shape]
+            m = M_DRAFT if mode == "w4a4" else M_VERIFY
+        w = torch.randn((n, k), generator=gen, device="cuda", dtype=torch.float32) * 0.02
+        wq, ws = qspec.quantize_weights(w, GROUP)
+        del w
+        x = torch.randn((m, k), generator=gen, device="cuda").to(torch.bfloat16)
+        for _ in range(3):
+            y = fn(x, wq, ws, GROUP)
+        torch.cuda.synchronize()
+        print(f"{mode} {shape}: y[{m}][{n}] sum |y| = {float(y.abs().sum()):.6g}")
+        del wq, ws, x, y
 
 
 def profile_accept(rule, batch=64, gamma=5, vocab=128256, sigma=0.5):
@@ -447,7 +452,10 @@ def main():
     n_acc = torch.empty((BATCH,), dtype=torch.int32, device=dev)
     tokens = torch.empty((BATCH, GAMMA + 1), dtype=torch.int32, device=dev)
 
-    # events bracketing a sample of launches inside the graph (layer 0 of each pass)
+    # Events at the section boundaries of the step only: before the first drafting pass,
+    # after each pass, after the verifying pass and after the accept step.  An event node
+    # between two calls ends the programmatic overlap of the second call with the first,
+    # so none is placed between the calls of a section: each section is timed as it runs.
     ev = {}
 
     def mark(key):
@@ -455,30 +463,24 @@ def main():
         e.record()
 
     def step(with_events):
+        if with_events:
+            mark("start")
         for pss in range(GAMMA):
             for li in range(L):
                 for si, (_, n, k) in enumerate(LAYERS):
-                    t = with_events and li == 0
-                    if t:
-                        mark(("w4a4", pss, si, 0))
                     qspec.gemm_w4a4(x16[si], wq[li][si], ws[li][si], GROUP, y=y16[si], work=work,
                                     weights_ready=True)
-                    if t:
-                        mark(("w4a4", pss, si, 1))
+            if with_events:
+                mark(("draft", pss))
         for li in range(L):
             for si, (_, n, k) in enumerate(LAYERS):
-                t = with_events and li == 0
-                if t:
-                    mark(("w4a16", 0, si, 0))
                 qspec.gemm_w4a16(x80[si], wq[li][si], ws[li][si], GROUP, y=y80[si], work=work,
                                  weights_ready=True)
-                if t:
-                    mark(("w4a16", 0, si, 1))
         if with_events:
-            mark(("accept", 0, 0, 0))
+            mark("verify")
         qspec.spec_accept(p, q, draft, u_acc, u_res, n_accepted=n_acc, tokens=tokens, work=acc_work)
         if with_events:
-            mark(("accept", 0, 0, 1))
+            mark("accept")
 
     launches_per_step = GAMMA * L * len(LAYERS) * 2 + L * len(LAYERS) + 1
     stream = torch.cuda.Stream(device=dev)
@@ -515,28 +517,30 @@ def main():
         ms_total = max_over_ranks(ms_total, dev)
         ms_step = ms_total / args.steps
 
-    # per-kernel durations from the last timed step
-    def dur(kind, pss, si):
-        return ev[(kind, pss, si, 0)].elapsed_time(ev[(kind, pss, si, 1)])
-
-    kern = {}
-    w4a4_b = w4a4_t = 0.0
-    gu_b = gu_t = 0.0
-    for si, (name, n, k) in enumerate(LAYERS):
-        t4 = [dur("w4a4", pss, si) for pss in range(GAMMA)]
-        t16 = dur("w4a16", 0, si)
-        b4, b16 = gemm_bytes(M_DRAFT, n, k, "w4a4"), gemm_bytes(M_VERIFY, n, k, "w4a16")
-        kern[name] = {"w4a4_us": 1e3 * statistics.mean(t4), "w4a4_gbs": b4 / (statistics.mean(t4) * 1e-3) / 1e9,
-                      "w4a4_tops": 2 * M_DRAFT * n * k / (statistics.mean(t4) * 1e-3) / 1e12,
-                      "w4a16_us": 1e3 * t16, "w4a16_gbs": b16 / (t16 * 1e-3) / 1e9,
-                      "w4a16_tflops": 2 * M_VERIFY * n * k / (t16 * 1e-3) / 1e12}
-        w4a4_b += b4 * GAMMA
-        w4a4_t += sum(t4)
-        if name == "gate_up":
-            gu_b, gu_t = b4 * GAMMA, sum(t4)
-    t_acc = dur("accept", 0, 0)
+    # section durations from the last timed step (ms)
+    bounds = ["start"] + [("draft", pss) for pss in range(GAMMA)]
+    t_pass = [ev[a].elapsed_time(ev[b]) for a, b in zip(bounds, bounds[1:])]
+    t_draft = sum(t_pass)
+    t_verify = ev[("draft", GAMMA - 1)].elapsed_time(ev["verify"])
+    t_acc = ev["verify"].elapsed_time(ev["accept"])
+    calls_pass = L * len(LAYERS)
+    b_pass = L * sum(gemm_bytes(M_DRAFT, n, k, "w4a4") for (_, n, k) in LAYERS)
+    b_verify = L * sum(gemm_bytes(M_VERIFY, n, k, "w4a16") for (_, n, k) in LAYERS)
     acc_b = accept_bytes(n_acc.cpu().numpy(), GAMMA, VOCAB)
-    kern["accept"] = {"us": 1e3 * t_acc, "gbs": acc_b / (t_acc * 1e-3) / 1e9}
+    kern = {
+        "drafting": {"passes": GAMMA, "calls_per_pass": calls_pass,
+                     "us_per_pass": [1e3 * t for t in t_pass],
+                     "us_per_call": 1e3 * t_draft / (GAMMA * calls_pass),
+                     "gbs": GAMMA * b_pass / (t_draft * 1e-3) / 1e9,
+                     "share_of_step": t_draft / ms_step},
+        "verifying": {"calls": calls_pass, "us": 1e3 * t_verify,
+                      "us_per_call": 1e3 * t_verify / calls_pass,
+                      "gbs": b_verify / (t_verify * 1e-3) / 1e9,
+                      "share_of_step": t_verify / ms_step},
+        "accept": {"us": 1e3 * t_acc, "gbs": acc_b / (t_acc * 1e-3) / 1e9,
+                   "share_of_step": t_acc / ms_step},
+        "timing": "CUDA events at the section boundaries of the last timed step",
+    }
 
     peaks = {}
     try:
@@ -545,16 +549,21 @@ def main():
     except Exception:
         pass
     hbm_peak = peaks.get("hbm_gbs", 6650.0)
-    # Dominant kernel: the W4A4 drafting GEMM.  The roofline object describes its
-    # largest launch (gate+up, 46.5 MB packed), timed live over the 4 draft passes
-    # of each step's layer 0; the all-shape figure is kept beside it.
-    achieved = gu_b / (gu_t * 1e-3) / 1e9
+    # Dominant kernel: the W4A4 drafting GEMM call (activation quantizer + qgemm), over
+    # all its launches in the step: achieved = the drafting passes' algorithmic bytes over
+    # their event-timed duration, i.e. average bytes per launch over average launch time.
+    drafting_calls = GAMMA * calls_pass
+    achieved = kern["drafting"]["gbs"]
+    traffic, traffic_src = traffic_from_profile()
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": traffic_from_profile(),
-                "kernel": "W4A4 drafting GEMM call on gate_up N=22016 K=4096 M=16 "
-                          "(per-token quant pre-pass + qgemm_kernel<int8,16>)",
-                "bytes_per_launch": gemm_bytes(M_DRAFT, 22016, 4096, "w4a4"),
-                "all_shapes_achieved": w4a4_b / (w4a4_t * 1e-3) / 1e9,
+                "frac": achieved / hbm_peak, "traffic": traffic,
+                "kernel": "W4A4 drafting GEMM call (per-token quant pre-pass + "
+                          "qgemm_kernel<int8,16>), M=16, all four Llama-2-7B decode shapes "
+                          "(qkv, o_proj, gate_up, down) as they run back to back in the step",
+                "launches_timed": drafting_calls,
+                "us_per_launch": 1e3 * t_draft / drafting_calls,
+                "bytes_per_launch": GAMMA * b_pass / drafting_calls,
+                "traffic_source": traffic_src,
                 "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)" if "hbm_gbs" in peaks
                 else "fallback 6650 GB/s"}
 
@@ -576,6 +585,13 @@ def main():
                "sample": desc_all + "; plus the accept step on one thread",
                "single_thread": {"value": bytes_step / t_cpu / 1e9, "unit": "GB/s", "cores": 1,
                                  "sample": desc}}
+
+    shapes_rep = None
+    if rank == 0 and world == 1:
+        shapes_rep = decode_shapes_report(torch, qspec, hbm_peak, wq, ws, L, x16, x80, work)
+        roofline["gate_up_back_to_back"] = {
+            "us_per_call": shapes_rep["gate_up"]["w4a4_us"],
+            "frac": shapes_rep["gate_up"]["w4a4_frac_hbm"]}
 
     large = None
     if rank == 0 and world == 1 and not args.no_large_m:
@@ -606,7 +622,8 @@ def main():
                 "tops": world * ops_step / (ms_step * 1e-3) / 1e12,
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps,
-                "clocks": clk.summary(), "kernels": kern, "large_m": large,
+                "clocks": clk.summary(), "kernels": kern, "decode_shapes": shapes_rep,
+                "large_m": large,
                 "m_sweep": sweep, "accept_large_vocab": acc_rep, "round_chained": chained,
                 "draft_variants": variants,
                 "fused_quant_ab": fused_ab}
@@ -663,6 +680,29 @@ def large_m_report(torch, qspec, peaks):
 SWEEP_SHAPES = (("qkv", 6144, 4096), ("o_proj", 4096, 4096), ("gate_up", 28672, 4096),
                 ("down", 4096, 14336))
 SWEEP_M = (1, 8, 32, 128, 256)
+
+
+def decode_shapes_report(torch, qspec, hbm, wq, ws, layers, x16, x80, work):
+    """Per decode shape and mode: device time per call in a CUDA graph of the shape's calls
+    over all the step's layers, back to back (the layers' weights together exceed the L2),
+    as the calls run inside a drafting or verifying pass."""
+    out = {}
+    for si, (name, n, k) in enumerate(LAYERS):
+        row = {"n": n, "k": k}
+        for mode, x, m in (("w4a4", x16[si], M_DRAFT), ("w4a16", x80[si], M_VERIFY)):
+            fn = qspec.gemm_w4a4 if mode == "w4a4" else qspec.gemm_w4a16
+            y = torch.empty((m, n), dtype=torch.float32, device="cuda")
+            calls = [(lambda li=li: fn(x, wq[li][si], ws[li][si], GROUP, y=y, work=work,
+                                       weights_ready=True)) for li in range(layers)]
+            t = _graph_time_per_call(torch, calls)
+            b = gemm_bytes(m, n, k, mode)
+            row[f"{mode}_us"] = t * 1e6
+            row[f"{mode}_gbs"] = b / t / 1e9
+            row[f"{mode}_frac_hbm"] = b / t / 1e9 / hbm
+        out[name] = row
+    out["timing"] = (f"CUDA graph of the shape's calls over {layers} layers' weights, back to "
+                     "back, median of 5 replays")
+    return out
 
 
 def _graph_time_per_call(torch, calls, reps=5):
@@ -1008,20 +1048,28 @@ def measure_e2e(torch, stream, graph, acts, accept_in, outs, steps, bytes_step):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
+TRAFFIC_PROFILE = "qgemm_w4a4_llama2_7b_decode_m16.json"
+
+
 def traffic_from_profile():
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current GEMM source; else null."""
-    path = os.path.join(ROOT, "profiles", "qgemm_w4a4_llama2_7b_gate_up_m16.json")
-    src = os.path.join(ROOT, "quantized_speculative_decoding_packed_b200", "csrc", "gemm.cuh")
+    """(DRAM bytes per W4A4 drafting call averaged over the four decode shapes, source)
+    from the committed ncu summary, if it was taken on the current GEMM and quantizer
+    sources; else (None, reason)."""
+    path = os.path.join(ROOT, "profiles", TRAFFIC_PROFILE)
+    csrc = os.path.join(ROOT, "quantized_speculative_decoding_packed_b200", "csrc")
     try:
         with open(path) as f:
             prof = json.load(f)
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
-        if prof.get("gemm_source_sha256") == sha:
-            return prof.get("dram_bytes_per_launch")
-    except Exception:
-        pass
-    return None
+        for name, sha in prof["source_sha256"].items():
+            if hashlib.sha256(open(os.path.join(csrc, name), "rb").read()).hexdigest() != sha:
+                return None, f"profiles/{TRAFFIC_PROFILE} predates the current {name}"
+        per_shape = prof["dram_bytes_per_call"]
+        return (sum(per_shape.values()) / len(per_shape),
+                f"profiles/{TRAFFIC_PROFILE}: ncu dram__bytes_read.sum + dram__bytes_write.sum "
+                "of the quantizer and GEMM launches of one call per shape, averaged over the "
+                "four shapes")
+    except Exception as e:  # missing or malformed summary: no traffic figure
+        return None, f"profiles/{TRAFFIC_PROFILE} unreadable ({type(e).__name__})"
 
 
 if __name__ == "__main__":
