@@ -323,3 +323,62 @@ def linear_chain(x0: np.ndarray, layers, mode: str, group: int):
         x = round_to_bf16(outs[-1][:, :k]) if outs else x
         outs.append(gemm(x, q, s_h, group))
     return outs
+
+
+# --------------------------------------------------------------------------
+# The KV cache shared by the two stages (QSpec abstract: the drafter and the
+# verifier reuse the KV cache as well as the weights).  The pages print no
+# layout or rule; the readings taken here:
+#  * one cache per layer, K and V each [B][H_kv][L_max][D], stored in bf16;
+#  * a pass over T new tokens per sequence appends their keys and values at
+#    positions lens[b] + offset + t (draft pass j: T = 1, offset = j; the
+#    verifying pass: T = gamma + 1, offset = 0, overwriting the drafted
+#    entries with the verifier's);
+#  * token (b, t) then attends causally to positions 0 .. lens[b] + offset + t
+#    with the textbook scaled dot-product softmax, query head h reading KV
+#    head h // (H / H_kv) (grouped-query attention);
+#  * after the accept step, lens[b] advances by n_accepted[b] + 1: the
+#    entries past it (rejected drafts) are simply overwritten later.
+# The token rows come from a fused QKV projection: row b * T + t holds the
+# H query heads, then the H_kv key heads, then the H_kv value heads, D
+# columns each.
+# --------------------------------------------------------------------------
+def kv_append(k_cache, v_cache, qkv, lens, offset: int, t_new: int, h_q: int, h_kv: int, d: int):
+    """Returns copies of the caches with the T new keys/values written (bf16-rounded)."""
+    k_out = np.array(k_cache, dtype=np.float32, copy=True)
+    v_out = np.array(v_cache, dtype=np.float32, copy=True)
+    qkv = np.asarray(qkv, dtype=np.float32)
+    for b in range(len(lens)):
+        for t in range(t_new):
+            pos = int(lens[b]) + offset + t
+            row = qkv[b * t_new + t]
+            for g in range(h_kv):
+                k_out[b, g, pos] = round_to_bf16(row[(h_q + g) * d:(h_q + g + 1) * d])
+                v_out[b, g, pos] = round_to_bf16(row[(h_q + h_kv + g) * d:(h_q + h_kv + g + 1) * d])
+    return k_out, v_out
+
+
+def decode_attention(qkv, k_cache, v_cache, lens, offset: int, t_new: int, h_q: int, h_kv: int,
+                     d: int) -> np.ndarray:
+    """Attention output [B*T][H*D] in float64 (query values as given, cache values as stored)."""
+    qkv = np.asarray(qkv, dtype=np.float64)
+    kc = np.asarray(k_cache, dtype=np.float64)
+    vc = np.asarray(v_cache, dtype=np.float64)
+    group = h_q // h_kv
+    out = np.zeros((len(lens) * t_new, h_q * d))
+    for b in range(len(lens)):
+        for t in range(t_new):
+            n_keys = int(lens[b]) + offset + t + 1
+            for h in range(h_q):
+                g = h // group
+                q = qkv[b * t_new + t, h * d:(h + 1) * d]
+                s = kc[b, g, :n_keys] @ q / np.sqrt(d)
+                w = np.exp(s - s.max())
+                out[b * t_new + t, h * d:(h + 1) * d] = (w / w.sum()) @ vc[b, g, :n_keys]
+    return out
+
+
+def kv_commit(lens, n_accepted) -> np.ndarray:
+    """Cache lengths after a round: the accepted drafts plus the token the
+    verifier produced at the first rejection (or the bonus token)."""
+    return np.asarray(lens, dtype=np.int64) + np.asarray(n_accepted, dtype=np.int64) + 1

@@ -482,3 +482,136 @@ def test_linear_chain_is_the_composition_of_the_pinned_gemms():
                 x = synth.bf16_bits_to_f32(synth.to_bf16_bits(outs[j - 1][:, :q.shape[1]].astype(np.float32)))
             assert np.array_equal(outs[j], fn(x, q, s_h, group)), (mode, j)
         assert outs[-1].shape == (m, 512)
+
+
+# ---------------------------------------------------------------- shared KV cache, decode attention
+def _kv_case(rng, b=2, t_new=3, h_q=4, h_kv=2, d=8, l_max=12, lens=(4, 7)):
+    kc = synth.bf16_bits_to_f32(synth.to_bf16_bits(rng.standard_normal((b, h_kv, l_max, d)).astype(np.float32)))
+    vc = synth.bf16_bits_to_f32(synth.to_bf16_bits(rng.standard_normal((b, h_kv, l_max, d)).astype(np.float32)))
+    qkv = rng.standard_normal((b * t_new, (h_q + 2 * h_kv) * d)).astype(np.float32)
+    return kc, vc, qkv, np.array(lens, dtype=np.int64)
+
+
+def test_kv_append_places_each_column_where_the_layout_says():
+    # qkv column c holds the value c (exact in bf16 below 256): the cache entry
+    # of kv head g, element i must hold the column (H + g) * D + i (keys) or
+    # (H + H_kv + g) * D + i (values), at position lens + offset + t only
+    b, t_new, h_q, h_kv, d, l_max = 2, 2, 4, 2, 8, 10
+    lens, offset = np.array([3, 6]), 1
+    qkv = np.tile(np.arange((h_q + 2 * h_kv) * d, dtype=np.float32), (b * t_new, 1))
+    kc = np.full((b, h_kv, l_max, d), -1.0, dtype=np.float32)
+    vc = np.full((b, h_kv, l_max, d), -2.0, dtype=np.float32)
+    k2, v2 = orc.kv_append(kc, vc, qkv, lens, offset, t_new, h_q, h_kv, d)
+    for bb in range(b):
+        for g in range(h_kv):
+            for pos in range(l_max):
+                written = lens[bb] + offset <= pos < lens[bb] + offset + t_new
+                for i in range(d):
+                    assert k2[bb, g, pos, i] == ((h_q + g) * d + i if written else -1.0)
+                    assert v2[bb, g, pos, i] == ((h_q + h_kv + g) * d + i if written else -2.0)
+    # values are stored rounded to bf16 (1 + 2^-9 is not a bf16 value; RNE gives 1)
+    qkv2 = np.full_like(qkv, 1.0 + 2.0 ** -9)
+    k3, _ = orc.kv_append(kc, vc, qkv2, lens, 0, t_new, h_q, h_kv, d)
+    assert k3[0, 0, lens[0], 0] == 1.0
+
+
+def test_attention_single_key_returns_its_value():
+    rng = np.random.default_rng(51)
+    kc, vc, qkv, _ = _kv_case(rng)
+    lens = np.array([0, 0])
+    out = orc.decode_attention(qkv, kc, vc, lens, 0, 1, 4, 2, 8)   # one key per row
+    for b in range(2):
+        for h in range(4):
+            assert np.array_equal(out[b, h * 8:(h + 1) * 8], vc[b, h // 2, 0].astype(np.float64))
+
+
+def test_attention_equal_scores_average_the_values():
+    # identical keys (or a zero query) weight every visible position equally
+    rng = np.random.default_rng(52)
+    kc, vc, qkv, lens = _kv_case(rng)
+    kc[:] = kc[:, :, :1, :]
+    out = orc.decode_attention(qkv, kc, vc, lens, 1, 3, 4, 2, 8)
+    for b in range(2):
+        for t in range(3):
+            n = lens[b] + 1 + t + 1
+            for h in range(4):
+                want = vc[b, h // 2, :n].astype(np.float64).mean(axis=0)
+                assert np.allclose(out[b * 3 + t, h * 8:(h + 1) * 8], want, rtol=0, atol=1e-12)
+    kc2, vc2, qkv2, lens2 = _kv_case(rng)
+    qkv2[:, :4 * 8] = 0.0
+    out2 = orc.decode_attention(qkv2, kc2, vc2, lens2, 0, 3, 4, 2, 8)
+    assert np.allclose(out2[0, :8], vc2[0, 0, :lens2[0] + 1].astype(np.float64).mean(axis=0),
+                       rtol=0, atol=1e-12)
+
+
+def test_attention_two_keys_hand_worked_weights():
+    # D = 4, so scores are q.k / 2.  k0 = 0 and k1 = e0 with q = 2 ln 3 e0 give
+    # scores 0 and ln 3: weights 1/4 and 3/4, so the output is (v0 + 3 v1) / 4.
+    d, h_q, h_kv = 4, 1, 1
+    kc = np.zeros((1, 1, 2, d), dtype=np.float32)
+    kc[0, 0, 1, 0] = 1.0
+    vc = np.zeros((1, 1, 2, d), dtype=np.float32)
+    vc[0, 0, 0] = [4.0, 0.0, -8.0, 1.0]
+    vc[0, 0, 1] = [0.0, 8.0, 4.0, 1.0]
+    qkv = np.zeros((1, (h_q + 2 * h_kv) * d), dtype=np.float32)
+    qkv[0, 0] = 2.0 * math.log(3.0)
+    out = orc.decode_attention(qkv, kc, vc, np.array([1]), 0, 1, h_q, h_kv, d)
+    assert np.allclose(out[0], [1.0, 6.0, 1.0, 1.0], rtol=0, atol=1e-7)
+    # the reversed query prefers k0 by the same factor
+    qkv[0, 0] = -2.0 * math.log(3.0)
+    out = orc.decode_attention(qkv, kc, vc, np.array([1]), 0, 1, h_q, h_kv, d)
+    assert np.allclose(out[0], [3.0, 2.0, -5.0, 1.0], rtol=0, atol=1e-7)
+
+
+def test_attention_is_causal_and_maps_query_heads_to_their_kv_head():
+    rng = np.random.default_rng(53)
+    b, t_new, h_q, h_kv, d, l_max = 2, 3, 8, 2, 8, 16
+    kc, vc, qkv, lens = _kv_case(rng, b, t_new, h_q, h_kv, d, l_max, (5, 9))
+    offset = 2
+    out = orc.decode_attention(qkv, kc, vc, lens, offset, t_new, h_q, h_kv, d)
+    # entries past each row's last visible position change nothing
+    kc2, vc2 = kc.copy(), vc.copy()
+    for bb in range(b):
+        first_hidden = lens[bb] + offset + 1          # row t = 0 sees lens + offset + 1 keys
+        kc2[bb, :, first_hidden + t_new - 1:] = 1e3
+        vc2[bb, :, first_hidden + t_new - 1:] = -1e3
+    out2 = orc.decode_attention(qkv, kc2, vc2, lens, offset, t_new, h_q, h_kv, d)
+    assert np.array_equal(out, out2)
+    # every value of KV head g equal to g: query head h must read g = h // (H / H_kv)
+    vc3 = np.broadcast_to(np.arange(h_kv, dtype=np.float32)[None, :, None, None], vc.shape).copy()
+    out3 = orc.decode_attention(qkv, kc, vc3, lens, offset, t_new, h_q, h_kv, d)
+    for h in range(h_q):
+        assert np.allclose(out3[:, h * d:(h + 1) * d], h // (h_q // h_kv), rtol=0, atol=1e-12)
+
+
+def test_attention_dominant_score_selects_one_value():
+    rng = np.random.default_rng(54)
+    d = 8
+    kc = np.zeros((1, 1, 6, d), dtype=np.float32)
+    kc[0, 0, :, :] = np.eye(6, d, dtype=np.float32)      # key j = e_j
+    vc = synth.bf16_bits_to_f32(synth.to_bf16_bits(rng.standard_normal((1, 1, 6, d)).astype(np.float32)))
+    qkv = np.zeros((1, 3 * d), dtype=np.float32)
+    qkv[0, 4] = 400.0                                      # score of key 4: 400 / sqrt(8) = 141
+    out = orc.decode_attention(qkv, kc, vc, np.array([5]), 0, 1, 1, 1, d)
+    assert np.allclose(out[0], vc[0, 0, 4], rtol=0, atol=1e-30)
+
+
+def test_kv_commit_and_a_round_on_the_shared_cache():
+    # gamma drafts append one entry each; the verifier overwrites the same
+    # positions; the commit keeps the accepted drafts plus one
+    rng = np.random.default_rng(55)
+    b, gamma, h_q, h_kv, d, l_max = 2, 3, 2, 1, 8, 16
+    lens = np.array([2, 5])
+    kc = np.zeros((b, h_kv, l_max, d), dtype=np.float32)
+    vc = np.zeros_like(kc)
+    for j in range(gamma):
+        qkv = rng.standard_normal((b, (h_q + 2 * h_kv) * d)).astype(np.float32)
+        kc, vc = orc.kv_append(kc, vc, qkv, lens, j, 1, h_q, h_kv, d)
+    qkv_v = rng.standard_normal((b * (gamma + 1), (h_q + 2 * h_kv) * d)).astype(np.float32)
+    kc, vc = orc.kv_append(kc, vc, qkv_v, lens, 0, gamma + 1, h_q, h_kv, d)
+    for bb in range(b):
+        for t in range(gamma + 1):
+            want = synth.bf16_bits_to_f32(synth.to_bf16_bits(qkv_v[bb * (gamma + 1) + t, h_q * d:(h_q + 1) * d]))
+            assert np.array_equal(kc[bb, 0, lens[bb] + t], want)
+    n_acc = np.array([0, 3])
+    assert orc.kv_commit(lens, n_acc).tolist() == [3, 9]
