@@ -273,6 +273,70 @@ qspec_status qspec_spec_accept_greedy(const float* p, const int32_t* draft, int3
                                       void* stream);
 
 /*
+ * The KV cache shared by the drafting and the verifying stage.
+ * QSpec page, abstract: the two stages reuse the KV cache as well as the
+ * weights.  The page gives no layout or rule; the ones taken here:
+ *  - one cache per layer, K and V each [batch][h_kv][l_max][head_dim] bf16
+ *    (device, caller-owned), head_dim = 128;
+ *  - `lens` (device int32 [batch]): the number of valid positions of each
+ *    sequence at the start of the round; only qspec_kv_commit changes it;
+ *  - a pass over t_new new tokens per sequence (drafting pass j: t_new = 1,
+ *    offset = j; the verifying pass: t_new = gamma + 1, offset = 0, which
+ *    overwrites the drafted entries with the verifier's) first appends the
+ *    tokens' keys and values at positions lens[b] + offset + t, then runs the
+ *    attention, in which token (b, t) sees positions 0 .. lens[b] + offset + t;
+ *  - after the accept step, qspec_kv_commit advances lens[b] by
+ *    n_accepted[b] + 1 (the accepted drafts plus the verifier's token); the
+ *    entries past it are rolled back simply by being overwritten later.
+ * Token rows come from the fused QKV projection (a GEMM output): row
+ * b * t_new + t of `qkv` (fp32, row stride ld_qkv floats, a multiple of 4,
+ * at least (h_q + 2 h_kv) * 128) holds the h_q query heads, then the h_kv
+ * key heads, then the h_kv value heads, 128 columns each.  Query head h reads
+ * KV head h / (h_q / h_kv); t_new * (h_q / h_kv) must be at most 32.
+ * Asynchronous on `stream`.  Host-side argument errors return
+ * QSPEC_ERR_INVALID_ARG and launch nothing; a position outside the cache
+ * (from the device-side lengths) is skipped and reported as
+ * QSPEC_ERR_BAD_INPUT through qspec_workspace_status on `workspace`
+ * (optional for append and commit: NULL, or >= 256 zeroed bytes).
+ */
+
+/* Writes the t_new new keys and values of every sequence, rounded to bf16
+ * (nearest even), at positions lens[b] + offset + t. */
+qspec_status qspec_kv_append(const float* qkv, int64_t ld_qkv, int32_t batch, int32_t t_new,
+                             int32_t h_q, int32_t h_kv, int32_t head_dim, const int32_t* lens,
+                             int32_t offset, uint16_t* k_cache, uint16_t* v_cache, int32_t l_max,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Decode attention over the shared cache (call after qspec_kv_append of the
+ * same tokens):  out[b*t_new + t][h*128 + i] = sum_j w_j v_j[i],
+ * w = softmax_j(q . k_j / sqrt(128)) over j = 0 .. lens[b] + offset + t, with
+ * q the token's query head h (fp32, as given), k_j, v_j the cached entries of
+ * KV head h / (h_q / h_kv).  Scores, weights and sums in fp32.
+ *  ctx_max    a bound on lens[b] + offset + t_new for every b, at most l_max
+ *             and 32768: it sizes the launch (one CTA per 256 keys); a
+ *             sequence past it gets zero output and QSPEC_ERR_BAD_INPUT.
+ *  out        fp32, row stride ld_out >= h_q * 128.
+ *  workspace  >= qspec_attn_workspace_size(...) bytes, 16-byte aligned, zeroed
+ *             before its first use; every call that completes leaves it ready
+ *             for the next.  Calls sharing one workspace must not overlap.
+ * The result does not depend on the order in which the CTAs finish. */
+qspec_status qspec_attn_decode(const float* qkv, int64_t ld_qkv, int32_t batch, int32_t t_new,
+                               int32_t h_q, int32_t h_kv, int32_t head_dim, const int32_t* lens,
+                               int32_t offset, const uint16_t* k_cache, const uint16_t* v_cache,
+                               int32_t l_max, int32_t ctx_max, float* out, int64_t ld_out,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace qspec_attn_decode needs (0 for invalid arguments). */
+size_t qspec_attn_workspace_size(int32_t batch, int32_t t_new, int32_t h_q, int32_t h_kv,
+                                 int32_t head_dim, int32_t ctx_max);
+
+/* lens[b] += n_accepted[b] + 1 for every sequence (device arrays); a count
+ * that is negative or would pass l_max leaves lens[b] unchanged and is
+ * reported as QSPEC_ERR_BAD_INPUT. */
+qspec_status qspec_kv_commit(int32_t* lens, const int32_t* n_accepted, int32_t batch,
+                             int32_t l_max, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * W4A16 verifying GEMM that allocates nothing and takes no workspace.
  * The pages have no counterpart to this entry point; it exists for callers
  * that cannot allocate device memory at the point of the call: a plugin
@@ -330,8 +394,9 @@ qspec_status qspec_workspace_status(void* workspace, void* stream);
 
 /* Version of this ABI (3: adds QSPEC_GEMM_TEST_STALL, qspec_gemm_w4a8, qspec_cast_bf16,
  * qspec_spec_accept_greedy and qspec_gemm_w4a16_noalloc_status; 4: adds
- * qspec_gemm_w4a4_f32in and qspec_gemm_w4a8_f32in). */
-#define QSPEC_ABI_VERSION 4
+ * qspec_gemm_w4a4_f32in and qspec_gemm_w4a8_f32in; 5: adds qspec_kv_append,
+ * qspec_attn_decode, qspec_attn_workspace_size and qspec_kv_commit). */
+#define QSPEC_ABI_VERSION 5
 int32_t qspec_abi_version(void);
 
 /* Static, human-readable name of a status code. */

@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "accept.cuh"
+#include "attention.cuh"
 #include "gemm.cuh"
 #include "qspec.h"
 #include "quantize.cuh"
@@ -533,6 +534,118 @@ qspec_status qspec_spec_accept_greedy(const float* p, const int32_t* draft, int3
   greedy_accept_kernel<<<batch * kAcceptCluster, kAcceptThreads, 0,
                          static_cast<cudaStream_t>(stream)>>>(
       p, draft, gamma, vocab, chunk, n_accepted, tokens, static_cast<uint32_t*>(workspace));
+  return cudaGetLastError() == cudaSuccess ? QSPEC_OK : QSPEC_ERR_CUDA;
+}
+
+namespace {
+
+// Shape checks shared by the three KV-cache calls (head_dim fixed at 128).
+bool kv_shape_ok(int32_t batch, int32_t t_new, int32_t h_q, int32_t h_kv, int32_t head_dim,
+                 int32_t l_max) {
+  if (batch < 1 || batch > 65535 || t_new < 1 || h_q < 1 || h_kv < 1 || h_kv > 65535) return false;
+  if (head_dim != kHeadDim || (h_q % h_kv) != 0 || l_max < 1) return false;
+  return static_cast<int64_t>(t_new) * (h_q / h_kv) <= kAttnMaxRows;
+}
+
+int32_t attn_chunks(int32_t ctx_max) { return (ctx_max + kAttnChunk - 1) / kAttnChunk; }
+
+}  // namespace
+
+size_t qspec_attn_workspace_size(int32_t batch, int32_t t_new, int32_t h_q, int32_t h_kv,
+                                 int32_t head_dim, int32_t ctx_max) {
+  if (!kv_shape_ok(batch, t_new, h_q, h_kv, head_dim, 1)) return 0;
+  if (ctx_max < 1 || attn_chunks(ctx_max) > kAttnMaxChunks) return 0;
+  const int64_t rows = static_cast<int64_t>(t_new) * (h_q / h_kv);
+  return static_cast<size_t>(attn_layout(batch, h_kv, attn_chunks(ctx_max), rows).total);
+}
+
+qspec_status qspec_kv_append(const float* qkv, int64_t ld_qkv, int32_t batch, int32_t t_new,
+                             int32_t h_q, int32_t h_kv, int32_t head_dim, const int32_t* lens,
+                             int32_t offset, uint16_t* k_cache, uint16_t* v_cache, int32_t l_max,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  if (!qkv || !lens || !k_cache || !v_cache) return QSPEC_ERR_INVALID_ARG;
+  if (!kv_shape_ok(batch, t_new, h_q, h_kv, head_dim, l_max) || offset < 0) return QSPEC_ERR_INVALID_ARG;
+  if (ld_qkv < static_cast<int64_t>(h_q + 2 * h_kv) * kHeadDim || (ld_qkv % 4) != 0)
+    return QSPEC_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(batch) * t_new > 0x7FFFFFFFll) return QSPEC_ERR_INVALID_ARG;
+  if (!aligned(qkv, 16) || !aligned(lens, 4) || !aligned(k_cache, 16) || !aligned(v_cache, 16))
+    return QSPEC_ERR_INVALID_ARG;
+  if (workspace && (workspace_bytes < 256 || !aligned(workspace, 16))) return QSPEC_ERR_INVALID_ARG;
+  qspec_status st = current_device(nullptr, nullptr);
+  if (st != QSPEC_OK) return st;
+  kv_append_kernel<<<static_cast<unsigned>(batch * t_new), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      qkv, ld_qkv, t_new, h_q, h_kv, lens, offset, k_cache, v_cache, l_max,
+      static_cast<uint32_t*>(workspace));
+  return cudaGetLastError() == cudaSuccess ? QSPEC_OK : QSPEC_ERR_CUDA;
+}
+
+qspec_status qspec_attn_decode(const float* qkv, int64_t ld_qkv, int32_t batch, int32_t t_new,
+                               int32_t h_q, int32_t h_kv, int32_t head_dim, const int32_t* lens,
+                               int32_t offset, const uint16_t* k_cache, const uint16_t* v_cache,
+                               int32_t l_max, int32_t ctx_max, float* out, int64_t ld_out,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  if (!qkv || !lens || !k_cache || !v_cache || !out || !workspace) return QSPEC_ERR_INVALID_ARG;
+  if (!kv_shape_ok(batch, t_new, h_q, h_kv, head_dim, l_max) || offset < 0) return QSPEC_ERR_INVALID_ARG;
+  if (ctx_max < 1 || ctx_max > l_max || attn_chunks(ctx_max) > kAttnMaxChunks) return QSPEC_ERR_INVALID_ARG;
+  if (ld_qkv < static_cast<int64_t>(h_q + 2 * h_kv) * kHeadDim || (ld_qkv % 4) != 0 ||
+      ld_out < static_cast<int64_t>(h_q) * kHeadDim)
+    return QSPEC_ERR_INVALID_ARG;
+  if (!aligned(qkv, 16) || !aligned(lens, 4) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(out, 4) || !aligned(workspace, 16))
+    return QSPEC_ERR_INVALID_ARG;
+  const int32_t chunks = attn_chunks(ctx_max);
+  const int32_t rows = t_new * (h_q / h_kv);
+  if (workspace_bytes < static_cast<size_t>(attn_layout(batch, h_kv, chunks, rows).total))
+    return QSPEC_ERR_WORKSPACE_TOO_SMALL;
+  int dev = 0;
+  qspec_status st = current_device(&dev, nullptr);
+  if (st != QSPEC_OK) return st;
+  const size_t smem = static_cast<size_t>(rows) * (kHeadDim + kAttnChunk) * 4 +
+                      (kAttnThreads / 32) * kAttnRowBlock * kHeadDim * 4;
+  static std::atomic<bool> attr_done[kMaxDevices];
+  if (!attr_done[dev].load(std::memory_order_acquire)) {
+    if (cudaFuncSetAttribute(attn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kAttnMaxRows * (kHeadDim + kAttnChunk) * 4 +
+                                              (kAttnThreads / 32) * kAttnRowBlock * kHeadDim * 4)) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return QSPEC_ERR_CUDA;
+    }
+    attr_done[dev].store(true, std::memory_order_release);
+  }
+  AttnArgs a;
+  a.qkv = qkv;
+  a.ld = ld_qkv;
+  a.lens = lens;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.out = out;
+  a.ld_out = ld_out;
+  a.work = static_cast<uint8_t*>(workspace);
+  a.t_new = t_new;
+  a.h_q = h_q;
+  a.h_kv = h_kv;
+  a.offset = offset;
+  a.l_max = l_max;
+  a.ctx_max = ctx_max;
+  a.chunks = chunks;
+  a.rows = rows;
+  attn_decode_kernel<<<dim3(static_cast<unsigned>(chunks), static_cast<unsigned>(h_kv),
+                            static_cast<unsigned>(batch)),
+                       kAttnThreads, smem, static_cast<cudaStream_t>(stream)>>>(a);
+  return cudaGetLastError() == cudaSuccess ? QSPEC_OK : QSPEC_ERR_CUDA;
+}
+
+qspec_status qspec_kv_commit(int32_t* lens, const int32_t* n_accepted, int32_t batch,
+                             int32_t l_max, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!lens || !n_accepted || batch < 1 || l_max < 1) return QSPEC_ERR_INVALID_ARG;
+  if (!aligned(lens, 4) || !aligned(n_accepted, 4)) return QSPEC_ERR_INVALID_ARG;
+  if (workspace && (workspace_bytes < 256 || !aligned(workspace, 16))) return QSPEC_ERR_INVALID_ARG;
+  qspec_status st = current_device(nullptr, nullptr);
+  if (st != QSPEC_OK) return st;
+  kv_commit_kernel<<<static_cast<unsigned>((batch + 127) / 128), 128, 0,
+                     static_cast<cudaStream_t>(stream)>>>(lens, n_accepted, batch, l_max,
+                                                          static_cast<uint32_t*>(workspace));
   return cudaGetLastError() == cudaSuccess ? QSPEC_OK : QSPEC_ERR_CUDA;
 }
 

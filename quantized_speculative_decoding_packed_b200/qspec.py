@@ -27,8 +27,10 @@ EXPORTED = ("qspec_quantize_weights", "qspec_quant_act", "qspec_cast_bf16", "qsp
             "qspec_spec_accept", "qspec_spec_accept_greedy", "qspec_workspace_size",
             "qspec_workspace_status",
             "qspec_status_string", "qspec_gemm_w4a16_noalloc", "qspec_gemm_w4a16_noalloc_status",
+            "qspec_kv_append", "qspec_attn_decode", "qspec_attn_workspace_size", "qspec_kv_commit",
             "qspec_abi_version")
-ABI_VERSION = 4
+ABI_VERSION = 5
+HEAD_DIM = 128           # the KV-cache calls' head dimension
 GEMM_WEIGHTS_READY = 1   # flag: wq/ws are not written by work still in flight
 GEMM_TEST_STALL = 0x100  # test hook: the GEMM's first wait runs out (QSPEC_GEMM_TEST_STALL)
 GEMM_FUSED_QUANT = 0x2   # drafting modes, m <= 32: activations quantized inside the GEMM kernel
@@ -65,13 +67,20 @@ def _load() -> ctypes.CDLL:
     lib.qspec_workspace_size.argtypes = [I32, I64, I64, I64, I32, I32, I32, I32]
     lib.qspec_workspace_size.restype = SZ
     lib.qspec_workspace_status.argtypes = [P, P]
+    lib.qspec_kv_append.argtypes = [P, I64, I32, I32, I32, I32, I32, P, I32, P, P, I32, P, SZ, P]
+    lib.qspec_attn_decode.argtypes = [P, I64, I32, I32, I32, I32, I32, P, I32, P, P, I32, I32, P,
+                                      I64, P, SZ, P]
+    lib.qspec_attn_workspace_size.argtypes = [I32, I32, I32, I32, I32, I32]
+    lib.qspec_attn_workspace_size.restype = SZ
+    lib.qspec_kv_commit.argtypes = [P, P, I32, I32, P, SZ, P]
     lib.qspec_status_string.argtypes = [I32]
     lib.qspec_status_string.restype = ctypes.c_char_p
     for name in ("qspec_quantize_weights", "qspec_quant_act", "qspec_cast_bf16", "qspec_gemm_w4a4",
                  "qspec_gemm_w4a8", "qspec_gemm_w4a4_f32in", "qspec_gemm_w4a8_f32in",
                  "qspec_gemm_w4a16", "qspec_spec_accept", "qspec_spec_accept_greedy",
                  "qspec_workspace_status",
-                 "qspec_gemm_w4a16_noalloc", "qspec_gemm_w4a16_noalloc_status"):
+                 "qspec_gemm_w4a16_noalloc", "qspec_gemm_w4a16_noalloc_status",
+                 "qspec_kv_append", "qspec_attn_decode", "qspec_kv_commit"):
         getattr(lib, name).restype = ctypes.c_int
     if lib.qspec_abi_version() != ABI_VERSION:
         raise ImportError(f"{_LIB_PATH} has ABI version {lib.qspec_abi_version()}, "
@@ -334,3 +343,67 @@ def spec_accept_greedy(p: torch.Tensor, draft: torch.Tensor, n_accepted: torch.T
                                         _ptr(tokens), _ptr(work), nbytes, _stream(stream)),
            "qspec_spec_accept_greedy")
     return n_accepted, tokens
+
+
+# ---------------------------------------------------------------- shared KV cache
+def _kv_cache_check(k_cache: torch.Tensor, v_cache: torch.Tensor):
+    for t, name in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor [B][H_kv][L_max][128]")
+    if k_cache.shape != v_cache.shape or k_cache.shape[3] != HEAD_DIM:
+        raise ValueError("k_cache and v_cache must both be [B][H_kv][L_max][128]")
+    b, h_kv, l_max, _ = k_cache.shape
+    return b, h_kv, l_max
+
+
+def _qkv_check(qkv: torch.Tensor):
+    if not qkv.is_cuda or qkv.dtype != torch.float32 or qkv.dim() != 2 or qkv.stride(1) != 1:
+        raise ValueError("qkv must be a CUDA fp32 [B*T][N] tensor with unit column stride")
+
+
+def attn_workspace_size(batch: int, t_new: int, h_q: int, h_kv: int, ctx_max: int) -> int:
+    return int(LIB.qspec_attn_workspace_size(batch, t_new, h_q, h_kv, HEAD_DIM, ctx_max))
+
+
+def kv_append(qkv: torch.Tensor, lens: torch.Tensor, offset: int, k_cache: torch.Tensor,
+              v_cache: torch.Tensor, h_q: int, work: torch.Tensor | None = None, stream=None):
+    """Write the new tokens' keys and values (rows b*T + t of the fused QKV output)
+    into the caches at positions lens[b] + offset + t."""
+    _qkv_check(qkv)
+    _need(lens, torch.int32, "lens")
+    b, h_kv, l_max = _kv_cache_check(k_cache, v_cache)
+    t_new = qkv.shape[0] // b
+    nbytes = 0 if work is None else work.numel()
+    _check(LIB.qspec_kv_append(_ptr(qkv), qkv.stride(0), b, t_new, h_q, h_kv, HEAD_DIM, _ptr(lens),
+                               offset, _ptr(k_cache), _ptr(v_cache), l_max, _ptr(work), nbytes,
+                               _stream(stream)), "qspec_kv_append")
+
+
+def attn_decode(qkv: torch.Tensor, lens: torch.Tensor, offset: int, k_cache: torch.Tensor,
+                v_cache: torch.Tensor, h_q: int, ctx_max: int, out: torch.Tensor | None = None,
+                work: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Decode attention of the new tokens over the shared cache -> fp32 [B*T][H*128]."""
+    _qkv_check(qkv)
+    _need(lens, torch.int32, "lens")
+    b, h_kv, l_max = _kv_cache_check(k_cache, v_cache)
+    t_new = qkv.shape[0] // b
+    if out is None:
+        out = torch.empty((b * t_new, h_q * HEAD_DIM), dtype=torch.float32, device=qkv.device)
+    if work is None:
+        work = workspace(attn_workspace_size(b, t_new, h_q, h_kv, ctx_max), qkv.device)
+    _check(LIB.qspec_attn_decode(_ptr(qkv), qkv.stride(0), b, t_new, h_q, h_kv, HEAD_DIM,
+                                 _ptr(lens), offset, _ptr(k_cache), _ptr(v_cache), l_max, ctx_max,
+                                 _ptr(out), out.stride(0), _ptr(work), work.numel(),
+                                 _stream(stream)), "qspec_attn_decode")
+    return out
+
+
+def kv_commit(lens: torch.Tensor, n_accepted: torch.Tensor, l_max: int,
+              work: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """lens += n_accepted + 1 on the device (the round's accepted drafts plus one)."""
+    _need(lens, torch.int32, "lens")
+    _need(n_accepted, torch.int32, "n_accepted")
+    nbytes = 0 if work is None else work.numel()
+    _check(LIB.qspec_kv_commit(_ptr(lens), _ptr(n_accepted), lens.numel(), l_max, _ptr(work),
+                               nbytes, _stream(stream)), "qspec_kv_commit")
+    return lens

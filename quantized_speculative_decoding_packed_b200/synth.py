@@ -206,3 +206,35 @@ def greedy_inputs(rng: np.random.Generator, p: np.ndarray, follow: float = 0.8,
     keep = rng.random((bsz, g1 - 1)) < follow
     draft = np.where(keep, planted[:, :g1 - 1], other).astype(np.int32)
     return p, draft
+
+
+# ---------------------------------------------------------------- shared KV cache
+# Decode attention of Llama-2-7B (32 heads, head dim 128, no grouping) and of
+# the grouped Llama-3-8B layout (32 query heads over 8 KV heads): cached keys
+# and values N(0, 1) rounded to bf16, and fused-QKV rows N(0, 1) in fp32 (a
+# projection output).  Positions past each sequence's length hold values too
+# (stale entries of rejected drafts), so a kernel that reads past the causal
+# limit gets a different answer.
+LLAMA2_7B_ATTN = (32, 32)          # (query heads, KV heads)
+LLAMA3_8B_ATTN = (32, 8)
+HEAD_DIM = 128
+
+
+@dataclasses.dataclass
+class KVInputs:
+    k_bits: np.ndarray      # uint16 [B][H_kv][L_max][128]
+    v_bits: np.ndarray
+    lens: np.ndarray        # int32 [B]
+
+
+def kv_cache_inputs(rng: np.random.Generator, batch: int, h_kv: int, l_max: int,
+                    lens) -> KVInputs:
+    shape = (batch, h_kv, l_max, HEAD_DIM)
+    k = to_bf16_bits(rng.standard_normal(shape, dtype=np.float32))
+    v = to_bf16_bits(rng.standard_normal(shape, dtype=np.float32))
+    return KVInputs(k, v, np.asarray(lens, dtype=np.int32))
+
+
+def qkv_rows(rng: np.random.Generator, rows: int, h_q: int, h_kv: int) -> np.ndarray:
+    """fp32 [rows][(h_q + 2 h_kv) * 128]: query heads, key heads, value heads."""
+    return rng.standard_normal((rows, (h_q + 2 * h_kv) * HEAD_DIM), dtype=np.float32)

@@ -30,12 +30,13 @@ def test_header_declares_the_boundary():
                  "qspec_gemm_w4a16", "qspec_spec_accept", "qspec_workspace_size",
                  "qspec_workspace_status", "qspec_status_string", "qspec_abi_version",
                  "qspec_spec_accept_greedy", "qspec_gemm_w4a16_noalloc_status",
-                 "qspec_gemm_w4a4_f32in", "qspec_gemm_w4a8_f32in"):
+                 "qspec_gemm_w4a4_f32in", "qspec_gemm_w4a8_f32in", "qspec_kv_append",
+                 "qspec_attn_decode", "qspec_attn_workspace_size", "qspec_kv_commit"):
         assert name in syms
 
 
 def test_abi_version(lib):
-    assert lib.LIB.qspec_abi_version() == lib.ABI_VERSION == 4
+    assert lib.LIB.qspec_abi_version() == lib.ABI_VERSION == 5
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -137,3 +138,55 @@ def test_stream_k_schedule_invariants(tmp_path):
 def test_greedy_accept_rejects(lib, b, g, v):
     assert lib.LIB.qspec_spec_accept_greedy(FAKE, FAKE, b, g, v, FAKE, FAKE, None, 0, None) == 1
     assert lib.LIB.qspec_spec_accept_greedy(None, FAKE, 2, 4, 32, FAKE, FAKE, None, 0, None) == 1
+
+
+def test_attn_workspace_size_closed_form(lib):
+    # batch 2, 3 new tokens, 4 query heads over 2 KV heads (6 rows per KV head),
+    # context 300 (2 chunks of 256 keys): 256-byte status block, 4 counters,
+    # 2x2x2x6 (max, sum) pairs, 2x2x2x6 rows of 128 floats, each part 256-aligned
+    assert lib.attn_workspace_size(2, 3, 4, 2, 300) == 256 + 256 + 512 + 24576
+    assert lib.attn_workspace_size(2, 3, 4, 2, 32768) > 0
+    assert lib.attn_workspace_size(2, 3, 4, 2, 32769) == 0      # past 128 chunks
+    assert lib.attn_workspace_size(2, 9, 8, 2, 300) == 0        # 36 rows per KV head
+    assert lib.attn_workspace_size(2, 3, 6, 4, 300) == 0        # 6 heads over 4 KV heads
+    assert lib.LIB.qspec_attn_workspace_size(2, 3, 4, 2, 64, 300) == 0   # head_dim 64
+
+
+def _attn(lib, **kw):
+    a = dict(qkv=FAKE, ld=1024, b=2, t=3, hq=4, hkv=2, d=128, lens=FAKE, off=0, kc=FAKE, vc=FAKE,
+             lmax=512, ctx=300, out=FAKE, ldo=512, ws=FAKE, nb=1 << 30)
+    a.update(kw)
+    return lib.LIB.qspec_attn_decode(a["qkv"], a["ld"], a["b"], a["t"], a["hq"], a["hkv"], a["d"],
+                                     a["lens"], a["off"], a["kc"], a["vc"], a["lmax"], a["ctx"],
+                                     a["out"], a["ldo"], a["ws"], a["nb"], None)
+
+
+def test_attn_decode_rejects(lib):
+    odd = ctypes.c_void_p(0x10008)
+    assert _attn(lib, d=64) == 1                     # head_dim other than 128
+    assert _attn(lib, hq=6) == 1                     # query heads not a multiple of KV heads
+    assert _attn(lib, t=9, hq=8) == 1                # 36 rows per KV head
+    assert _attn(lib, ld=1020) == 1                  # row stride below (4 + 2*2) * 128
+    assert _attn(lib, ld=1026) == 1                  # row stride not a multiple of 4
+    assert _attn(lib, ldo=500) == 1                  # output stride below 4 * 128
+    assert _attn(lib, ctx=513) == 1                  # context past the cache
+    assert _attn(lib, ctx=0) == 1
+    assert _attn(lib, off=-1) == 1
+    assert _attn(lib, kc=odd) == 1                   # cache not 16-byte aligned
+    assert _attn(lib, qkv=None) == 1
+    assert _attn(lib, ws=None) == 1
+    assert _attn(lib, nb=1024) == 4                  # workspace too small
+
+
+def test_kv_append_and_commit_reject(lib):
+    f = lib.LIB.qspec_kv_append
+    ok = [FAKE, 1024, 2, 3, 4, 2, 128, FAKE, 0, FAKE, FAKE, 512, None, 0, None]
+    bad = [(6, 64), (4, 6), (1, 1020), (8, -1), (11, 0), (0, None), (9, ctypes.c_void_p(0x10008))]
+    for i, v in bad:
+        args = list(ok)
+        args[i] = v
+        assert f(*args) == 1, (i, v)
+    assert f(*(ok[:12] + [FAKE, 64, None])) == 1       # a workspace below 256 bytes
+    assert lib.LIB.qspec_kv_commit(FAKE, FAKE, 0, 512, None, 0, None) == 1
+    assert lib.LIB.qspec_kv_commit(None, FAKE, 2, 512, None, 0, None) == 1
+    assert lib.LIB.qspec_kv_commit(FAKE, FAKE, 2, 0, None, 0, None) == 1
