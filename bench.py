@@ -63,6 +63,11 @@ def parse():
                     help="skip the chained-round report (layers fed by the previous layer)")
     ap.add_argument("--no-draft-variants", action="store_true",
                     help="skip the W4A4 / W4A8 drafting-variant report")
+    ap.add_argument("--no-attention", action="store_true",
+                    help="skip the shared-KV-cache decode attention report")
+    ap.add_argument("--profile-attn", metavar="T", type=int, default=None,
+                    help="profiling driver: three decode-attention calls over one Llama-2-7B "
+                         "layer's cache (batch 16, context 1024) with T new tokens, then exit")
     ap.add_argument("--profile-accept", metavar="RULE", default=None,
                     help="profiling driver: three calls of the accept step (RULE sampling|greedy) "
                          "at vocab 128256, batch 64, gamma 5, sigma 0.5, then exit")
@@ -101,6 +106,90 @@ def profile_gemm(spec):
         torch.cuda.synchronize()
         print(f"{mode} {shape}: y[{m}][{n}] sum |y| = {float(y.abs().sum()):.6g}")
         del wq, ws, x, y
+
+
+ATTN_BATCH, ATTN_CTX, ATTN_HEADS = 16, 1024, (32, 32)   # Llama-2-7B: 32 query heads, 32 KV heads
+
+
+def attn_bytes(lens, offset, t_new, h_q, h_kv):
+    """Compulsory HBM bytes of one decode-attention call: every visible key and value
+    (bf16) once, the query rows read (fp32) and the outputs written (fp32)."""
+    kv = sum(int(n) + offset + t_new for n in lens) * h_kv * 128 * 2 * 2
+    return kv + 2 * len(lens) * t_new * h_q * 128 * 4
+
+
+def append_bytes(batch, t_new, h_kv):
+    """The new keys and values: read in fp32 from the QKV rows, written in bf16."""
+    return batch * t_new * 2 * h_kv * 128 * (4 + 2)
+
+
+def _attn_setup(torch, qspec, layers, t_max, heads=ATTN_HEADS, batch=ATTN_BATCH, ctx=ATTN_CTX,
+                stream_id=0):
+    from quantized_speculative_decoding_packed_b200 import synth
+    h_q, h_kv = heads
+    l_max = ctx + t_max + 8
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(rank_seed(0) + 31 + stream_id)
+    caches = []
+    for _ in range(layers):
+        kc = torch.randn((batch, h_kv, l_max, 128), generator=gen, device="cuda").to(torch.bfloat16)
+        vc = torch.randn((batch, h_kv, l_max, 128), generator=gen, device="cuda").to(torch.bfloat16)
+        caches.append((kc, vc))
+    lens = torch.full((batch,), ctx, dtype=torch.int32, device="cuda")
+    qkv = torch.randn((batch * t_max, (h_q + 2 * h_kv) * 128), generator=gen, device="cuda")
+    return caches, lens, qkv, l_max
+
+
+def profile_attn(t_new):
+    """Three decode-attention calls over one layer's cache, for a profiler to capture one."""
+    import torch
+    from quantized_speculative_decoding_packed_b200 import qspec
+    caches, lens, qkv, l_max = _attn_setup(torch, qspec, 1, t_new)
+    h_q, h_kv = ATTN_HEADS
+    kc, vc = caches[0]
+    x = qkv[: ATTN_BATCH * t_new]
+    ctx = ATTN_CTX + t_new
+    for _ in range(3):
+        out = qspec.attn_decode(x, lens, 0, kc, vc, h_q, ctx)
+    torch.cuda.synchronize()
+    print(f"attention T={t_new}: sum |out| = {float(out.abs().sum()):.6g}")
+
+
+def attention_report(torch, qspec, hbm):
+    """Decode attention over the shared KV cache (Llama-2-7B: 32 heads of 128, batch 16,
+    context 1024 at the start of the round), per layer: a drafting pass (append + attention
+    of 1 token at offset 0) and the verifying pass (5 tokens); plus the grouped Llama-3-8B
+    layout (32 query heads over 8 KV heads) for the verifying pass.  Device time per call in
+    a CUDA graph over 4 layers' caches (1.1 GB, past L2), median of 5 replays."""
+    out = {"workload": "shared KV cache, batch 16, head dim 128, context 1024 before the round",
+           "timing": "CUDA graph of calls over 4 layers' caches (past L2), median of 5 replays",
+           "peak_hbm_gbs": hbm}
+    for name, heads, passes in (("llama2_7b", ATTN_HEADS, ((1, "draft"), (5, "verify"))),
+                                ("llama3_8b_gqa", (32, 8), ((5, "verify"),))):
+        h_q, h_kv = heads
+        caches, lens, qkv, l_max = _attn_setup(torch, qspec, 4, 5, heads)
+        lens_h = [ATTN_CTX] * ATTN_BATCH
+        for t_new, label in passes:
+            x = qkv[: ATTN_BATCH * t_new]
+            ctx = ATTN_CTX + t_new
+            o = torch.empty((ATTN_BATCH * t_new, h_q * 128), dtype=torch.float32, device="cuda")
+            work = torch.zeros(qspec.attn_workspace_size(ATTN_BATCH, t_new, h_q, h_kv, ctx),
+                               dtype=torch.uint8, device="cuda")
+            att = [(lambda c=c: qspec.attn_decode(x, lens, 0, c[0], c[1], h_q, ctx, out=o,
+                                                  work=work)) for c in caches] * 2
+            app = [(lambda c=c: qspec.kv_append(x, lens, 0, c[0], c[1], h_q)) for c in caches] * 2
+            t_att = _graph_time_per_call(torch, att)
+            t_app = _graph_time_per_call(torch, app)
+            b_att = attn_bytes(lens_h, 0, t_new, h_q, h_kv)
+            b_app = append_bytes(ATTN_BATCH, t_new, h_kv)
+            out[f"{name}_{label}_t{t_new}"] = {
+                "h_q": h_q, "h_kv": h_kv, "t_new": t_new,
+                "attn_us": t_att * 1e6, "attn_gbs": b_att / t_att / 1e9,
+                "attn_frac_hbm": b_att / t_att / 1e9 / hbm, "attn_bytes": b_att,
+                "append_us": t_app * 1e6, "append_gbs": b_app / t_app / 1e9}
+        del caches
+        torch.cuda.empty_cache()
+    return out
 
 
 def profile_accept(rule, batch=64, gamma=5, vocab=128256, sigma=0.5):
@@ -382,6 +471,9 @@ def workload_config(layers):
 # ---------------------------------------------------------------- GPU arm
 def main():
     args = parse()
+    if args.profile_attn:
+        profile_attn(args.profile_attn)
+        return
     if args.profile_gemm:
         profile_gemm(args.profile_gemm)
         return
@@ -605,6 +697,9 @@ def main():
     variants = None
     if rank == 0 and world == 1 and not args.no_draft_variants:
         variants = draft_variants_report(torch, qspec, peaks)
+    attn = None
+    if rank == 0 and world == 1 and not args.no_attention:
+        attn = attention_report(torch, qspec, hbm_peak)
     fused_ab = None
     if rank == 0 and world == 1 and not args.no_chained:
         fused_ab = fused_quant_report(torch, qspec, wq, ws, L, x16)
@@ -625,7 +720,7 @@ def main():
                 "clocks": clk.summary(), "kernels": kern, "decode_shapes": shapes_rep,
                 "large_m": large,
                 "m_sweep": sweep, "accept_large_vocab": acc_rep, "round_chained": chained,
-                "draft_variants": variants,
+                "draft_variants": variants, "attention": attn,
                 "fused_quant_ab": fused_ab}
         print(json.dumps(line))
     if world > 1:

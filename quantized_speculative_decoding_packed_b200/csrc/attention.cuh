@@ -14,15 +14,15 @@
 // (rejected drafts) are overwritten by the next round.
 //
 // Layout on B200 (decode attention is HBM-bound: every key and value is
-// read once per pass): one CTA per (sequence, KV head, chunk of 256 keys),
-// so the cache streams through all SMs whatever the batch.  In a CTA each
-// lane owns one key for the scores (its 256-byte row in registers, the
-// queries broadcast from shared memory), the softmax of the chunk is exact
-// (its own maximum), and for the values the lanes span the head dimension
-// (4 columns each, a warp per 64 keys).  Each CTA leaves its (max, sum,
-// weighted values) per query row in the workspace; the last CTA of a
-// (sequence, KV head) to arrive merges the chunks in chunk order, so the
-// result does not depend on which CTA finishes last.
+// read once per pass): one CTA per (sequence, KV head, chunk of 128 keys),
+// so the cache streams through all SMs whatever the batch.  A CTA copies its
+// chunk's keys and values (32 KB each, contiguous) into shared memory with
+// two TMA bulk copies; each lane then owns one key for the scores, the
+// softmax of the chunk is exact (its own maximum), and for the values each
+// lane owns one column of the head.  Each CTA leaves its (max, sum, weighted
+// values) per query row in the workspace; the last CTA of a (sequence, KV
+// head) to arrive merges the chunks in chunk order, so the result does not
+// depend on which CTA finishes last.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -33,11 +33,11 @@
 namespace qspec {
 
 constexpr int kHeadDim = 128;
-constexpr int kAttnChunk = 256;              // keys per CTA
+constexpr int kAttnChunk = 128;              // keys per CTA
 constexpr int kAttnThreads = 128;            // 4 warps
 constexpr int kAttnMaxRows = 32;             // (query heads per KV head) x new tokens
 constexpr int kAttnRowBlock = 8;             // query rows per register block
-constexpr int kAttnMaxChunks = 128;          // context up to 32768 keys
+constexpr int kAttnMaxChunks = 256;          // context up to 32768 keys
 constexpr float kInvSqrtHeadDim = 0.08838834764831845f;   // 1 / sqrt(128)
 
 // Workspace of the attention call: status word, then one arrival counter per
@@ -119,15 +119,24 @@ struct AttnArgs {
   int t_new, h_q, h_kv, offset, l_max, ctx_max, chunks, rows;
 };
 
-// grid (chunks, h_kv, batch), kAttnThreads threads; dynamic shared memory:
-// queries [rows][128] + weights [rows][256] + merge [4][8][128] floats.
+// Dynamic shared memory of one CTA: the chunk's keys and values (bf16,
+// [kAttnChunk][128] each, copied by TMA), the queries [rows][128] and the
+// weights [rows][kAttnChunk] in fp32.
+__host__ __device__ inline int64_t attn_smem_bytes(int rows) {
+  return 2ll * kAttnChunk * kHeadDim * 2 + static_cast<int64_t>(rows) * (kHeadDim + kAttnChunk) * 4;
+}
+
+// grid (chunks, h_kv, batch), kAttnThreads threads.
 __global__ void __launch_bounds__(kAttnThreads, 4) attn_decode_kernel(const AttnArgs a) {
-  extern __shared__ float4 attn_smem4[];
-  float* const q_s = reinterpret_cast<float*>(attn_smem4);          // [rows][128]
-  float* const p_s = q_s + a.rows * kHeadDim;                       // [rows][256]
-  float* const red = p_s + a.rows * kAttnChunk;                     // [4][8][128]
+  extern __shared__ __align__(128) uint8_t attn_smem[];
+  uint16_t* const k_s = reinterpret_cast<uint16_t*>(attn_smem);                  // [chunk][128]
+  uint16_t* const v_s = k_s + kAttnChunk * kHeadDim;                              // [chunk][128]
+  float* const q_s = reinterpret_cast<float*>(v_s + kAttnChunk * kHeadDim);       // [rows][128]
+  float* const p_s = q_s + a.rows * kHeadDim;                                     // [rows][chunk]
+  __shared__ __align__(8) uint64_t kv_bar;
   __shared__ float row_m[kAttnMaxRows], row_l[kAttnMaxRows];
   __shared__ int is_last;
+  __shared__ int abort_flag;
 
   const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -150,7 +159,29 @@ __global__ void __launch_bounds__(kAttnThreads, 4) attn_decode_kernel(const Attn
   // row r = t * group + hh: token t, query head g * group + hh
   auto row_limit = [&](int r) { return len + a.offset + r / group; };   // last visible key
 
-  // queries of this KV head's rows into shared memory
+  const uint16_t* const kc = a.k_cache + ((static_cast<int64_t>(b) * a.h_kv + g) * a.l_max + k0) * kHeadDim;
+  const uint16_t* const vc = a.v_cache + ((static_cast<int64_t>(b) * a.h_kv + g) * a.l_max + k0) * kHeadDim;
+  const uint32_t bar = static_cast<uint32_t>(__cvta_generic_to_shared(&kv_bar));
+  // The chunk's keys and values are contiguous rows of 256 bytes: one bulk
+  // copy each into shared memory, completing on one transaction barrier.
+  if (tid == 0) {
+    abort_flag = 0;
+    mbar_init(bar, 1);
+    fence_barrier_init();
+    if (n_keys > 0) {
+      const uint32_t bytes = static_cast<uint32_t>(n_keys) * kHeadDim * 2;
+      mbar_arrive_expect_tx(bar, 2 * bytes);
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+          ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(k_s))), "l"(kc), "r"(bytes), "r"(bar)
+          : "memory");
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+          ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(v_s))), "l"(vc), "r"(bytes), "r"(bar)
+          : "memory");
+    }
+  }
+  // queries of this KV head's rows into shared memory meanwhile
   for (int e = tid * 4; e < rows * kHeadDim; e += kAttnThreads * 4) {
     const int r = e / kHeadDim, i = e % kHeadDim;
     const int t = r / group, h = g * group + r % group;
@@ -159,34 +190,37 @@ __global__ void __launch_bounds__(kAttnThreads, 4) attn_decode_kernel(const Attn
     *reinterpret_cast<float4*>(q_s + e) = v;
   }
   __syncthreads();
+  const bool ok = __syncthreads_and(n_keys == 0 || mbar_wait(bar, 0, &abort_flag, status));
+  if (!ok && tid == 0) {
+    // the copies did not land in time (reported): let them finish before
+    // the shared memory is released, and leave an empty partial
+    mbar_wait_drain(bar, 0);
+  }
+  const int n_live = ok ? n_keys : 0;
 
-  const uint16_t* const kc = a.k_cache + (static_cast<int64_t>(b) * a.h_kv + g) * a.l_max * kHeadDim;
-  const uint16_t* const vc = a.v_cache + (static_cast<int64_t>(b) * a.h_kv + g) * a.l_max * kHeadDim;
-
-  // ---- scores: lane = key (two keys of 32 per warp pass, 64 per warp)
-  for (int pass = 0; pass < 2; ++pass) {
-    const int jl = warp * 64 + pass * 32 + lane;                    // key within the chunk
-    const bool have = jl < n_keys;
-    uint4 kr[kHeadDim / 8];
-    if (have) {
-      const uint4* src = reinterpret_cast<const uint4*>(kc + (k0 + jl) * kHeadDim);
-#pragma unroll
-      for (int c = 0; c < kHeadDim / 8; ++c) kr[c] = __ldcs(src + c);
-    }
+  // ---- scores: lane = key.  Lane l reads its row's 16-byte pieces in the
+  // order (c + l) mod 16, so the 8 lanes of a quarter warp hit 8 different
+  // bank groups; the queries are read at the same pieces.
+  {
+    const int jl = warp * 32 + lane;
+    const bool have = jl < n_live;
+    const uint4* krow = reinterpret_cast<const uint4*>(k_s + jl * kHeadDim);
     for (int r0 = 0; r0 < rows; r0 += kAttnRowBlock) {
       float acc[kAttnRowBlock];
 #pragma unroll
       for (int rr = 0; rr < kAttnRowBlock; ++rr) acc[rr] = 0.f;
       if (have) {
-#pragma unroll
+#pragma unroll 4
         for (int c = 0; c < kHeadDim / 8; ++c) {
-          const float kf[8] = {bf16_lo(kr[c].x), bf16_hi(kr[c].x), bf16_lo(kr[c].y), bf16_hi(kr[c].y),
-                               bf16_lo(kr[c].z), bf16_hi(kr[c].z), bf16_lo(kr[c].w), bf16_hi(kr[c].w)};
+          const int cc = (c + lane) & (kHeadDim / 8 - 1);
+          const uint4 kw = krow[cc];
+          const float kf[8] = {bf16_lo(kw.x), bf16_hi(kw.x), bf16_lo(kw.y), bf16_hi(kw.y),
+                               bf16_lo(kw.z), bf16_hi(kw.z), bf16_lo(kw.w), bf16_hi(kw.w)};
 #pragma unroll
           for (int rr = 0; rr < kAttnRowBlock; ++rr) {
             if (r0 + rr < rows) {
-              const float4 qa = *reinterpret_cast<const float4*>(q_s + (r0 + rr) * kHeadDim + c * 8);
-              const float4 qb = *reinterpret_cast<const float4*>(q_s + (r0 + rr) * kHeadDim + c * 8 + 4);
+              const float4 qa = *reinterpret_cast<const float4*>(q_s + (r0 + rr) * kHeadDim + cc * 8);
+              const float4 qb = *reinterpret_cast<const float4*>(q_s + (r0 + rr) * kHeadDim + cc * 8 + 4);
               acc[rr] = fmaf(qa.x, kf[0], acc[rr]);
               acc[rr] = fmaf(qa.y, kf[1], acc[rr]);
               acc[rr] = fmaf(qa.z, kf[2], acc[rr]);
@@ -233,47 +267,46 @@ __global__ void __launch_bounds__(kAttnThreads, 4) attn_decode_kernel(const Attn
   }
   __syncthreads();
 
-  // ---- weighted values: a warp per 64 keys, lanes over the head dimension
+  // ---- weighted values: warp w owns head columns 32w .. 32w+31 (lane = one
+  // column) over all the chunk's keys, so no cross-warp sum is needed
   const int64_t part = (static_cast<int64_t>(b) * a.h_kv + g) * a.chunks + chunk;
   float* const part_o = reinterpret_cast<float*>(a.work + lay.off_o) + part * rows * kHeadDim;
   float* const part_ml = reinterpret_cast<float*>(a.work + lay.off_ml) + part * rows * 2;
-  const int j_lo = warp * 64;
-  const int j_hi = min(j_lo + 64, n_keys);
+  const int d = warp * 32 + lane;
   for (int r0 = 0; r0 < rows; r0 += kAttnRowBlock) {
-    float o[kAttnRowBlock][4];
+    float o[kAttnRowBlock];
 #pragma unroll
-    for (int rr = 0; rr < kAttnRowBlock; ++rr)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) o[rr][i] = 0.f;
-    for (int j = j_lo; j < j_hi; ++j) {
-      const uint2 vr = __ldcs(reinterpret_cast<const uint2*>(vc + (k0 + j) * kHeadDim + lane * 4));
-      const float vf[4] = {bf16_lo(vr.x), bf16_hi(vr.x), bf16_lo(vr.y), bf16_hi(vr.y)};
+    for (int rr = 0; rr < kAttnRowBlock; ++rr) o[rr] = 0.f;
+    const int n4 = n_live & ~3;
+    for (int j = 0; j < n4; j += 4) {
+      const float v0 = __uint_as_float(static_cast<uint32_t>(v_s[(j + 0) * kHeadDim + d]) << 16);
+      const float v1 = __uint_as_float(static_cast<uint32_t>(v_s[(j + 1) * kHeadDim + d]) << 16);
+      const float v2 = __uint_as_float(static_cast<uint32_t>(v_s[(j + 2) * kHeadDim + d]) << 16);
+      const float v3 = __uint_as_float(static_cast<uint32_t>(v_s[(j + 3) * kHeadDim + d]) << 16);
 #pragma unroll
       for (int rr = 0; rr < kAttnRowBlock; ++rr) {
         if (r0 + rr < rows) {
-          const float p = p_s[(r0 + rr) * kAttnChunk + j];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) o[rr][i] = fmaf(p, vf[i], o[rr][i]);
+          const float4 p = *reinterpret_cast<const float4*>(p_s + (r0 + rr) * kAttnChunk + j);
+          o[rr] = fmaf(p.x, v0, o[rr]);
+          o[rr] = fmaf(p.y, v1, o[rr]);
+          o[rr] = fmaf(p.z, v2, o[rr]);
+          o[rr] = fmaf(p.w, v3, o[rr]);
         }
       }
     }
+    for (int j = n4; j < n_live; ++j) {
+      const float v = __uint_as_float(static_cast<uint32_t>(v_s[j * kHeadDim + d]) << 16);
+#pragma unroll
+      for (int rr = 0; rr < kAttnRowBlock; ++rr)
+        if (r0 + rr < rows) o[rr] = fmaf(p_s[(r0 + rr) * kAttnChunk + j], v, o[rr]);
+    }
 #pragma unroll
     for (int rr = 0; rr < kAttnRowBlock; ++rr)
-      *reinterpret_cast<float4*>(red + (warp * kAttnRowBlock + rr) * kHeadDim + lane * 4) =
-          make_float4(o[rr][0], o[rr][1], o[rr][2], o[rr][3]);
-    __syncthreads();
-    // the four warps' sums in warp order; thread = column of the head
-    for (int rr = 0; rr < kAttnRowBlock && r0 + rr < rows; ++rr) {
-      float s = 0.f;
-#pragma unroll
-      for (int w = 0; w < kAttnThreads / 32; ++w) s += red[(w * kAttnRowBlock + rr) * kHeadDim + tid];
-      part_o[(r0 + rr) * kHeadDim + tid] = s;
-    }
-    __syncthreads();
+      if (r0 + rr < rows) part_o[(r0 + rr) * kHeadDim + d] = o[rr];
   }
   if (tid < rows) {
-    part_ml[tid * 2] = row_m[tid];
-    part_ml[tid * 2 + 1] = row_l[tid];
+    part_ml[tid * 2] = ok ? row_m[tid] : -INFINITY;
+    part_ml[tid * 2 + 1] = ok ? row_l[tid] : 0.f;
   }
 
   // ---- the last chunk of this (sequence, KV head) to arrive merges all chunks

@@ -600,13 +600,11 @@ qspec_status qspec_attn_decode(const float* qkv, int64_t ld_qkv, int32_t batch, 
   int dev = 0;
   qspec_status st = current_device(&dev, nullptr);
   if (st != QSPEC_OK) return st;
-  const size_t smem = static_cast<size_t>(rows) * (kHeadDim + kAttnChunk) * 4 +
-                      (kAttnThreads / 32) * kAttnRowBlock * kHeadDim * 4;
+  const size_t smem = static_cast<size_t>(attn_smem_bytes(rows));
   static std::atomic<bool> attr_done[kMaxDevices];
   if (!attr_done[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(attn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kAttnMaxRows * (kHeadDim + kAttnChunk) * 4 +
-                                              (kAttnThreads / 32) * kAttnRowBlock * kHeadDim * 4)) !=
+                             static_cast<int>(attn_smem_bytes(kAttnMaxRows))) !=
         cudaSuccess) {
       cudaGetLastError();
       return QSPEC_ERR_CUDA;

@@ -67,3 +67,13 @@ def test_job_throughput_is_whole_job():
     one = bench.job_throughput(1e9, 1, 10.0)
     assert one == pytest.approx(100.0)                  # 1 GB in 10 ms = 100 GB/s
     assert bench.job_throughput(1e9, 8, 10.0) == pytest.approx(8 * one)
+
+
+def test_attention_bytes_closed_forms():
+    import bench
+    # batch 16 at length 1024, one new token, 32 heads of 128 (no grouping): 1025
+    # keys and values of 256 bytes per head and sequence, plus fp32 query and output rows
+    assert bench.attn_bytes([1024] * 16, 0, 1, 32, 32) == 16 * 1025 * 32 * 512 + 2 * 16 * 32 * 512
+    # grouped: 8 KV heads serve 32 query heads; 5 new tokens at offset 2
+    assert bench.attn_bytes([100, 200], 2, 5, 32, 8) == (107 + 207) * 8 * 512 + 2 * 2 * 5 * 32 * 512
+    assert bench.append_bytes(16, 5, 32) == 16 * 5 * 2 * 32 * 128 * 6

@@ -51,12 +51,14 @@ def _pass(qs, rng, kv, kc, vc, lens_d, offset, t_new, h_q, h_kv, l_max, ctx_max,
     qkv = synth.qkv_rows(rng, b * t_new, h_q, h_kv)
     qkv_d = cuda_f32(qkv)
     qs.kv_append(qkv_d, lens_d, offset, kc, vc, h_q, work=work)
-    out = qs.attn_decode(qkv_d, lens_d, offset, kc, vc, h_q, ctx_max)
+    aw = torch.zeros(qs.attn_workspace_size(b, t_new, h_q, h_kv, ctx_max), dtype=torch.uint8,
+                     device="cuda")
+    out = qs.attn_decode(qkv_d, lens_d, offset, kc, vc, h_q, ctx_max, work=aw)
     ref_k, ref_v = orc.kv_append(_f32(kv.k_bits), _f32(kv.v_bits), qkv, kv.lens, offset, t_new,
                                  h_q, h_kv, D)
     ref = orc.decode_attention(qkv, ref_k, ref_v, kv.lens, offset, t_new, h_q, h_kv, D)
     torch.cuda.synchronize()
-    assert qs.workspace_status(work) == 0
+    assert qs.workspace_status(work) == 0 and qs.workspace_status(aw) == 0
     got_k, got_v = _bits(kc), _bits(vc)
     assert np.array_equal(got_k, synth.to_bf16_bits(ref_k)), "key cache"
     assert np.array_equal(got_v, synth.to_bf16_bits(ref_v)), "value cache"
@@ -79,7 +81,7 @@ def test_append_and_attention_match_oracle(qs, b, t_new, h_q, h_kv, lens, offset
     kv = synth.kv_cache_inputs(rng, b, h_kv, l_max, lens)
     kc, vc = cuda_bf16(kv.k_bits), cuda_bf16(kv.v_bits)
     lens_d = cuda_i32(kv.lens)
-    work = qs.workspace(256)
+    work = torch.zeros(256, dtype=torch.uint8, device="cuda")
     _pass(qs, rng, kv, kc, vc, lens_d, offset, t_new, h_q, h_kv, l_max, ctx_max, work)
 
 
@@ -92,7 +94,7 @@ def test_draft_verify_commit_round_on_one_cache(qs):
     kv = synth.kv_cache_inputs(rng, b, h_kv, l_max, (3, 250, 511, 900))
     kc, vc = cuda_bf16(kv.k_bits), cuda_bf16(kv.v_bits)
     lens_d = cuda_i32(kv.lens)
-    work = qs.workspace(256)
+    work = torch.zeros(256, dtype=torch.uint8, device="cuda")
     for rnd, n_acc in enumerate(((0, 4, 2, 1), (3, 0, 4, 2))):
         ctx = int(kv.lens.max()) + gamma + 1
         for j in range(gamma):
@@ -115,7 +117,7 @@ def test_llama2_7b_decode_full_size(qs):
     kv = synth.kv_cache_inputs(rng, b, h_kv, l_max, lens)
     kc, vc = cuda_bf16(kv.k_bits), cuda_bf16(kv.v_bits)
     lens_d = cuda_i32(kv.lens)
-    work = qs.workspace(256)
+    work = torch.zeros(256, dtype=torch.uint8, device="cuda")
     ctx = int(kv.lens.max()) + gamma + 1
     _pass(qs, rng, kv, kc, vc, lens_d, 0, 1, h_q, h_kv, l_max, ctx, work)
     _pass(qs, rng, kv, kc, vc, lens_d, 0, gamma + 1, h_q, h_kv, l_max, ctx, work)
@@ -129,7 +131,7 @@ def test_grouped_llama3_8b_verify_full_size(qs):
     kv = synth.kv_cache_inputs(rng, b, h_kv, l_max, lens)
     kc, vc = cuda_bf16(kv.k_bits), cuda_bf16(kv.v_bits)
     lens_d = cuda_i32(kv.lens)
-    work = qs.workspace(256)
+    work = torch.zeros(256, dtype=torch.uint8, device="cuda")
     _pass(qs, rng, kv, kc, vc, lens_d, 0, gamma + 1, h_q, h_kv, l_max, int(kv.lens.max()) + gamma + 1,
           work)
 

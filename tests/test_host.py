@@ -142,11 +142,11 @@ def test_greedy_accept_rejects(lib, b, g, v):
 
 def test_attn_workspace_size_closed_form(lib):
     # batch 2, 3 new tokens, 4 query heads over 2 KV heads (6 rows per KV head),
-    # context 300 (2 chunks of 256 keys): 256-byte status block, 4 counters,
-    # 2x2x2x6 (max, sum) pairs, 2x2x2x6 rows of 128 floats, each part 256-aligned
-    assert lib.attn_workspace_size(2, 3, 4, 2, 300) == 256 + 256 + 512 + 24576
+    # context 300 (3 chunks of 128 keys): 256-byte status block, 4 counters,
+    # 2x2x3x6 (max, sum) pairs, 2x2x3x6 rows of 128 floats, each part 256-aligned
+    assert lib.attn_workspace_size(2, 3, 4, 2, 300) == 256 + 256 + 768 + 36864
     assert lib.attn_workspace_size(2, 3, 4, 2, 32768) > 0
-    assert lib.attn_workspace_size(2, 3, 4, 2, 32769) == 0      # past 128 chunks
+    assert lib.attn_workspace_size(2, 3, 4, 2, 32769) == 0      # past 256 chunks
     assert lib.attn_workspace_size(2, 9, 8, 2, 300) == 0        # 36 rows per KV head
     assert lib.attn_workspace_size(2, 3, 6, 4, 300) == 0        # 6 heads over 4 KV heads
     assert lib.LIB.qspec_attn_workspace_size(2, 3, 4, 2, 64, 300) == 0   # head_dim 64
