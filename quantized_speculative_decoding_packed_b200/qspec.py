@@ -361,6 +361,12 @@ def _qkv_check(qkv: torch.Tensor):
         raise ValueError("qkv must be a CUDA fp32 [B*T][N] tensor with unit column stride")
 
 
+def _tokens_per_sequence(qkv: torch.Tensor, batch: int) -> int:
+    if qkv.shape[0] % batch != 0 or qkv.shape[0] == 0:
+        raise ValueError(f"qkv has {qkv.shape[0]} rows, not a positive multiple of the batch {batch}")
+    return qkv.shape[0] // batch
+
+
 def attn_workspace_size(batch: int, t_new: int, h_q: int, h_kv: int, ctx_max: int) -> int:
     return int(LIB.qspec_attn_workspace_size(batch, t_new, h_q, h_kv, HEAD_DIM, ctx_max))
 
@@ -372,7 +378,7 @@ def kv_append(qkv: torch.Tensor, lens: torch.Tensor, offset: int, k_cache: torch
     _qkv_check(qkv)
     _need(lens, torch.int32, "lens")
     b, h_kv, l_max = _kv_cache_check(k_cache, v_cache)
-    t_new = qkv.shape[0] // b
+    t_new = _tokens_per_sequence(qkv, b)
     nbytes = 0 if work is None else work.numel()
     _check(LIB.qspec_kv_append(_ptr(qkv), qkv.stride(0), b, t_new, h_q, h_kv, HEAD_DIM, _ptr(lens),
                                offset, _ptr(k_cache), _ptr(v_cache), l_max, _ptr(work), nbytes,
@@ -386,7 +392,7 @@ def attn_decode(qkv: torch.Tensor, lens: torch.Tensor, offset: int, k_cache: tor
     _qkv_check(qkv)
     _need(lens, torch.int32, "lens")
     b, h_kv, l_max = _kv_cache_check(k_cache, v_cache)
-    t_new = qkv.shape[0] // b
+    t_new = _tokens_per_sequence(qkv, b)
     if out is None:
         out = torch.empty((b * t_new, h_q * HEAD_DIM), dtype=torch.float32, device=qkv.device)
     if work is None:
