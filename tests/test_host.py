@@ -190,3 +190,16 @@ def test_kv_append_and_commit_reject(lib):
     assert lib.LIB.qspec_kv_commit(FAKE, FAKE, 0, 512, None, 0, None) == 1
     assert lib.LIB.qspec_kv_commit(None, FAKE, 2, 512, None, 0, None) == 1
     assert lib.LIB.qspec_kv_commit(FAKE, FAKE, 2, 0, None, 0, None) == 1
+
+
+def test_kv_binding_checks_its_tensors(lib):
+    import torch
+    qkv = torch.zeros((4, 8 * 128))
+    lens = torch.zeros(2, dtype=torch.int32)
+    cache = torch.zeros((2, 2, 16, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="qkv"):
+        lib.attn_decode(qkv, lens, 0, cache, cache, 4, 16)          # host tensors
+    with pytest.raises(ValueError, match="qkv"):
+        lib.kv_append(qkv.half(), lens, 0, cache, cache, 4)
+    with pytest.raises(ValueError):
+        lib.kv_commit(lens, lens.long(), 16)
